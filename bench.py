@@ -1,0 +1,492 @@
+"""Benchmark: paged decode attention on B200, KV-read GB/s per decode step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--partition-size P] [--engine auto|core|mma]
+
+A step is one decode step of the workload's batch: copy-on-write block
+copies (when the host manager reports any), the cache write of the step's new
+tokens, and decode attention over every sequence.  The host metadata of every
+step (slot mapping, copy pairs, block tables, lengths) is produced by the
+library's C++ manager before the timed region and sits in HBM with the
+queries and new K/V rows, so the timed region holds only the library's
+kernels.  Timing: CUDA events on the launching stream around K consecutive
+steps after W warm-up steps, synchronised on both sides; every step is a new
+token of the same sequences (the KV cache, 0.6-2.7 GB, is larger than the
+126 MB L2, so no flush is needed).
+
+value = algorithmic bytes of the K steps / timed span, algorithmic bytes per
+step = sum_s L_s * Hkv * D * 2 * e (K and V) + 2 * S * Hq * D * e (q, out)
++ sum_s ceil(L_s / bs) * 4 (block-table entries).
+
+e2e = the same metric through the public API with host buffers: the C++
+manager appends the step's tokens live, pinned host buffers are copied to the
+device, the kernels run and the output comes back to the host, every step.
+
+Multi-GPU: independent replicas (the decode path has no exchange step); each
+rank runs its own copy of the batch; value = bytes of all ranks / max-over-
+ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention: KV-read GB/s (% of B200 HBM peak) and seqs/s per step"
+DEFAULT_WORKLOAD = "mha7b_f16"
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def algorithmic_bytes(lens, hq, hkv, d, bs, esize):
+    kv = sum(lens) * hkv * d * 2 * esize
+    qo = 2 * len(lens) * hq * d * esize
+    tab = sum(-(-L // bs) for L in lens) * 4
+    return kv + qo + tab
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.index), "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- our path
+
+class Session:
+    """One replica: caches, the C++ manager, and per-step device inputs."""
+
+    def __init__(self, w, P, dev):
+        import paged_kv_cache_426_b200 as pa
+        self.pa, self.w, self.P, self.dev = pa, w, P, dev
+        dt = w.torch_dtype
+        self.esize = torch.tensor([], dtype=dt).element_size()
+        self.kc = torch.empty((w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim), dtype=dt,
+                              device=dev)
+        self.vc = torch.empty_like(self.kc)
+        self.err = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.max_len = max(w.meta["lens"]) - 1 + w.num_steps
+        self.mb = -(-self.max_len // w.block_size)
+        steps = [op for op in w.ops if op[0] == "step"]
+        self.S = len(steps[0][1])
+        self.ws = pa.alloc_workspace(self.S, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                     self.max_len, P, dev)
+
+    def new_manager(self):
+        pa = self.pa
+        alloc = pa.BlockAllocator(self.w.num_blocks, self.w.free_order)
+        return alloc, pa.BlockManager(alloc, self.w.block_size)
+
+    def prefill(self, write=True):
+        """Run the script up to the first step; write the prefill K/V (untimed)."""
+        w, pa = self.w, self.pa
+        alloc, mgr = self.new_manager()
+        ks, vs, slots = [], [], []
+        for op in w.ops:
+            if op[0] == "add":
+                mgr.add_seq(op[1])
+            elif op[0] == "fork":
+                mgr.fork(op[1], op[2])
+            elif op[0] == "write":
+                sl, cow = mgr.append(op[1], w.kv["k" + op[2]].shape[0])
+                if cow and write:     # a write into a shared block copies it first
+                    self._flush(ks, vs, slots)
+                    pa.pa_copy_blocks(self.kc, self.vc, torch.tensor(cow, device=self.dev))
+                ks.append(w.kv["k" + op[2]])
+                vs.append(w.kv["v" + op[2]])
+                slots.append(sl)
+            elif op[0] == "step":
+                break
+        if write:
+            self._flush(ks, vs, slots)
+            torch.cuda.synchronize()
+        return alloc, mgr
+
+    def _flush(self, ks, vs, slots):
+        if not ks:
+            return
+        k = torch.cat(ks).to(self.dev)
+        v = torch.cat(vs).to(self.dev)
+        s = torch.cat(slots).to(self.dev)
+        self.pa.pa_reshape_and_cache(k, v, self.kc, self.vc, s)
+        ks.clear(); vs.clear(); slots.clear()
+
+    def plan_steps(self, mgr, n):
+        """Host metadata of steps 0..n-1, uploaded to HBM with the step inputs."""
+        w = self.w
+        plan = []
+        for k in range(n):
+            seqs = w.step_seqs(k)
+            slots, cow = mgr.append_step(seqs)
+            tab, lens = mgr.block_tables(seqs, self.mb)
+            plan.append(dict(
+                slots=slots.to(self.dev), cow=cow.to(self.dev) if cow.shape[0] else None,
+                tab=tab.to(self.dev), lens=lens.to(self.dev), lens_host=lens.tolist(),
+                q=w.step_q[k].to(self.dev), k=w.step_k[k].to(self.dev),
+                v=w.step_v[k].to(self.dev)))
+        return plan
+
+    def run_step(self, st, out):
+        pa, w = self.pa, self.w
+        n = 0
+        if st["cow"] is not None:
+            pa.pa_copy_blocks(self.kc, self.vc, st["cow"], err_flag=self.err)
+            n += 1
+        pa.pa_reshape_and_cache(st["k"], st["v"], self.kc, self.vc, st["slots"], err_flag=self.err)
+        return n + 1
+
+    def decode(self, st, out):
+        self.pa.pa_decode(out, st["q"], self.kc, self.vc, st["tab"], st["lens"], self.max_len,
+                          self.w.scale, partition_size=self.P, workspace=self.ws,
+                          err_flag=self.err)
+
+    def bytes_of(self, lens):
+        w = self.w
+        return algorithmic_bytes(lens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                                 self.esize)
+
+
+def run_ours(args, rank, world, local):
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    n_steps = args.warmup + args.steps
+    w = workloads.make(args.workload, steps=n_steps)
+    P = w.partition_size if args.partition_size is None else args.partition_size
+    import paged_kv_cache_426_b200 as pa
+    pa.pa_set_decode_engine({"auto": 0, "core": 1, "mma": 2}[args.engine])
+    sess = Session(w, P, dev)
+    _, mgr = sess.prefill()
+    plan = sess.plan_steps(mgr, n_steps)
+    out = torch.empty_like(plan[0]["q"])
+    stream = torch.cuda.current_stream()
+
+    # clock soak: step 0 again and again (idempotent writes) while the sampler starts
+    sampler = ClockSampler(local)
+    sampler.start()
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(10):
+            sess.run_step(plan[0], out)
+            sess.decode(plan[0], out)
+        torch.cuda.synchronize()
+
+    for k in range(args.warmup):
+        sess.run_step(plan[k], out)
+        sess.decode(plan[k], out)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    launches = 0
+    for i in range(args.steps):
+        st = plan[args.warmup + i]
+        ev[i][0].record(stream)
+        launches += sess.run_step(st, out)
+        ev[i][1].record(stream)
+        sess.decode(st, out)
+        launches += 1
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    assert int(sess.err.item()) == 0, f"device error flag {int(sess.err.item())}"
+    span_ms = ev[0][0].elapsed_time(ev[-1][2])
+    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    span_ms = max_over_ranks(span_ms, world)
+    step_bytes = [sess.bytes_of(plan[args.warmup + i]["lens_host"]) for i in range(args.steps)]
+    total_bytes = sum(step_bytes) * world
+    value = total_bytes / (span_ms * 1e-3) / 1e9
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    dec_gbs = (sum(step_bytes) / len(step_bytes)) / (dec_avg_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    S = sess.S
+
+    e2e = run_e2e(sess, w, args, world) if args.e2e else None
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(span_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded; see workloads/)",
+        "config": {"workload": w.name, "num_seqs": S, "num_q_heads": w.num_q_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+                   "block_size": w.block_size, "partition_size": P,
+                   "mean_context_len": round(sum(plan[args.warmup]["lens_host"]) / S, 1),
+                   "kv_bytes_per_step": step_bytes[0],
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (KV cache >= 0.6 GB vs 126 MB)",
+                   "engine": args.engine},
+        "seqs_per_s": round(S * world / (span_ms * 1e-3 / args.steps), 1),
+        "decode_only": {"gbs": round(dec_gbs, 1), "ms": round(dec_avg_ms, 4),
+                        "seqs_per_s": round(S / (dec_avg_ms * 1e-3), 1)},
+        "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(dec_gbs / peak, 4), "traffic": None,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "pa_decode"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if e2e:
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    return result
+
+
+def run_e2e(sess, w, args, world):
+    """Same metric through the public API with host buffers, every step:
+    live C++ manager appends, H2D from pinned buffers, kernels, D2H of out."""
+    pa = sess.pa
+    dev = sess.dev
+    _, mgr = sess.prefill(write=False)       # same script -> same pool state
+    S, mb = sess.S, sess.mb
+    hq, hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
+    pin = dict(slots=torch.empty(S, dtype=torch.int64).pin_memory(),
+               cow=torch.empty((S, 2), dtype=torch.int64).pin_memory(),
+               tab=torch.empty((S, mb), dtype=torch.int32).pin_memory(),
+               lens=torch.empty(S, dtype=torch.int32).pin_memory(),
+               out=torch.empty((S, hq, d), dtype=w.torch_dtype).pin_memory())
+    qs = [w.step_q[k].pin_memory() for k in range(w.num_steps)]
+    kk = [w.step_k[k].pin_memory() for k in range(w.num_steps)]
+    vv = [w.step_v[k].pin_memory() for k in range(w.num_steps)]
+    dq = torch.empty((S, hq, d), dtype=w.torch_dtype, device=dev)
+    dk = torch.empty((S, hkv, d), dtype=w.torch_dtype, device=dev)
+    dvv = torch.empty_like(dk)
+    dslots = torch.empty(S, dtype=torch.int64, device=dev)
+    dcow = torch.empty((S, 2), dtype=torch.int64, device=dev)
+    dtab = torch.empty((S, mb), dtype=torch.int32, device=dev)
+    dlens = torch.empty(S, dtype=torch.int32, device=dev)
+    dout = torch.empty((S, hq, d), dtype=w.torch_dtype, device=dev)
+    h2d = d2h = 0
+    total_bytes = 0
+    times = []
+    for k in range(args.warmup + args.steps):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        seqs = w.step_seqs(k)
+        slots, cow = mgr.append_step(seqs, slots_out=pin["slots"], cow_out=pin["cow"])
+        tab, lens = mgr.block_tables(seqs, mb, tables_out=pin["tab"], lens_out=pin["lens"])
+        ncow = cow.shape[0]
+        dq.copy_(qs[k], non_blocking=True)
+        dk.copy_(kk[k], non_blocking=True)
+        dvv.copy_(vv[k], non_blocking=True)
+        dslots.copy_(pin["slots"], non_blocking=True)
+        dtab.copy_(pin["tab"], non_blocking=True)
+        dlens.copy_(pin["lens"], non_blocking=True)
+        if ncow:
+            dcow[:ncow].copy_(pin["cow"][:ncow], non_blocking=True)
+            pa.pa_copy_blocks(sess.kc, sess.vc, dcow[:ncow], err_flag=sess.err)
+        pa.pa_reshape_and_cache(dk, dvv, sess.kc, sess.vc, dslots, err_flag=sess.err)
+        pa.pa_decode(dout, dq, sess.kc, sess.vc, dtab, dlens, sess.max_len, w.scale,
+                     partition_size=sess.P, workspace=sess.ws, err_flag=sess.err)
+        pin["out"].copy_(dout, non_blocking=True)
+        torch.cuda.synchronize()
+        t1 = time.perf_counter()
+        if k >= args.warmup:
+            times.append(t1 - t0)
+            total_bytes += sess.bytes_of(lens.tolist())
+            h2d = sum(t.numel() * t.element_size() for t in (qs[k], kk[k], vv[k], pin["slots"],
+                                                              pin["tab"], pin["lens"]))
+            h2d += ncow * 16
+            d2h = pin["out"].numel() * pin["out"].element_size()
+    span = max_over_ranks(sum(times), world)
+    return {"value": round(total_bytes * world / span / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(span / args.steps * 1e3, 4)}
+
+
+# ----------------------------------------------------------------------------- the oracle on the host
+
+def cpu_baseline(w, seconds):
+    """The oracle, as it stands, on the host cores: float64 decode of as many
+    whole sequences of the first step's batch as fit in about ``seconds``."""
+    import numpy as np
+    import oracle
+    from threadpoolctl import threadpool_info
+    rec = oracle.run(w, decode=False, steps=1)
+    st = rec.steps[0]
+    q = oracle.as_storage(w.step_q[0], w.dtype)
+    esize = torch.tensor([], dtype=w.torch_dtype).element_size()
+    done, nbytes, t0 = 0, 0, time.perf_counter()
+    order = list(range(len(st.seqs)))
+    while done < len(order):
+        s = order[done]
+        oracle.paged_decode(q[s:s + 1], rec.key_cache, rec.value_cache, st.block_tables[s:s + 1],
+                            st.context_lens[s:s + 1], w.scale, w.dtype)
+        nbytes += algorithmic_bytes([int(st.context_lens[s])], w.num_q_heads, w.num_kv_heads,
+                                    w.head_dim, w.block_size, esize)
+        done += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{done} of {len(order)} sequences of step 0 of {w.name}, float64 numpy "
+                      f"(gather through the block table + softmax attention), {dt:.1f} s",
+            "seqs_per_s": round(done / dt, 3), "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host: each step a bounded sample of the batch."""
+    if rank != 0:
+        return None
+    w = workloads.make(args.workload, steps=1)
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        cpu_baseline(w, 0.5)
+    vals = []
+    base = None
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        base = cpu_baseline(w, per_step)
+        vals.append(base["value"])
+    span = time.perf_counter() - t0
+    value = sum(vals) / len(vals)
+    base["value"] = round(value, 4)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(span / args.steps * 1e3, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; see workloads/)",
+            "config": {"workload": w.name, "parallelism": "host cores"},
+            "cpu_baseline": base,
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=29)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BUILDERS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--engine", default="auto", choices=["auto", "core", "mma"])
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of clock soak")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    rank, world, local = (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+                          int(os.environ.get("LOCAL_RANK", "0")))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    res = run_ours(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * pa.h - C ABI of the B200 paged KV-cache decode library (libpa_b200.so).
+ *
+ * PagedAttention keeps each request's K/V cache in fixed-size physical blocks
+ * that a per-request block table maps from logical order; attention reads the
+ * scattered blocks through that table.  Sources, by page title and section:
+ *   [KVC]  "KV Cache & PagedAttention" studynote (agnusdei1207), II
+ *          (block table, copy-on-write) and III (attention kernel modified);
+ *   [VLLM] "vLLM PagedAttention" studynote (agnusdei1207), II (fixed-size
+ *          blocks, e.g. 16 tokens; logical -> physical block table);
+ *   [119]  "09. PagedAttention" (119-ai-studio), 해법 (logical / physical
+ *          blocks, block table; only the last block is partly filled);
+ *   [VEL]  "Paged Attention" (velog @junegood), 작동 예시 (on-demand block
+ *          growth), 메모리 공유 (copy-on-write for beams), 구현 세부사항
+ *          (BlockAllocator.allocate_block / free_block).
+ *
+ * Conventions for every call:
+ *  - Return value: a pa_status (0 = PA_OK).  Host-side argument checks run
+ *    before anything is launched; a failed check launches nothing.
+ *  - Device pointers are caller-owned (e.g. PyTorch tensors).  The library
+ *    never allocates or frees device memory and never synchronises; it
+ *    launches only on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *  - `err_flag` (nullable) is a device int32 that kernels set to a
+ *    PA_DEV_* code when they meet bad data (first code wins; 0 is never
+ *    written).  The bad access is skipped; no kernel traps.  The caller
+ *    clears and reads it.
+ *  - Cache layout (part of this ABI): key_cache and value_cache are each
+ *    [num_blocks][num_kv_heads][block_size][head_dim] elements of `dtype`,
+ *    row-major, 16-byte aligned.  One (block, KV head) tile is
+ *    block_size*head_dim contiguous elements; slot = block*block_size + offset.
+ *  - Supported: head_dim 64 or 128; block_size 8, 16, 32, 64 or 128;
+ *    dtype f32, f16, bf16; num_q_heads = G * num_kv_heads with G in 1,2,4,8.
+ *  - Host objects (allocator, manager) are not thread-safe.
+ */
+#ifndef PA_B200_H
+#define PA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID = -1,      /* bad argument (null pointer, size, range) */
+    PA_ERR_UNSUPPORTED = -2,  /* valid but not built (head_dim, dtype, G)  */
+    PA_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed      */
+    PA_ERR_OOM = -4,          /* the block pool is empty                   */
+    PA_ERR_STATE = -5         /* refcount / sequence state violated        */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/* Codes written to *err_flag by kernels. */
+enum {
+    PA_DEV_BAD_SLOT = 1,      /* slot_mapping entry >= num_blocks*block_size */
+    PA_DEV_BAD_BLOCK = 2,     /* block table entry outside [0, num_blocks)   */
+    PA_DEV_BAD_LEN = 3,       /* context_len < 0, > max_context_len, or
+                                 > max_blocks_per_seq*block_size (clamped)  */
+    PA_DEV_BAD_PAIR = 4,      /* copy pair id outside [0, num_blocks)        */
+    PA_DEV_TIMEOUT = 5        /* a pipeline wait exceeded its time limit     */
+};
+
+/* Human-readable name of a pa_status. */
+const char* pa_status_string(int status);
+/* ABI version (major*100 + minor). */
+int pa_version(void);
+
+/* --------------------------------------------------------------------------
+ * pa_reshape_and_cache - write each new token's K and V rows into its slot.
+ *
+ * [119] 해법 / [VEL] 작동 예시: a token's K/V goes into the physical block the
+ * table assigns to its logical position.  For t < num_tokens and every KV
+ * head h:  key_cache[s / bs][h][s % bs][:] = key[t][h][:]  (same for value),
+ * s = slot_mapping[t].  s < 0 marks padding: skipped.  s >= num_blocks*bs sets
+ * PA_DEV_BAD_SLOT and is skipped.
+ *   key, value    device [num_tokens][num_kv_heads][head_dim] dtype, contiguous
+ *   slot_mapping  device int64 [num_tokens]; distinct non-negative entries
+ * Bit copy: the cache holds exactly the input bits.
+ */
+int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
+                         void* value_cache, const int64_t* slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, pa_dtype dtype,
+                         int32_t* err_flag, void* stream);
+
+/* --------------------------------------------------------------------------
+ * pa_decode - one decode step of paged attention.
+ *
+ * [KVC] II-III / [119] 해법: attention reads K/V through the block table.  For
+ * sequence s, query head h, KV head j = h / G (G = num_q_heads/num_kv_heads),
+ * tokens t < L = context_lens[s] (L counts the token written this step):
+ *   K_t = key_cache[block_tables[s][t / bs]][j][t % bs][:],  V_t likewise,
+ *   x_t = scale * <query[s][h], K_t>,  w = softmax(x),  out[s][h] = sum_t w_t V_t
+ * fp32 accumulation; out is rounded to nearest even in dtype.  L = 0 gives 0.
+ * Long contexts are split into partitions of `partition_size` tokens
+ * (a positive multiple of 16; 0 = one partition per sequence) whose partial
+ * results are merged with their log-sum-exp weights in the same launch.
+ *   out           device [num_seqs][num_q_heads][head_dim] dtype
+ *   query         device [num_seqs][num_q_heads][head_dim] dtype, 16-B aligned
+ *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past
+ *                 ceil(L/bs) are ignored (conventionally -1)
+ *   context_lens  device int32 [num_seqs]
+ *   max_context_len  host upper bound of context_lens (sizes the workspace)
+ *   workspace     device, >= pa_decode_workspace_size() bytes, 256-B aligned;
+ *                 must be zero-filled before its first use (see
+ *                 pa_decode_workspace_init); every call leaves its scheduler
+ *                 words zero again.  Calls sharing one workspace must not
+ *                 overlap on the GPU.
+ * The physical placement of blocks does not change the result: summation
+ * order depends only on logical token positions.
+ */
+int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
+                             int head_dim, int max_context_len,
+                             int partition_size, size_t* bytes);
+int pa_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+int pa_decode(void* out, const void* query, const void* key_cache,
+              const void* value_cache, const int32_t* block_tables,
+              int max_blocks_per_seq, const int32_t* context_lens,
+              int max_context_len, int num_seqs, int num_q_heads,
+              int num_kv_heads, int head_dim, int block_size, int num_blocks,
+              float scale, int partition_size, void* workspace,
+              size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
+              void* stream);
+
+/* Decode engine selection (for measurement): PA_ENGINE_AUTO picks tensor-core
+ * MMA for f16/bf16 and CUDA cores for f32; PA_ENGINE_CUDA_CORE forces the
+ * CUDA-core dot products.  Process-wide; returns the previous value. */
+enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_MMA = 2 };
+int pa_set_decode_engine(int engine);
+
+/* --------------------------------------------------------------------------
+ * pa_copy_blocks - copy-on-write block copies.
+ *
+ * [KVC] II (copy-on-write) / [VEL] 메모리 공유: before a sharer writes into a
+ * shared block, the block is copied to a fresh one.  For each pair p:
+ * key_cache[dst] = key_cache[src] (all KV heads and offsets), same for value.
+ *   block_pairs  device int64 [num_pairs][2] = (src, dst); dsts distinct and
+ *                disjoint from srcs.  An id outside [0, num_blocks) sets
+ *                PA_DEV_BAD_PAIR and that pair is skipped.
+ */
+int pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs,
+                   int num_pairs, int num_kv_heads, int head_dim, int block_size,
+                   int num_blocks, pa_dtype dtype, int32_t* err_flag, void* stream);
+
+/* --------------------------------------------------------------------------
+ * Host block allocator ([VEL] 구현 세부사항: allocate_block / free_block).
+ *
+ * A first-in-first-out pool of free physical block ids with a reference
+ * count per block.  create: `free_order` (nullable) lists the ids handed out
+ * first, `num_free` of them; ids not listed start held (count 1) by an outside
+ * owner, which models a pool other requests have fragmented.  NULL = all ids
+ * free in ascending order.  allocate: pops the front (count 1), PA_ERR_OOM
+ * when empty.  incref: shares an allocated block (PA_ERR_STATE if free).
+ * free: drops one reference; at zero the id joins the back of the pool;
+ * PA_ERR_STATE on a free block (double free).
+ */
+typedef struct pa_allocator pa_allocator;
+int pa_allocator_create(int num_blocks, const int32_t* free_order, int num_free,
+                        pa_allocator** out);
+void pa_allocator_destroy(pa_allocator* a);
+int pa_allocator_allocate(pa_allocator* a, int32_t* block_id);
+int pa_allocator_incref(pa_allocator* a, int32_t block_id);
+int pa_allocator_free(pa_allocator* a, int32_t block_id);
+int pa_allocator_refcount(const pa_allocator* a, int32_t block_id, int32_t* refcount);
+int pa_allocator_num_free(const pa_allocator* a, int32_t* num_free);
+
+/* --------------------------------------------------------------------------
+ * Host block-table manager: per-sequence logical -> physical tables over an
+ * allocator ([119] 해법; [VEL] 작동 예시, 메모리 공유).
+ *
+ * append (one token at position p = current length): if p % bs == 0 a new
+ * block is taken; otherwise the token goes into the last block, and if that
+ * block is shared (count > 1) it is first replaced by a fresh block, the pair
+ * (old, new) is reported for pa_copy_blocks and the old block loses one
+ * reference.  slot = table[p / bs] * bs + p % bs.  Appends are all-or-nothing:
+ * PA_ERR_OOM leaves every table and count unchanged.
+ *   pa_manager_append       num_tokens tokens to one sequence; slots[num_tokens];
+ *                           cow_pairs int64 [>=1][2], *num_cow in {0,1}
+ *   pa_manager_append_step  one token to each of seq_ids[0..n); slots[n];
+ *                           cow_pairs int64 [n][2]; *num_cow <= n
+ *   pa_manager_fork         child shares every block of parent (incref)
+ *   pa_manager_free_seq     drops the sequence's references
+ *   pa_manager_block_tables rows [n][max_blocks] padded with -1, lengths [n];
+ *                           PA_ERR_INVALID if a table is longer than max_blocks
+ * The manager borrows the allocator, which must outlive it.
+ */
+typedef struct pa_manager pa_manager;
+int pa_manager_create(pa_allocator* alloc, int block_size, pa_manager** out);
+void pa_manager_destroy(pa_manager* m);
+int pa_manager_add_seq(pa_manager* m, int64_t seq_id);
+int pa_manager_fork(pa_manager* m, int64_t parent, int64_t child);
+int pa_manager_free_seq(pa_manager* m, int64_t seq_id);
+int pa_manager_append(pa_manager* m, int64_t seq_id, int num_tokens,
+                      int64_t* slots, int64_t* cow_pairs, int* num_cow);
+int pa_manager_append_step(pa_manager* m, const int64_t* seq_ids, int num_seqs,
+                           int64_t* slots, int64_t* cow_pairs, int* num_cow);
+int pa_manager_seq_len(const pa_manager* m, int64_t seq_id, int32_t* len);
+int pa_manager_block_tables(const pa_manager* m, const int64_t* seq_ids,
+                            int num_seqs, int32_t* block_tables, int max_blocks,
+                            int32_t* context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PA_B200_H */

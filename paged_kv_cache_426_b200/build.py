@@ -1,0 +1,92 @@
+"""Build libpa_b200.so in-tree with nvcc for sm_100a (B200).
+
+    python -m paged_kv_cache_426_b200.build [--force] [--ptxas-info]
+
+Objects go to ``_build/`` next to the package; the shared library lands in the
+package directory, where the binding loads it.  The CUDA runtime is linked
+statically so the library does not depend on the runtime version torch ships.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+from concurrent.futures import ThreadPoolExecutor
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+BUILD = os.path.join(ROOT, "_build")
+LIB = os.path.join(PKG, "libpa_b200.so")
+
+SOURCES = ["pa_host.cpp", "pa_cache_ops.cu", "pa_decode.cu"]
+HEADERS = [os.path.join(CSRC, "pa_common.cuh"), os.path.join(INCLUDE, "pa.h")]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", shutil.which("nvcc")):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def _flags(ptxas_info: bool):
+    f = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
+                "-I", CSRC, "--expt-relaxed-constexpr"]
+    if ptxas_info:
+        f += ["-Xptxas", "-v"]
+    return f
+
+
+def _stale(target: str, deps) -> bool:
+    if not os.path.exists(target):
+        return True
+    t = os.path.getmtime(target)
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    cc = nvcc()
+    objs, jobs = [], []
+    for src in SOURCES:
+        path = os.path.join(CSRC, src)
+        obj = os.path.join(BUILD, src + ".o")
+        objs.append(obj)
+        if force or ptxas_info or _stale(obj, [path] + HEADERS):
+            jobs.append([cc, *_flags(ptxas_info), "-c", path, "-o", obj])
+
+    def run(cmd):
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"nvcc failed:\n{' '.join(cmd)}\n{r.stdout}\n{r.stderr}")
+        return r.stdout + r.stderr
+
+    with ThreadPoolExecutor(max_workers=len(jobs) or 1) as ex:
+        logs = list(ex.map(run, jobs))
+    if ptxas_info:
+        for log in logs:
+            sys.stdout.write(log)
+    if force or jobs or _stale(LIB, objs):
+        run([cc, *ARCH, "-shared", "-cudart", "static", *objs, "-o", LIB + ".tmp"])
+        os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--ptxas-info", action="store_true")
+    ap.add_argument("-v", "--verbose", action="store_true")
+    a = ap.parse_args()
+    print(build(force=a.force, ptxas_info=a.ptxas_info, verbose=a.verbose))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,1023 @@
+// pa_decode: paged decode attention for sm_100a (B200).
+//
+// What it computes ("KV Cache & PagedAttention" studynote, II-III: attention
+// reads K/V scattered over blocks through the block table; "09. PagedAttention"
+// (119-ai-studio), 해법: logical blocks -> physical blocks): for sequence s,
+// query head h, KV head j = h / G and tokens t < L_s,
+//   x_t = scale <q_h, K_t>,  out_h = sum_t softmax(x)_t V_t,
+//   K_t = key_cache[block_tables[s][t / bs]][j][t % bs][:].
+//
+// How (one launch per decode step):
+//  * Work unit = (sequence s, KV head j, partition i) covering tokens
+//    [i*P, min(L_s, (i+1)*P)).  All G query heads of the group are served by
+//    one pass over the group's K/V, so every K/V byte is read from HBM once.
+//  * Persistent CTAs (one per SM).  Each CTA computes the prefix sums of the
+//    partition counts (tiny), then one producer warp takes units from an
+//    atomic counter in the workspace (dynamic load balance, units of at most
+//    P tokens) and streams each unit as 16-token stages into a shared-memory
+//    ring: 2-D tensor TMA copies of 128-byte-wide boxes with 128B swizzle,
+//    one box row per token, so that all later shared-memory reads are free of
+//    bank conflicts.  The block table is read 32 entries at a time by the
+//    producer's lanes, ahead of use.  A 16-token stage never crosses a block
+//    (bs >= 16) or covers two (bs = 8).
+//  * Consumer warps take a unit's stages round-robin by logical stage index
+//    and keep a per-warp online softmax (running max m, sum l, output o) in
+//    the log2 domain.  Two compute engines:
+//      CUDA cores: 8 (or 16) lanes per token, 16-byte loads, warp-shuffle
+//        reduce-scatter of the G dot products, then p*V with each lane owning
+//        head_dim/32 output columns of all G heads;
+//      MMA (16-bit types): S = Q K^T and O += P V with m16n8k16 tensor-core
+//        MMAs; the query heads sit in the M dimension (rows >= G are zero),
+//        K and V come from the swizzled stage with ldmatrix(.trans), and the
+//        accumulators of S are reused directly as the A operand of P V.
+//  * At the end of a unit the consumer warps merge their states in shared
+//    memory.  A single-partition sequence writes `out` directly.  Otherwise
+//    the unit writes (m, l, o) to the workspace and bumps a per-(s, j)
+//    counter; the CTA that completes the last partition merges all partials
+//    with their log-sum-exp weights and writes `out` (and re-zeroes the
+//    counter).  No CTA ever waits for another.
+//  * Summation order depends only on logical positions (stage index within
+//    the unit, warp index, partition index), never on physical block ids or
+//    on which CTA ran a unit, so results are bit-identical under any
+//    permutation of the pool and for block sizes 16..128.
+//  * Every wait is bounded (2 s); a timeout sets PA_DEV_TIMEOUT, makes the
+//    other warps give up quickly, waits (bounded) for the CTA's own copies
+//    in flight and returns.  Bad block ids or lengths set err_flag and the
+//    affected tokens are skipped.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int TOK = 16;       // tokens per pipeline stage
+constexpr int NUR = 8;        // unit-descriptor ring slots
+constexpr int BOXB = TOK * 128;   // bytes of one 16-row x 128-byte box
+
+struct alignas(16) UnitDesc {
+    int s, j, i, t0, t1, n_p, stage_base, n_stages, end, pad0, pad1, pad2;
+};
+
+struct alignas(16) WsHeader {
+    int next_unit;   // dynamic scheduler ticket
+    int done_ctas;   // CTAs finished; the last one re-zeroes both
+    int pad[62];
+};
+
+struct DecodeParams {
+    void* out;
+    const void* q;
+    const int32_t* tables;
+    const int32_t* lens;
+    int mbps, max_len, S, Hq, Hkv, NB, bs, P, n_pmax, nstage;
+    float scale_log2e;
+    WsHeader* hdr;
+    int* counters;     // [S*Hkv]
+    float* part_ml;    // [S*Hkv][n_pmax][G][2]
+    float* part_o;     // [S*Hkv][n_pmax][G][D]
+    int32_t* err;
+};
+
+// Shared-memory layout (dynamic, 1024-byte aligned base).
+template <typename T, int D, int G, int NCW>
+struct Layout {
+    static constexpr int E = sizeof(T);
+    static constexpr int ROWB = D * E;               // bytes per token row
+    static constexpr int NBOX = ROWB / 128;          // 128-byte boxes per row
+    static constexpr int KV_BYTES = NBOX * BOXB;     // one stage of K (or V)
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int QB = ((G * D * E + 127) / 128) * 128;
+    static constexpr int RING_BYTES = NUR * (int)(sizeof(UnitDesc) + QB);
+    static constexpr int SCRATCH = NCW * 2 * G * TOK * 4;        // xs + ps
+    static constexpr int MBUF = 2 * NCW * G * (D + 2) * 4;       // double buffered
+    int nstage, S;
+    __host__ __device__ Layout(int nstage_, int S_) : nstage(nstage_), S(S_) {}
+    __host__ __device__ size_t ring() const { return (size_t)nstage * STAGE_BYTES; }
+    __host__ __device__ size_t bars() const { return ring() + RING_BYTES; }
+    __host__ __device__ size_t stage_ok() const { return bars() + (size_t)(2 * nstage + 2 * NUR) * 8; }
+    __host__ __device__ size_t scratch() const { return ((stage_ok() + 4 * nstage + 15) / 16) * 16; }
+    __host__ __device__ size_t mbuf() const { return scratch() + SCRATCH; }
+    __host__ __device__ size_t misc() const { return mbuf() + MBUF; }          // 64 ints
+    __host__ __device__ size_t lens() const { return misc() + 256; }
+    __host__ __device__ size_t pre() const { return lens() + 4 * (size_t)S; }
+    __host__ __device__ size_t total() const { return pre() + 4 * (size_t)(S + 1); }
+    static __host__ __device__ size_t fixed_bytes(int S_) { return Layout(0, S_).total(); }
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__device__ __forceinline__ int clamp_len(int L, const DecodeParams& p) {
+    const int hi = min(p.max_len, p.mbps * p.bs);
+    if (L < 0 || L > hi) {
+        set_err(p.err, PA_DEV_BAD_LEN);
+        L = max(0, min(L, hi));
+    }
+    return L;
+}
+
+__device__ __forceinline__ int n_parts(int L, int P) { return max(1, ceil_div(L, P)); }
+
+// Bounded wait that also gives up as soon as another warp has given up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
+                                              volatile int* abort_flag, int32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            set_err(err, PA_DEV_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Sum over the LPT lanes of one token of v[h(lane)], h(lane) = (lane % LPT) / (LPT / G):
+// a butterfly that halves the head set at each step while G > 1.
+template <int G, int LPT>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane) {
+    float a[G];
+#pragma unroll
+    for (int k = 0; k < G; ++k) a[k] = v[k];
+    int cnt = G;
+#pragma unroll
+    for (int off = LPT / 2; off >= 1; off >>= 1) {
+        if (cnt > 1) {
+            const int half = cnt / 2;
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int k = 0; k < half; ++k) {
+                const float send = upper ? a[k] : a[k + half];
+                const float keep = upper ? a[k + half] : a[k];
+                a[k] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+            cnt = half;
+        } else {
+            a[0] += __shfl_xor_sync(0xffffffffu, a[0], off);
+        }
+    }
+    return a[0];
+}
+
+// ------------------------------------------------------------ compute engines
+// Per-warp online-softmax state and one stage's update.  Stage smem: K boxes
+// then V boxes; box b holds columns [b*128, b*128+128) bytes of 16 rows, with
+// the 16-byte chunk c of row r stored at chunk position c ^ (r & 7).
+
+template <typename T, int D, int G, int NCW>
+struct CoreEngine {
+    using LY = Layout<T, D, G, NCW>;
+    static constexpr int E = sizeof(T);
+    static constexpr int VEC = 16 / E;                       // elements per chunk
+    static constexpr int CHUNKS = LY::ROWB / 16;             // chunks per row
+    static constexpr int LPT = (G >= 8 && CHUNKS >= 16) ? 16 : 8;
+    static constexpr int TPW = 32 / LPT;                     // tokens per warp step
+    static constexpr int NCH = CHUNKS / LPT;                 // chunks per lane
+    static constexpr int DPL = D / 32;                       // PV columns per lane
+    static constexpr int NPASS = (G + 1) / 2;
+    static_assert(G <= LPT, "group larger than lanes per token");
+
+    float qf[G][NCH * VEC];
+    float o[G][DPL];
+    float m_half[NPASS], l_half[NPASS];
+
+    __device__ void begin_unit(const T* qs, int lane, float scale_log2e) {
+        const int r = lane % LPT;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e)
+                    qf[g][c * VEC + e] =
+                        DT<T>::to_float(qs[g * D + (r + c * LPT) * VEC + e]) * scale_log2e;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
+#pragma unroll
+        for (int k = 0; k < NPASS; ++k) { m_half[k] = -INFINITY; l_half[k] = 0.f; }
+    }
+
+    __device__ void stage(const uint8_t* Ks, const uint8_t* Vs, int nv, float* xs, float* ps,
+                          int lane) {
+        const int r = lane % LPT;
+        // ---- x_t = <q_g, K_t> (pre-scaled to log2 units)
+#pragma unroll
+        for (int step = 0; step < TOK / TPW; ++step) {
+            const int tok = step * TPW + lane / LPT;
+            float acc[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                const int ch = r + c * LPT;
+                const uint4 raw = *reinterpret_cast<const uint4*>(
+                    Ks + (ch >> 3) * BOXB + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4));
+                float x[VEC];
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) Unpack<T>::run(w[k], &x[k * Unpack<T>::N]);
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) acc[g] = fmaf(qf[g][c * VEC + e], x[e], acc[g]);
+            }
+            const float v = reduce_scatter<G, LPT>(acc, lane);
+            constexpr int LPH = LPT / G;           // lanes holding one head's total
+            if ((r % LPH) == 0) xs[(r / LPH) * TOK + tok] = (tok < nv) ? v : -INFINITY;
+        }
+        __syncwarp();
+        // ---- online softmax over the stage's tokens, two heads per pass
+        float alpha[G];
+#pragma unroll
+        for (int pass = 0; pass < NPASS; ++pass) {
+            const int g = 2 * pass + (lane >> 4);
+            const int t = lane & 15;
+            const bool live = g < G;
+            const float x = live ? xs[g * TOK + t] : -INFINITY;
+            float bm = x;
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+            const float mo = m_half[pass];
+            const float mn = fmaxf(mo, bm);
+            const float pr = live ? exp2f(x - mn) : 0.f;
+            float sum = pr;
+#pragma unroll
+            for (int off = 8; off >= 1; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            const float a = live ? exp2f(mo - mn) : 1.f;
+            if (live) {
+                m_half[pass] = mn;
+                l_half[pass] = l_half[pass] * a + sum;
+                ps[t * G + g] = pr;
+            }
+            alpha[2 * pass] = __shfl_sync(0xffffffffu, a, 0);
+            if (2 * pass + 1 < G) alpha[2 * pass + 1] = __shfl_sync(0xffffffffu, a, 16);
+        }
+        __syncwarp();
+        // ---- o = alpha o + sum_t p_t V_t
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) o[g][e] *= alpha[g];
+        const int byte = lane * DPL * E;                  // this lane's columns
+        const int box = byte >> 7, cc = (byte & 127) >> 4, sub = byte & 15;
+        auto pv_token = [&](int t) {
+            const uint8_t* src = Vs + box * BOXB + t * 128 + (((cc ^ (t & 7)) << 4) | sub);
+            float v[DPL];
+            if constexpr (DPL * E == 16) {
+                const uint4 raw = *reinterpret_cast<const uint4*>(src);
+                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) Unpack<T>::run(w[k], &v[k * Unpack<T>::N]);
+            } else if constexpr (DPL * E == 8) {
+                const uint2 raw = *reinterpret_cast<const uint2*>(src);
+                Unpack<T>::run(raw.x, &v[0]);
+                Unpack<T>::run(raw.y, &v[Unpack<T>::N]);
+            } else {
+                const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
+                Unpack<T>::run(raw, &v[0]);
+            }
+            float pv[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) pv[g] = ps[t * G + g];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) o[g][e] = fmaf(pv[g], v[e], o[g][e]);
+        };
+        if (nv == TOK) {
+#pragma unroll
+            for (int t = 0; t < TOK; ++t) pv_token(t);
+        } else {
+            for (int t = 0; t < nv; ++t) pv_token(t);
+        }
+        __syncwarp();
+    }
+
+    // Write this warp's (m, l, o) into the merge buffer [G][D+2].
+    __device__ void dump(float* mb, int lane) const {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) mb[g * (D + 2) + 2 + lane * DPL + e] = o[g][e];
+#pragma unroll
+        for (int pass = 0; pass < NPASS; ++pass) {
+            const int g = 2 * pass + (lane >> 4);
+            if ((lane & 15) == 0 && g < G) {
+                mb[g * (D + 2) + 0] = m_half[pass];
+                mb[g * (D + 2) + 1] = l_half[pass];
+            }
+        }
+    }
+};
+
+template <typename T, int D, int G, int NCW>
+struct MmaEngine {
+    static_assert(sizeof(T) == 2, "tensor-core engine takes 16-bit types");
+    static_assert(G <= 8, "query heads of a group must fit 8 MMA rows");
+    static constexpr int KSTEPS = D / 16;
+    static constexpr int NDT = D / 8;          // 8-column output tiles
+
+    uint32_t qa[KSTEPS][2];    // A fragments of Q (rows lane/4, k low / k high)
+    float oacc[NDT][4];        // O rows lane/4 (and padding rows +8)
+    float m, l;                // state of row lane/4
+
+    __device__ void begin_unit(const T* qs, int lane, float) {
+        const int r = lane >> 2, c = lane & 3;
+        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qs);
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+            qa[k][0] = (r < G) ? q32[(r * D + 16 * k + 2 * c) >> 1] : 0u;
+            qa[k][1] = (r < G) ? q32[(r * D + 16 * k + 8 + 2 * c) >> 1] : 0u;
+        }
+#pragma unroll
+        for (int n = 0; n < NDT; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) oacc[n][e] = 0.f;
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    __device__ void stage(const uint8_t* Ks, uint8_t* Vs, int nv, float scale_log2e, int lane) {
+        const uint32_t kbase = smem_u32(Ks), vbase = smem_u32(Vs);
+        if (nv < TOK) {
+            // rows >= nv hold bytes of other tokens (or never-written memory);
+            // zero them so that p = 0 never meets a NaN in the P V product
+            constexpr int ROW16 = D * 2 / 16;
+            for (int idx = lane; idx < (TOK - nv) * ROW16; idx += 32) {
+                const int row = nv + idx / ROW16, ch = idx % ROW16;
+                *reinterpret_cast<uint4*>(Vs + (ch >> 3) * BOXB + row * 128 +
+                                          (((ch & 7) ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+            }
+            __syncwarp();
+        }
+        // ---- S = Q K^T  (rows: heads, columns: 16 tokens as two n-tiles)
+        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+        const int mi = lane >> 3, lr = lane & 7;
+#pragma unroll
+        for (int k = 0; k < KSTEPS; ++k) {
+            const int row = (mi >> 1) * 8 + lr, ch = 2 * k + (mi & 1);
+            uint32_t b00, b01, b10, b11;
+            ldsm_x4(kbase + (ch >> 3) * BOXB + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b00, b01,
+                    b10, b11);
+            mma16816<T>(s0, qa[k][0], 0u, qa[k][1], 0u, b00, b01);
+            mma16816<T>(s1, qa[k][0], 0u, qa[k][1], 0u, b10, b11);
+        }
+        // ---- online softmax of row lane/4 over this stage's tokens
+        const int c = lane & 3;
+        const int t0 = 2 * c, t1 = 2 * c + 1, t2 = 8 + 2 * c, t3 = 9 + 2 * c;
+        float x0 = (t0 < nv) ? s0[0] * scale_log2e : -INFINITY;
+        float x1 = (t1 < nv) ? s0[1] * scale_log2e : -INFINITY;
+        float x2 = (t2 < nv) ? s1[0] * scale_log2e : -INFINITY;
+        float x3 = (t3 < nv) ? s1[1] * scale_log2e : -INFINITY;
+        float bm = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+        const float mn = fmaxf(m, bm);
+        const float a = exp2f(m - mn);
+        const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
+        const float p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
+        float rs = (p0 + p1) + (p2 + p3);
+        rs += __shfl_xor_sync(0xffffffffu, rs, 1);
+        rs += __shfl_xor_sync(0xffffffffu, rs, 2);
+        l = l * a + rs;
+        m = mn;
+#pragma unroll
+        for (int n = 0; n < NDT; ++n) {
+            oacc[n][0] *= a;
+            oacc[n][1] *= a;
+        }
+        const uint32_t pa0 = pack2<T>(p0, p1), pa2 = pack2<T>(p2, p3);
+        // ---- O += P V  (B operand = V [tokens x columns] via ldmatrix.trans)
+#pragma unroll
+        for (int n2 = 0; n2 < NDT / 2; ++n2) {
+            const int row = (mi & 1) * 8 + lr, ch = 2 * n2 + (mi >> 1);
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(vbase + (ch >> 3) * BOXB + row * 128 + (((ch & 7) ^ (row & 7)) << 4), v0, v1,
+                      v2, v3);
+            mma16816<T>(oacc[2 * n2], pa0, 0u, pa2, 0u, v0, v1);
+            mma16816<T>(oacc[2 * n2 + 1], pa0, 0u, pa2, 0u, v2, v3);
+        }
+    }
+
+    __device__ void dump(float* mb, int lane) const {
+        const int r = lane >> 2, c = lane & 3;
+        if (r < G) {
+#pragma unroll
+            for (int n = 0; n < NDT; ++n)
+                *reinterpret_cast<float2*>(&mb[r * (D + 2) + 2 + 8 * n + 2 * c]) =
+                    make_float2(oacc[n][0], oacc[n][1]);
+            if (c == 0) {
+                mb[r * (D + 2) + 0] = m;
+                mb[r * (D + 2) + 1] = l;
+            }
+        }
+    }
+};
+
+// ------------------------------------------------------------ the kernel
+template <typename T, int D, int G, int NCW, bool MMA>
+__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+              DecodeParams p) {
+    using LY = Layout<T, D, G, NCW>;
+    using Engine = typename std::conditional<MMA, MmaEngine<T, D, G, NCW>,
+                                             CoreEngine<T, D, G, NCW>>::type;
+    constexpr int NT = (NCW + 1) * 32;
+    constexpr int CT = NCW * 32;                 // consumer threads
+    constexpr int E = sizeof(T);
+    constexpr int BOX_ELEMS = 128 / E;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 128B-swizzled TMA boxes need 1024-byte aligned destinations
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const LY ly(p.nstage, p.S);
+    uint8_t* stages = smem;
+    uint8_t* ring = smem + ly.ring();
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars());
+    uint64_t* empty = full + p.nstage;
+    uint64_t* ufull = empty + p.nstage;
+    uint64_t* uempty = ufull + NUR;
+    int* stage_ok = reinterpret_cast<int*>(smem + ly.stage_ok());
+    float* scratch = reinterpret_cast<float*>(smem + ly.scratch());
+    float* mbuf = reinterpret_cast<float*>(smem + ly.mbuf());
+    int* misc = reinterpret_cast<int*>(smem + ly.misc());
+    int* lens_s = reinterpret_cast<int*>(smem + ly.lens());
+    int* pre = reinterpret_cast<int*>(smem + ly.pre());
+    volatile int* abort_flag = misc + 0;
+    volatile int* last_flag = misc + 1;
+    int* wsum = misc + 32;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto desc_at = [&](int slot) {
+        return reinterpret_cast<UnitDesc*>(ring + slot * (sizeof(UnitDesc) + LY::QB));
+    };
+    auto q_at = [&](int slot) {
+        return reinterpret_cast<T*>(ring + slot * (sizeof(UnitDesc) + LY::QB) + sizeof(UnitDesc));
+    };
+
+    if (tid == 0) {
+        for (int k = 0; k < p.nstage; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, 1);
+        }
+        for (int k = 0; k < NUR; ++k) {
+            mbar_init(ufull + k, 1);
+            mbar_init(uempty + k, 1);
+        }
+        misc[0] = 0;
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == NCW && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+    }
+
+    // ---- prefix sums of partitions per sequence (each CTA, tiny)
+    {
+        const int per = (p.S + NT - 1) / NT;
+        const int beg = min(p.S, tid * per), end = min(p.S, beg + per);
+        int local = 0;
+        for (int k = beg; k < end; ++k) {
+            const int L = clamp_len(__ldg(p.lens + k), p);
+            lens_s[k] = L;
+            local += n_parts(L, p.P);
+        }
+        int incl = local;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int v = (lane < NCW + 1) ? wsum[lane] : 0;
+            int iv = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, iv, off);
+                if (lane >= off) iv += u;
+            }
+            if (lane < NCW + 1) wsum[lane] = iv - v;     // exclusive warp offsets
+        }
+        __syncthreads();
+        int run = wsum[warp] + incl - local;
+        for (int k = beg; k < end; ++k) {
+            pre[k] = run;
+            run += n_parts(lens_s[k], p.P);
+        }
+        if (tid == NT - 1) pre[p.S] = run;
+    }
+    __syncthreads();
+    const int U = pre[p.S] * p.Hkv;
+
+    if (warp == NCW) {
+        // ================================================= producer warp
+        const uint64_t policy = policy_evict_first();
+        const size_t qrow = (size_t)p.Hq * D * E;
+        int gstage = 0, ucount = 0;
+        bool ok = true;
+        while (ok) {
+            int u = 0;
+            if (lane == 0) u = atomicAdd(&p.hdr->next_unit, 1);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            const int slot = ucount % NUR;
+            if (ucount >= NUR) {
+                bool w = true;
+                if (lane == 0) w = wait_or_abort(uempty + slot, ((ucount / NUR) - 1) & 1, abort_flag, p.err);
+                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+            }
+            UnitDesc* d = desc_at(slot);
+            if (u >= U) {
+                if (lane == 0) {
+                    d->end = 1;
+                    mbar_arrive(ufull + slot);
+                }
+                ++ucount;
+                break;
+            }
+            const int x = u / p.Hkv;
+            int lo = 0, hi = p.S;                      // pre[lo] <= x < pre[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pre[mid] <= x) lo = mid; else hi = mid;
+            }
+            const int s = lo, i = x - pre[s], j = u - x * p.Hkv;
+            const int L = lens_s[s];
+            const int t0 = min(i * p.P, L), t1 = min(t0 + p.P, L);
+            const int nst = (t1 - t0 + TOK - 1) / TOK;
+            if (lane == 0) {
+                d->s = s; d->j = j; d->i = i; d->t0 = t0; d->t1 = t1;
+                d->n_p = n_parts(L, p.P);
+                d->stage_base = gstage; d->n_stages = nst; d->end = 0;
+                mbar_arrive_expect_tx(ufull + slot, G * D * E);
+                bulk_g2s(q_at(slot),
+                         reinterpret_cast<const uint8_t*>(p.q) + (size_t)s * qrow + (size_t)j * G * D * E,
+                         G * D * E, ufull + slot);
+            }
+            ++ucount;
+            // block ids of this unit, 32 at a time, one lane each
+            const int32_t* trow = p.tables + (size_t)s * p.mbps;
+            const int b0 = t0 / p.bs;
+            const int b_end = (t1 + p.bs - 1) / p.bs;
+            int win = 0;                                // first block id index in `ids`
+            int ids = (lane < b_end - b0) ? __ldg(trow + b0 + lane) : -1;
+            for (int c = 0; c < nst && ok; ++c) {
+                const int tok0 = t0 + c * TOK;
+                const int nv = min(TOK, t1 - tok0);
+                const int st = gstage % p.nstage;
+                if (gstage >= p.nstage) {
+                    bool w = true;
+                    if (lane == 0) w = wait_or_abort(empty + st, ((gstage / p.nstage) - 1) & 1, abort_flag, p.err);
+                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+                }
+                // block of each 8- or 16-token piece
+                const int npiece = (p.bs >= TOK) ? 1 : TOK / p.bs;
+                int blk[2] = {-1, -1}, off[2] = {0, 0}, rows[2] = {0, 0};
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    if (k < npiece) {
+                        const int tok = tok0 + k * p.bs;
+                        const int bi = tok / p.bs - b0;
+                        if (bi - win >= 32) {           // advance the id window
+                            win += 32;
+                            ids = (lane + win < b_end - b0) ? __ldg(trow + b0 + win + lane) : -1;
+                        }
+                        const int id = __shfl_sync(0xffffffffu, ids, (bi - win) & 31);
+                        if (tok < t1) {
+                            blk[k] = id;
+                            off[k] = tok % p.bs;
+                            rows[k] = (p.bs >= TOK) ? TOK : p.bs;
+                        }
+                    }
+                }
+                if (lane == 0) {
+                    bool valid = true;
+                    uint32_t bytes = 0;
+                    for (int k = 0; k < npiece; ++k) {
+                        if (rows[k] == 0) continue;
+                        if (blk[k] < 0 || blk[k] >= p.NB) valid = false;
+                        bytes += 2u * rows[k] * LY::ROWB;
+                    }
+                    stage_ok[st] = valid ? 1 : 0;
+                    uint8_t* Kd = stages + (size_t)st * LY::STAGE_BYTES;
+                    uint8_t* Vd = Kd + LY::KV_BYTES;
+                    if (!valid) {
+                        set_err(p.err, PA_DEV_BAD_BLOCK);
+                        mbar_arrive(full + st);
+                    } else {
+                        mbar_arrive_expect_tx(full + st, bytes);
+                        for (int k = 0; k < npiece; ++k) {
+                            if (rows[k] == 0) continue;
+                            const int y = (blk[k] * p.Hkv + j) * p.bs + off[k];
+                            const int rofs = k * p.bs * 128;      // piece row offset in a box
+#pragma unroll
+                            for (int b = 0; b < LY::NBOX; ++b) {
+                                tma_load_2d(Kd + b * BOXB + rofs, &kmap, b * BOX_ELEMS, y, full + st, policy);
+                                tma_load_2d(Vd + b * BOXB + rofs, &vmap, b * BOX_ELEMS, y, full + st, policy);
+                            }
+                        }
+                    }
+                    (void)nv;
+                }
+                ++gstage;
+            }
+        }
+        // make sure no copy of this CTA is still landing in shared memory
+        if (lane == 0) {
+            const int first = max(0, gstage - p.nstage);
+            for (int g = first; g < gstage; ++g) mbar_wait(full + g % p.nstage, (g / p.nstage) & 1);
+            const int ufirst = max(0, ucount - NUR);
+            for (int k = ufirst; k < ucount; ++k) mbar_wait(ufull + k % NUR, (k / NUR) & 1);
+        }
+    } else {
+        // ================================================= consumer warps
+        Engine eng;
+        float* xs = scratch + warp * 2 * G * TOK;
+        float* ps = xs + G * TOK;
+        int ucount = 0;
+        while (true) {
+            const int slot = ucount % NUR;
+            if (!wait_or_abort(ufull + slot, (ucount / NUR) & 1, abort_flag, p.err)) break;
+            const UnitDesc d = *desc_at(slot);
+            if (d.end) break;
+            eng.begin_unit(q_at(slot), lane, p.scale_log2e);
+            for (int c = warp; c < d.n_stages; c += NCW) {
+                const int g = d.stage_base + c;
+                const int st = g % p.nstage;
+                const bool have = wait_or_abort(full + st, (g / p.nstage) & 1, abort_flag, p.err);
+                if (have && stage_ok[st]) {
+                    const int nv = min(TOK, d.t1 - (d.t0 + c * TOK));
+                    uint8_t* Ks = stages + (size_t)st * LY::STAGE_BYTES;
+                    if constexpr (MMA) {
+                        eng.stage(Ks, Ks + LY::KV_BYTES, nv, p.scale_log2e, lane);
+                        if (nv < TOK) fence_proxy_async_smem();
+                    } else {
+                        eng.stage(Ks, Ks + LY::KV_BYTES, nv, xs, ps, lane);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + st);
+            }
+            // ---- merge the warps' states of this unit
+            float* mb = mbuf + (size_t)(ucount & 1) * NCW * G * (D + 2);
+            eng.dump(mb + (size_t)warp * G * (D + 2), lane);   // m=-inf, l=0, o=0 if no stage
+            named_bar_sync(1, CT);
+            if (tid == 0) mbar_arrive(uempty + slot);   // q and the descriptor are consumed
+            const size_t sj = (size_t)d.s * p.Hkv + d.j;
+            for (int idx = tid; idx < G * D; idx += CT) {
+                const int g = idx / D, dd = idx % D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < NCW; ++w) M = fmaxf(M, mb[(w * G + g) * (D + 2)]);
+                float Lsum = 0.f, O = 0.f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < NCW; ++w) {
+                        const float* e = mb + (w * G + g) * (D + 2);
+                        const float f = exp2f(e[0] - M);
+                        Lsum += e[1] * f;
+                        O += e[2 + dd] * f;
+                    }
+                }
+                if (d.n_p == 1) {
+                    T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.s * p.Hq + (size_t)d.j * G + g) * D + dd;
+                    *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+                } else {
+                    const size_t pi = (sj * p.n_pmax + d.i) * G + g;
+                    p.part_o[pi * D + dd] = O;
+                    if (dd == 0) {
+                        p.part_ml[pi * 2 + 0] = M;
+                        p.part_ml[pi * 2 + 1] = Lsum;
+                    }
+                }
+            }
+            if (d.n_p > 1) {
+                __threadfence();
+                named_bar_sync(1, CT);
+                if (tid == 0) {
+                    const int prev = atomicAdd(p.counters + sj, 1);
+                    const int last = (prev == d.n_p - 1);
+                    if (last) p.counters[sj] = 0;      // every partition has arrived
+                    *last_flag = last;
+                }
+                named_bar_sync(1, CT);
+                if (*last_flag) {
+                    __threadfence();
+                    const size_t base = sj * p.n_pmax;
+                    for (int idx = tid; idx < G * D; idx += CT) {
+                        const int g = idx / D, dd = idx % D;
+                        float M = -INFINITY;
+                        for (int i = 0; i < d.n_p; ++i)
+                            M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
+                        float Lsum = 0.f, O = 0.f;
+                        if (M != -INFINITY) {
+                            int i = 0;
+                            for (; i + 4 <= d.n_p; i += 4) {
+                                float mm[4], ll[4], oo[4];
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const size_t pi = (base + i + k) * G + g;
+                                    mm[k] = __ldcg(p.part_ml + pi * 2);
+                                    ll[k] = __ldcg(p.part_ml + pi * 2 + 1);
+                                    oo[k] = __ldcg(p.part_o + pi * D + dd);
+                                }
+#pragma unroll
+                                for (int k = 0; k < 4; ++k) {
+                                    const float f = exp2f(mm[k] - M);
+                                    Lsum += ll[k] * f;
+                                    O += oo[k] * f;
+                                }
+                            }
+                            for (; i < d.n_p; ++i) {
+                                const size_t pi = (base + i) * G + g;
+                                const float f = exp2f(__ldcg(p.part_ml + pi * 2) - M);
+                                Lsum += __ldcg(p.part_ml + pi * 2 + 1) * f;
+                                O += __ldcg(p.part_o + pi * D + dd) * f;
+                            }
+                        }
+                        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.s * p.Hq + (size_t)d.j * G + g) * D + dd;
+                        *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+                    }
+                }
+            }
+            ++ucount;
+        }
+    }
+
+    __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const int done = atomicAdd(&p.hdr->done_ctas, 1);
+        if (done == (int)gridDim.x - 1) {
+            p.hdr->next_unit = 0;
+            p.hdr->done_ctas = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ------------------------------------------------------------ host side
+namespace {
+
+int g_engine = PA_ENGINE_AUTO;
+std::mutex g_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Tensor map over a cache viewed as [num_blocks*Hkv*bs rows][D columns]; box =
+// 128 bytes x box_rows, 128B swizzle.
+int make_map(CUtensorMap* map, const void* base, pa_dtype dt, int D, int64_t rows, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return PA_ERR_CUDA;
+    const int esz = (int)dtype_size(dt);
+    CUtensorMapDataType t = dt == PA_F32   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                            : dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * esz};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, t, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+struct DevInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+int dev_info(DevInfo* out) {
+    static DevInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!have[dev]) {
+        if (cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&cache[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess)
+            return PA_ERR_CUDA;
+        have[dev] = true;
+    }
+    *out = cache[dev];
+    return PA_OK;
+}
+
+constexpr int kMaxStages = 24;
+
+size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
+    size_t b = sizeof(WsHeader);
+    b += (((size_t)S * Hkv * 4 + 255) / 256) * 256;
+    if (n_pmax > 1) {
+        b += (((size_t)S * Hq * n_pmax * 2 * 4 + 255) / 256) * 256;
+        b += (size_t)S * Hq * n_pmax * D * 4;
+    }
+    return b;
+}
+
+struct Launch {
+    CUtensorMap kmap, vmap;
+    DecodeParams p;
+    dim3 grid;
+    int threads;
+    size_t smem;
+    cudaStream_t stream;
+};
+
+template <typename T, int D, int G, int NCW, bool MMA>
+int run_decode(Launch& L, const DevInfo& di) {
+    using LY = Layout<T, D, G, NCW>;
+    auto kern = decode_kernel<T, D, G, NCW, MMA>;
+    const size_t fixed = LY::fixed_bytes(L.p.S) + 1024;   // + alignment slack
+    if ((size_t)di.smem_optin < fixed + (size_t)(NCW + 2) * LY::STAGE_BYTES) return PA_ERR_UNSUPPORTED;
+    int nstage = (int)((di.smem_optin - fixed) / LY::STAGE_BYTES);
+    nstage = std::min(nstage, kMaxStages);
+    L.p.nstage = nstage;
+    L.smem = LY(nstage, L.p.S).total() + 1024;
+    L.threads = (NCW + 1) * 32;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev & 63]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.smem_optin) !=
+            cudaSuccess)
+            return PA_ERR_CUDA;
+        attr_set[dev & 63] = true;
+    }
+    kern<<<L.grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D, int G>
+int dispatch_engine(Launch& L, const DevInfo& di, bool mma) {
+    if constexpr (sizeof(T) == 2) {
+        if (mma) return run_decode<T, D, G, 8, true>(L, di);
+    }
+    return run_decode<T, D, G, 8, false>(L, di);
+}
+
+template <typename T, int D>
+int dispatch_group(Launch& L, const DevInfo& di, int G, bool mma) {
+    switch (G) {
+        case 1: return dispatch_engine<T, D, 1>(L, di, mma);
+        case 2: return dispatch_engine<T, D, 2>(L, di, mma);
+        case 4: return dispatch_engine<T, D, 4>(L, di, mma);
+        case 8: return dispatch_engine<T, D, 8>(L, di, mma);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+int dispatch_dim(Launch& L, const DevInfo& di, int D, int G, bool mma) {
+    switch (D) {
+        case 64: return dispatch_group<T, 64>(L, di, G, mma);
+        case 128: return dispatch_group<T, 128>(L, di, G, mma);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+}  // namespace
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+int pa_set_decode_engine(int engine) {
+    if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_MMA) return PA_ERR_INVALID;
+    std::lock_guard<std::mutex> lk(g_mu);
+    const int prev = g_engine;
+    g_engine = engine;
+    return prev;
+}
+
+int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                             int max_context_len, int partition_size, size_t* bytes) {
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_context_len < 0 || partition_size < 0 || (partition_size % TOK) != 0 ||
+        num_q_heads % num_kv_heads != 0)
+        return PA_ERR_INVALID;
+    const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
+    const int n_pmax = std::max(1, (max_context_len + P - 1) / P);
+    *bytes = ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, n_pmax);
+    return PA_OK;
+}
+
+int pa_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < sizeof(WsHeader)) return PA_ERR_INVALID;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
+
+int pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+              const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+              int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int num_blocks, float scale, int partition_size, void* workspace,
+              size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag, void* stream) {
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
+        !workspace)
+        return PA_ERR_INVALID;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0 ||
+        partition_size % TOK != 0 || num_q_heads % num_kv_heads != 0)
+        return PA_ERR_INVALID;
+    if (dtype != PA_F32 && dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
+        block_size != 128)
+        return PA_ERR_UNSUPPORTED;
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return PA_ERR_INVALID;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (rows >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    size_t need = 0;
+    pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                             partition_size, &need);
+    if (workspace_bytes < need) return PA_ERR_INVALID;
+    const int G = num_q_heads / num_kv_heads;
+
+    DevInfo di;
+    if (dev_info(&di) != PA_OK) return PA_ERR_CUDA;
+    // the per-CTA prefix array must leave room for the pipeline
+    if (num_seqs > 16384) return PA_ERR_UNSUPPORTED;
+
+    static thread_local Launch L;
+    const int box_rows = block_size >= TOK ? TOK : block_size;
+    int st = make_map(&L.kmap, key_cache, dtype, head_dim, rows, box_rows);
+    if (st == PA_OK) st = make_map(&L.vmap, value_cache, dtype, head_dim, rows, box_rows);
+    if (st != PA_OK) return st;
+
+    const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
+    const int n_pmax = std::max(1, (max_context_len + P - 1) / P);
+    DecodeParams& p = L.p;
+    p.out = out;
+    p.q = query;
+    p.tables = block_tables;
+    p.lens = context_lens;
+    p.mbps = max_blocks_per_seq;
+    p.max_len = max_context_len;
+    p.S = num_seqs;
+    p.Hq = num_q_heads;
+    p.Hkv = num_kv_heads;
+    p.NB = num_blocks;
+    p.bs = block_size;
+    p.P = P;
+    p.n_pmax = n_pmax;
+    p.scale_log2e = scale * 1.4426950408889634f;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.hdr = reinterpret_cast<WsHeader*>(ws);
+    p.counters = reinterpret_cast<int*>(ws + sizeof(WsHeader));
+    const size_t cnt_bytes = (((size_t)num_seqs * num_kv_heads * 4 + 255) / 256) * 256;
+    p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader) + cnt_bytes);
+    p.part_o = p.part_ml + ((((size_t)num_seqs * num_q_heads * n_pmax * 2 * 4 + 255) / 256) * 256) / 4;
+    p.err = err_flag;
+
+    const int64_t units_ub = (int64_t)num_seqs * num_kv_heads * n_pmax;
+    L.grid = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(units_ub, di.sms)));
+    L.stream = (cudaStream_t)stream;
+
+    int engine;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        engine = g_engine;
+    }
+    const bool mma = dtype != PA_F32 && engine != PA_ENGINE_CUDA_CORE;
+    if (engine == PA_ENGINE_MMA && dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+    switch (dtype) {
+        case PA_F32: return dispatch_dim<float>(L, di, head_dim, G, false);
+        case PA_F16: return dispatch_dim<__half>(L, di, head_dim, G, mma);
+        case PA_BF16: return dispatch_dim<__nv_bfloat16>(L, di, head_dim, G, mma);
+    }
+    return PA_ERR_INVALID;
+}
+
+}  // extern "C"

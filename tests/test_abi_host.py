@@ -1,0 +1,179 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/pa.h declares, rejects bad arguments before launching anything, and
+its host block manager reproduces the oracle's block tables, slot mappings and
+copy-on-write pairs bit for bit on every workload script."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pa = pytest.importorskip("paged_kv_cache_426_b200")
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "pa.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 20
+    lib = C.CDLL(pa.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(names) == set(pa.SIGNATURES), "binding and header disagree"
+
+
+def test_status_strings_and_version():
+    assert pa.lib.pa_status_string(pa.PA_ERR_OOM) == b"PA_ERR_OOM"
+    assert pa.lib.pa_version() >= 100
+
+
+def test_bad_arguments_rejected_before_launch():
+    L = pa.lib
+    # null pointers
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 4, 2, 128, 16, 8, 1, None, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(None, None, None, None, None, 4, None, 64, 2, 4, 2, 128, 16, 8, 1.0, 0,
+                       None, 0, 1, None, None) == pa.PA_ERR_INVALID
+    assert L.pa_copy_blocks(None, None, None, 3, 2, 128, 16, 8, 1, None, None) == pa.PA_ERR_INVALID
+    # unsupported shapes
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 4, 2, 96, 16, 8, 1, None, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_copy_blocks(None, None, None, 3, 2, 128, 12, 8, 1, None, None) == pa.PA_ERR_UNSUPPORTED
+    fake = 1 << 20   # never dereferenced: validation fails first
+    assert L.pa_decode(fake, fake, fake, fake, fake, 4, fake, 64, 2, 4, 2, 96, 16, 8, 1.0, 0,
+                       fake, 1 << 20, 1, None, None) == pa.PA_ERR_UNSUPPORTED
+    # group not dividing, partition not a multiple of 16, bad dtype, short workspace
+    assert L.pa_decode(fake, fake, fake, fake, fake, 4, fake, 64, 2, 6, 4, 128, 16, 8, 1.0, 0,
+                       fake, 1 << 20, 1, None, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(fake, fake, fake, fake, fake, 4, fake, 64, 2, 4, 2, 128, 16, 8, 1.0, 24,
+                       fake, 1 << 20, 1, None, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(fake, fake, fake, fake, fake, 4, fake, 64, 2, 4, 2, 128, 16, 8, 1.0, 0,
+                       fake, 1 << 20, 7, None, None) == pa.PA_ERR_INVALID
+    assert L.pa_decode(fake, fake, fake, fake, fake, 4, fake, 4096, 2, 4, 2, 128, 16, 8, 1.0, 16,
+                       fake, 300, 1, None, None) == pa.PA_ERR_INVALID
+    # empty work is a no-op
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 2, 128, 16, 8, 1, None, None) == pa.PA_OK
+    assert L.pa_copy_blocks(None, None, None, 0, 2, 128, 16, 8, 1, None, None) == pa.PA_OK
+
+
+def test_workspace_size_formula():
+    # scheduler header + counters only when nothing is split
+    n0 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 0)
+    assert n0 == 256 + 64 * 32 * 4
+    n1 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 512)
+    n_p = 5
+    assert n1 == 256 + 64 * 32 * 4 + 64 * 32 * n_p * 2 * 4 + 64 * 32 * n_p * 128 * 4
+
+
+def test_allocator_errors():
+    a = pa.BlockAllocator(3, [2, 0])
+    assert a.refcount(1) == 1
+    assert a.allocate_block() == 2 and a.allocate_block() == 0
+    with pytest.raises(pa.PAError) as e:
+        a.allocate_block()
+    assert e.value.status == pa.PA_ERR_OOM
+    a.free_block(2)
+    with pytest.raises(pa.PAError) as e:
+        a.free_block(2)
+    assert e.value.status == pa.PA_ERR_STATE
+    with pytest.raises(pa.PAError):
+        pa.BlockAllocator(3, [1, 1])
+
+
+def test_append_is_all_or_nothing():
+    a = pa.BlockAllocator(3)
+    m = pa.BlockManager(a, 4)
+    m.add_seq(0)
+    m.append(0, 10)                       # 3 blocks
+    before = (m.seq_len(0), a.num_free())
+    with pytest.raises(pa.PAError) as e:
+        m.append(0, 3)                    # needs a 4th block at the 13th token
+    assert e.value.status == pa.PA_ERR_OOM
+    assert (m.seq_len(0), a.num_free()) == before
+    m.add_seq(1)
+    m.fork(0, 2)
+    with pytest.raises(pa.PAError):
+        m.append_step([0, 2, 1])          # 0 copies its shared last block: no free block
+    assert m.seq_len(0) == 10 and m.seq_len(2) == 10 and m.seq_len(1) == 0
+    assert [a.refcount(b) for b in range(3)] == [2, 2, 2]
+
+
+def test_beam_sharing_example_matches_page():
+    """velog 메모리 공유 example, through the C++ manager."""
+    from tests.conftest import golden
+    fx = golden("velog_beam_sharing.json")
+    a = pa.BlockAllocator(fx["num_blocks"], fx["free_order"])
+    m = pa.BlockManager(a, fx["block_size"])
+    m.add_seq(0)
+    m.append(0, fx["prompt_tokens"])
+    m.fork(0, 1)
+    _, c0 = m.append(0)
+    _, c1 = m.append(1)
+    tab, _ = m.block_tables([0, 1], 4)
+    assert tab[0, :3].tolist() == fx["expect_tables"]["A"]
+    assert tab[1, :3].tolist() == fx["expect_tables"]["B"]
+    for b, rc in fx["expect_refcounts"].items():
+        assert a.refcount(int(b)) == rc
+    assert c0 == [] and c1 == []
+    m.free_seq(0)
+    m.free_seq(1)
+    assert a.num_free() == fx["num_blocks"]
+
+
+def _replay(w, steps=None):
+    """C++ manager through the workload script; compare with the oracle's record."""
+    rec = oracle.run(w, decode=False, steps=steps)
+    a = pa.BlockAllocator(w.num_blocks, w.free_order)
+    m = pa.BlockManager(a, w.block_size)
+    mb = oracle.max_blocks_needed(w)
+    k = 0
+    for op in w.ops:
+        if op[0] == "add":
+            m.add_seq(op[1])
+        elif op[0] == "fork":
+            m.fork(op[1], op[2])
+        elif op[0] == "write":
+            slots, cow = m.append(op[1], w.kv["k" + op[2]].shape[0])
+            assert np.array_equal(slots.numpy(), rec.prefill_slots[(op[1], op[2])])
+        elif op[0] == "step":
+            if k >= len(rec.steps):
+                break
+            st = rec.steps[k]
+            slots, cow = m.append_step(op[1])
+            assert np.array_equal(slots.numpy(), st.slot_mapping)
+            assert [tuple(c) for c in cow.tolist()] == [tuple(c) for c in st.cow_pairs]
+            tab, lens = m.block_tables(op[1], mb)
+            assert np.array_equal(tab.numpy(), st.block_tables)
+            assert np.array_equal(lens.numpy(), st.context_lens)
+            k += 1
+    for b in range(w.num_blocks):
+        assert a.refcount(b) == rec.manager.alloc.refcount[b]
+    assert a.num_free() == rec.manager.alloc.num_free()
+    return m, a, rec
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny_f32", {}),
+    ("mha7b_f16", dict(steps=32)),
+    ("gqa8b_bf16_bs16", {}),
+    ("gqa8b_bf16_bs32", {}),
+    ("prefix_f16", {}),
+    ("prefix_f16", dict(duplicate_prefix=True)),
+])
+def test_manager_matches_oracle(name, kw):
+    w = workloads.make(name, **kw)
+    m, a, rec = _replay(w)
+    # every sequence freed -> all references back to the outside holders only
+    for s in list(rec.manager.tables):
+        m.free_seq(s)
+    held = w.num_blocks - len(w.free_order)
+    assert a.num_free() == w.num_blocks - held

@@ -1,0 +1,318 @@
+"""GPU parity: the CUDA path against the float64 oracle on the same seeded inputs.
+
+* cache writes and copy-on-write copies: bit-exact over the whole caches
+  (untouched slots keep their previous bits);
+* host metadata (slot mappings, copy pairs, block tables): equal to the
+  oracle's;
+* decode outputs: fp32 max-abs 1e-5; fp16/bf16 |gpu - ref| <= 3e-3 + 1e-2 |ref|
+  element-wise, plus a per-(sequence, head) normalised L2 error <= 5e-3 (fp16)
+  / 1e-2 (bf16).
+
+Small variants of the five workloads are compared element by element (they
+span several stages, partitions and a ragged tail); the full-size workloads,
+in the launch configuration the benchmark times, are compared on sampled
+(sequence, head) outputs that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.harness import (GpuRun, check_close, oracle_sampled, out_f64, sample_pairs,
+                           to_torch_storage)
+
+pytestmark = pytest.mark.gpu
+pa = pytest.importorskip("paged_kv_cache_426_b200")
+
+ENGINES = {"auto": 0, "core": 1}
+
+
+@pytest.fixture(params=list(ENGINES))
+def engine(request):
+    prev = pa.pa_set_decode_engine(ENGINES[request.param])
+    yield request.param
+    pa.pa_set_decode_engine(prev)
+
+
+def run_full_compare(w, partition_size=None, steps=None):
+    rec = oracle.run(w, keep_prefill_cache=True, steps=steps)
+    g = GpuRun(w, rec, partition_size=partition_size)
+    g.replay_prefill()
+    errs = []
+    for k in range(len(rec.steps)):
+        out = g.step(k)
+        errs.append(check_close(out_f64(out, w.dtype), rec.steps[k].out, w.dtype,
+                                f"{w.name} step {k} P={g.P}"))
+    assert g.caches_equal_oracle(), "caches differ from the oracle after the steps"
+    return errs
+
+
+# ---------------------------------------------------------------- element by element
+
+@pytest.mark.parametrize("P", [0, 16, 32])
+def test_tiny_f32(engine, P):
+    run_full_compare(workloads.tiny_f32(), partition_size=P)
+
+
+@pytest.mark.parametrize("P", [0, 64, 512])
+def test_mha_f16_small(engine, P):
+    run_full_compare(workloads.mha7b_f16(steps=3, num_seqs=5), partition_size=P)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_gqa_bf16_small(engine, bs):
+    run_full_compare(workloads.gqa8b_bf16(block_size=bs, num_seqs=10), partition_size=512)
+
+
+def test_prefix_f16_small(engine):
+    w = workloads.prefix_f16(n_req=6, plen=64, suffix_max=40, n_fork=2, heads=4)
+    run_full_compare(w, partition_size=32)
+
+
+def test_long_bf16_small(engine):
+    w = workloads.custom("bf16", [3001, 4096, 1500], 32, 8, 128, 64, seed=77,
+                         partition_size=512)
+    run_full_compare(w)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_shapes_and_groups(engine, dtype, d, G):
+    hkv = 2
+    w = workloads.custom(dtype, [1, 15, 16, 17, 100, 257], hkv * G, hkv, d, 16, seed=G * d,
+                         partition_size=64)
+    run_full_compare(w)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
+def test_block_sizes(engine, bs):
+    w = workloads.custom("f16", [3, 8, 9, 129, 300], 8, 2, 128, bs, seed=bs, partition_size=128)
+    run_full_compare(w)
+
+
+# ---------------------------------------------------------------- invariances
+
+def _decode_outputs(w, P, engine_id=0):
+    prev = pa.pa_set_decode_engine(engine_id)
+    try:
+        rec = oracle.run(w, keep_prefill_cache=True, decode=False)
+        g = GpuRun(w, rec, partition_size=P)
+        g.replay_prefill()
+        return [g.step(k).cpu() for k in range(len(rec.steps))], rec
+    finally:
+        pa.pa_set_decode_engine(prev)
+
+
+def test_block_size_invariance_bit_identical():
+    """Same logical K/V, block 16 vs 32, different fragmented pools."""
+    a, _ = _decode_outputs(workloads.gqa8b_bf16(block_size=16, num_seqs=12), 512)
+    b, _ = _decode_outputs(workloads.gqa8b_bf16(block_size=32, num_seqs=12), 512)
+    assert torch.equal(a[0], b[0])
+
+
+def test_physical_permutation_invariance_bit_identical():
+    w1 = workloads.mha7b_f16(steps=2, num_seqs=4)
+    w2 = workloads.mha7b_f16(steps=2, num_seqs=4)
+    w2.free_order = list(reversed(w2.free_order))
+    a, _ = _decode_outputs(w1, 64)
+    b, _ = _decode_outputs(w2, 64)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_shared_vs_duplicated_prefix_bit_identical():
+    kw = dict(n_req=6, plen=64, suffix_max=40, n_fork=2, heads=4)
+    a, ra = _decode_outputs(workloads.prefix_f16(**kw), 32)
+    b, rb = _decode_outputs(workloads.prefix_f16(duplicate_prefix=True, **kw), 32)
+    assert torch.equal(a[0], b[0])
+    # the shared layout really holds fewer blocks
+    assert ra.manager.alloc.num_free() > rb.manager.alloc.num_free()
+
+
+@pytest.mark.parametrize("P", [16, 512, 1024, 2048])
+def test_partition_sizes_agree(P):
+    w = workloads.custom("bf16", [5000, 2049, 77], 16, 4, 128, 32, seed=3)
+    ref, _ = _decode_outputs(w, 0)
+    got, _ = _decode_outputs(w, P)
+    check_close(got[0].double().numpy(), ref[0].double().numpy(), "bf16", f"P={P} vs unsplit")
+
+
+def test_engines_agree():
+    w = workloads.gqa8b_bf16(num_seqs=8)
+    a, rec = _decode_outputs(w, 512, 1)
+    b, _ = _decode_outputs(w, 512, 0)
+    check_close(a[0].double().numpy(), b[0].double().numpy(), "bf16", "core vs mma")
+
+
+# ---------------------------------------------------------------- edge cases
+
+def _cache(NB, hkv, bs, d, dt, fill=0):
+    return torch.full((NB, hkv, bs, d), fill, dtype=dt, device="cuda")
+
+
+def test_zero_and_one_token():
+    d, hkv, G, bs = 128, 2, 4, 16
+    kc = torch.randn(4, hkv, bs, d, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(4, hkv, bs, d, device="cuda").to(torch.bfloat16)
+    q = torch.randn(3, hkv * G, d, device="cuda").to(torch.bfloat16)
+    tab = torch.tensor([[2, -1], [-1, -1], [1, 3]], dtype=torch.int32, device="cuda")
+    lens = torch.tensor([1, 0, 17], dtype=torch.int32, device="cuda")
+    ws = pa.alloc_workspace(3, hkv * G, hkv, d, 32, 16)
+    out = torch.full_like(q, float("nan"))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    for h in range(hkv * G):                       # one token: exactly its V row
+        assert torch.equal(out[0, h], vc[2, h // G, 0])
+    assert not out[1].any()                        # no token: zeros
+    ref = oracle.paged_decode(oracle.as_storage(q.cpu(), "bf16"), oracle.as_storage(kc.cpu(), "bf16"),
+                              oracle.as_storage(vc.cpu(), "bf16"), tab.cpu().numpy(),
+                              lens.cpu().numpy(), 0.1, "bf16")
+    check_close(out_f64(out[2:], "bf16"), ref[2:], "bf16", "17 tokens over two blocks")
+
+
+def test_max_context_fills_table_exactly():
+    w = workloads.custom("f16", [256, 255], 8, 8, 128, 16, seed=11, partition_size=64)
+    rec = oracle.run(w, keep_prefill_cache=True)
+    g = GpuRun(w, rec, max_blocks=16)            # 256 tokens = 16 blocks exactly
+    g.replay_prefill()
+    out = g.step(0)
+    check_close(out_f64(out, "f16"), rec.steps[0].out, "f16", "full table")
+
+
+def test_bad_block_id_sets_flag_without_fault():
+    d, bs = 128, 16
+    kc = torch.randn(4, 1, bs, d, device="cuda").half()
+    vc = torch.randn(4, 1, bs, d, device="cuda").half()
+    q = torch.randn(2, 1, d, device="cuda").half()
+    tab = torch.tensor([[0, 9], [1, 2]], dtype=torch.int32, device="cuda")   # 9 >= num_blocks
+    lens = torch.tensor([20, 20], dtype=torch.int32, device="cuda")
+    ws = pa.alloc_workspace(2, 1, 1, d, 32, 0)
+    out = torch.zeros_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEV_BAD_BLOCK
+    ref = oracle.paged_decode(oracle.as_storage(q.cpu(), "f16"), oracle.as_storage(kc.cpu(), "f16"),
+                              oracle.as_storage(vc.cpu(), "f16"), tab.cpu().numpy()[1:],
+                              lens.cpu().numpy()[1:], 0.1, "f16")
+    check_close(out_f64(out[1:], "f16"), ref, "f16", "the valid sequence is unaffected")
+    # the workspace is still usable: a clean call succeeds
+    err.zero_()
+    tab[0, 1] = 3
+    pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+
+
+def test_bad_length_is_clamped_and_flagged():
+    d = 64
+    kc = torch.randn(4, 1, 16, d, device="cuda")
+    vc = torch.randn(4, 1, 16, d, device="cuda")
+    q = torch.randn(1, 1, d, device="cuda")
+    tab = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
+    lens = torch.tensor([40], dtype=torch.int32, device="cuda")      # > 2 blocks * 16
+    ws = pa.alloc_workspace(1, 1, 1, d, 64, 0)
+    out = torch.zeros_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_decode(out, q, kc, vc, tab, lens, 64, 0.125, workspace=ws, err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEV_BAD_LEN
+    ref = oracle.paged_decode(q.cpu().numpy(), kc.cpu().numpy(), vc.cpu().numpy(),
+                              tab.cpu().numpy(), np.array([32]), 0.125, "f32")
+    check_close(out.double().cpu().numpy(), ref, "f32", "clamped to the table")
+
+
+# ---------------------------------------------------------------- cache ops
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("bs", [8, 16, 64])
+def test_reshape_and_cache_bit_exact(dtype, bs):
+    g = torch.Generator().manual_seed(bs)
+    NB, hkv, d, T = 9, 3, 128, 40
+    k = torch.randn(T, hkv, d, generator=g).to(dtype)
+    v = torch.randn(T, hkv, d, generator=g).to(dtype)
+    slots = torch.randperm(NB * bs, generator=g)[:T].to(torch.int64)
+    slots[5] = -1
+    name = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[dtype]
+    kc0 = oracle.empty_cache(NB, hkv, bs, d, name, fill=0x5A5A)
+    vc0 = oracle.empty_cache(NB, hkv, bs, d, name, fill=0x3C3C)
+    kc_gpu = to_torch_storage(kc0.copy(), name).cuda()
+    vc_gpu = to_torch_storage(vc0.copy(), name).cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_reshape_and_cache(k.cuda(), v.cuda(), kc_gpu, vc_gpu, slots.cuda(), err_flag=err)
+    oracle.reshape_and_cache(kc0, vc0, oracle.as_storage(k, name), oracle.as_storage(v, name),
+                             slots.numpy())
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert np.array_equal(oracle.as_storage(kc_gpu.cpu(), name).view(np.uint8), kc0.view(np.uint8))
+    assert np.array_equal(oracle.as_storage(vc_gpu.cpu(), name).view(np.uint8), vc0.view(np.uint8))
+
+
+def test_reshape_and_cache_bad_slot():
+    kc = torch.zeros(2, 1, 16, 64, device="cuda")
+    vc = torch.zeros_like(kc)
+    k = torch.ones(2, 1, 64, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_reshape_and_cache(k, k, kc, vc, torch.tensor([3, 32], device="cuda"), err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEV_BAD_SLOT
+    assert kc[0, 0, 3].eq(1).all() and kc.sum().item() == 64
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+def test_copy_blocks_bit_exact(dtype):
+    name = {torch.float32: "f32", torch.float16: "f16", torch.bfloat16: "bf16"}[dtype]
+    g = torch.Generator().manual_seed(1)
+    kc = torch.randn(12, 4, 16, 128, generator=g).to(dtype)
+    vc = torch.randn(12, 4, 16, 128, generator=g).to(dtype)
+    pairs = [(1, 7), (3, 0), (3, 11), (10, 2)]
+    kg, vg = kc.cuda(), vc.cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pa.pa_copy_blocks(kg, vg, torch.tensor(pairs, dtype=torch.int64, device="cuda"), err_flag=err)
+    ko, vo = oracle.as_storage(kc, name).copy(), oracle.as_storage(vc, name).copy()
+    oracle.copy_blocks(ko, vo, pairs)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert np.array_equal(oracle.as_storage(kg.cpu(), name).view(np.uint8), ko.view(np.uint8))
+    assert np.array_equal(oracle.as_storage(vg.cpu(), name).view(np.uint8), vo.view(np.uint8))
+    err.zero_()
+    pa.pa_copy_blocks(kg, vg, torch.tensor([[0, 12]], device="cuda"), err_flag=err)
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEV_BAD_PAIR
+
+
+# ---------------------------------------------------------------- full-size workloads
+
+FULL = [
+    ("mha7b_f16", dict(steps=32)),
+    ("gqa8b_bf16_bs16", {}),
+    ("gqa8b_bf16_bs32", {}),
+    ("prefix_f16", {}),
+    ("long_bf16", {}),
+]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,kw", FULL, ids=[f[0] for f in FULL])
+def test_full_size_sampled(name, kw):
+    """Full-size workload, the benchmark's launch configuration (its partition
+    size), every decode step; sampled outputs against the oracle one by one,
+    and the whole caches bit-exact after the last step."""
+    w = workloads.make(name, **kw)
+    rec = oracle.run(w, keep_prefill_cache=True, decode=False)
+    g = GpuRun(w, rec)
+    g.replay_prefill()
+    S, Hq = rec.steps[0].context_lens.shape[0], w.num_q_heads
+    for k in range(len(rec.steps)):
+        out = g.step(k)
+        if k in (0, len(rec.steps) - 1) or k % 8 == 0:
+            pairs = sample_pairs(S, Hq, 48, seed=k)
+            ref = oracle_sampled(w, rec, k, pairs)
+            got = out_f64(out, w.dtype)
+            for (s, h), r in ref.items():
+                check_close(got[s, h][None, None], r[None, None], w.dtype, f"{name} step {k} ({s},{h})")
+    assert g.caches_equal_oracle()

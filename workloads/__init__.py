@@ -208,20 +208,22 @@ def gqa8b_bf16(block_size: int = 16, steps: int = 1, num_seqs: int = 256,
                                      "in random order", sigma=sigma))
 
 
-def prefix_f16(steps: int = 1, duplicate_prefix: bool = False) -> Workload:
+def prefix_f16(steps: int = 1, duplicate_prefix: bool = False, n_req: int = 64,
+               plen: int = 1024, suffix_max: int = 256, n_fork: int = 16,
+               heads: int = 32) -> Workload:
     """Shared-prefix / parallel-sampling batch, fp16: 64 requests share one
     1024-token prefix; each then appends its own suffix of U{0..256} tokens;
     16 of them (a seeded choice) fork into beam width 4 (3 children each, so
     112 sequences); then decode steps in which every sequence appends one
     token.  32 = 32 heads, head dim 128, block 16, q/K/V ~ N(0,1), shuffled
     ids.  With ``duplicate_prefix`` every request writes its own copy of the
-    same prefix instead of sharing it (same logical K/V, other layout)."""
-    hq = hkv = 32
+    same prefix instead of sharing it (same logical K/V, other layout).  The
+    keyword sizes shrink the batch for element-by-element tests."""
+    hq = hkv = heads
     d, bs = 128, 16
     g = _gen(BASE_SEED + 4)
-    n_req, plen = 64, 1024
-    suffix = _uniform_int(g, 0, 256, n_req)
-    forkers = sorted(_perm(g, n_req)[:16])
+    suffix = _uniform_int(g, 0, suffix_max, n_req)
+    forkers = sorted(_perm(g, n_req)[:n_fork])
     kv = {"kprefix": _normal(g, (plen, hkv, d), "f16"),
           "vprefix": _normal(g, (plen, hkv, d), "f16")}
     for r in range(n_req):

@@ -125,9 +125,11 @@ int pa_decode(void* out, const void* query, const void* key_cache,
               size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
               void* stream);
 
-/* Decode engine selection (for measurement): PA_ENGINE_AUTO picks tensor-core
- * MMA for f16/bf16 and CUDA cores for f32; PA_ENGINE_CUDA_CORE forces the
- * CUDA-core dot products.  Process-wide; returns the previous value. */
+/* Decode engine selection (for measurement).  PA_ENGINE_AUTO and
+ * PA_ENGINE_CUDA_CORE use CUDA-core dot products.  PA_ENGINE_MMA uses
+ * m16n8k16 tensor-core MMAs; it is accepted only for f16/bf16 with
+ * num_q_heads == num_kv_heads (other shapes return PA_ERR_UNSUPPORTED).
+ * Process-wide; returns the previous value. */
 enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_MMA = 2 };
 int pa_set_decode_engine(int engine);
 

@@ -4,7 +4,7 @@ Argument marshalling only.  Every step of the hot path runs in the library's
 CUDA kernels (cache write, copy-on-write block copy, decode attention) or its
 C++ host code (block allocator, block tables); PyTorch supplies device memory
 and streams.  There is no fallback: importing this package fails if the
-library has not been built (``python -m paged_kv_cache_426_b200.build``).
+library has not been built (``python paged_kv_cache_426_b200/build.py``).
 
 The functions keep the C names (``pa_reshape_and_cache``, ``pa_decode``,
 ``pa_copy_blocks``, ...).  Tensor arguments give the pointers and the sizes;
@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_426_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python paged_kv_cache_426_b200/build.py` "
         "(nvcc, sm_100a).  There is no CPU or PyTorch fallback.")
 lib = C.CDLL(LIB_PATH)
 

@@ -1,6 +1,8 @@
 """Build libpa_b200.so in-tree with nvcc for sm_100a (B200).
 
-    python -m paged_kv_cache_426_b200.build [--force] [--ptxas-info]
+    python paged_kv_cache_426_b200/build.py [--force] [--ptxas-info]
+
+(run it as a script: importing the package needs the library already built)
 
 Objects go to ``_build/`` next to the package; the shared library lands in the
 package directory, where the binding loads it.  The CUDA runtime is linked

@@ -107,31 +107,39 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                  : "memory");
 }
 
+// try_wait with a suspend-time hint: the warp sleeps until the phase
+// completes (or the hint expires) instead of spinning.
+constexpr uint32_t kSuspendHintNs = 1000000u;   // 1 ms
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs and returns false (the caller records PA_DEV_TIMEOUT).
+// kWaitLimitNs and returns false (the caller records PA_DEV_TIMEOUT).  The
+// clock is read only every 64 unsuccessful probes.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+        if ((it & 63) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
     }
 }
 
+// Named barrier over `nthreads` threads.  The non-.aligned form: a warp may
+// reach it with its lanes out of step; __syncwarp first reconverges it.
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+    __syncwarp();
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- TMA

@@ -22,7 +22,8 @@
 //    (bs >= 16) or covers two (bs = 8).
 //  * Consumer warps take a unit's stages round-robin by logical stage index
 //    and keep a per-warp online softmax (running max m, sum l, output o) in
-//    the log2 domain.  Two compute engines:
+//    the log2 domain.  Two compute engines (CUDA cores by default; the
+//    tensor-core one on request, G = 1 only):
 //      CUDA cores: 8 (or 16) lanes per token, 16-byte loads, warp-shuffle
 //        reduce-scatter of the G dot products, then p*V with each lane owning
 //        head_dim/32 output columns of all G heads;
@@ -54,8 +55,13 @@
 
 namespace pa {
 
-constexpr int TOK = 16;       // tokens per pipeline stage
-constexpr int NUR = 8;        // unit-descriptor ring slots
+constexpr int TOK = 16;           // tokens per pipeline stage
+constexpr int NCONS = 2;          // consumer warps per pipeline (alternate stages)
+constexpr int PIPE_WARPS = 1 + NCONS;
+// independent producer/consumer pipelines per CTA: 4, or 2 when a stage is
+// 16 KB (fp32, head_dim 128) so that the rings still fit in shared memory
+template <typename T, int D> constexpr int pipes_for() { return sizeof(T) * D > 256 ? 2 : 4; }
+constexpr int NUR = 4;            // unit-descriptor slots per pipeline
 constexpr int BOXB = TOK * 128;   // bytes of one 16-row x 128-byte box
 
 struct alignas(16) UnitDesc {
@@ -73,7 +79,7 @@ struct DecodeParams {
     const void* q;
     const int32_t* tables;
     const int32_t* lens;
-    int mbps, max_len, S, Hq, Hkv, NB, bs, P, n_pmax, nstage;
+    int mbps, max_len, S, Hq, Hkv, NB, bs, bs_log2, P, n_pmax, nst;
     float scale_log2e;
     WsHeader* hdr;
     int* counters;     // [S*Hkv]
@@ -82,30 +88,40 @@ struct DecodeParams {
     int32_t* err;
 };
 
-// Shared-memory layout (dynamic, 1024-byte aligned base).
-template <typename T, int D, int G, int NCW>
+// Shared-memory layout (dynamic, 1024-byte aligned base).  Every pipeline has
+// its own stage ring, unit-descriptor ring, barriers, scratch and merge buffer.
+template <typename T, int D, int G>
 struct Layout {
+    static constexpr int NPIPE = pipes_for<T, D>();
+    static constexpr int NTHREADS = NPIPE * PIPE_WARPS * 32;
     static constexpr int E = sizeof(T);
     static constexpr int ROWB = D * E;               // bytes per token row
     static constexpr int NBOX = ROWB / 128;          // 128-byte boxes per row
     static constexpr int KV_BYTES = NBOX * BOXB;     // one stage of K (or V)
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int QB = ((G * D * E + 127) / 128) * 128;
-    static constexpr int RING_BYTES = NUR * (int)(sizeof(UnitDesc) + QB);
-    static constexpr int SCRATCH = NCW * 2 * G * TOK * 4;        // xs + ps
-    static constexpr int MBUF = 2 * NCW * G * (D + 2) * 4;       // double buffered
-    int nstage, S;
-    __host__ __device__ Layout(int nstage_, int S_) : nstage(nstage_), S(S_) {}
-    __host__ __device__ size_t ring() const { return (size_t)nstage * STAGE_BYTES; }
-    __host__ __device__ size_t bars() const { return ring() + RING_BYTES; }
-    __host__ __device__ size_t stage_ok() const { return bars() + (size_t)(2 * nstage + 2 * NUR) * 8; }
-    __host__ __device__ size_t scratch() const { return ((stage_ok() + 4 * nstage + 15) / 16) * 16; }
-    __host__ __device__ size_t mbuf() const { return scratch() + SCRATCH; }
-    __host__ __device__ size_t misc() const { return mbuf() + MBUF; }          // 64 ints
+    static constexpr int UNIT_BYTES = (int)sizeof(UnitDesc) + QB;
+    static constexpr int SCRATCH = NCONS * 2 * G * TOK * 4;      // per pipe: xs + ps
+    static constexpr int MBUF = NCONS * G * (D + 2) * 4;         // per pipe
+    int nst, S;                                                  // stages per pipe
+    __host__ __device__ Layout(int nst_, int S_) : nst(nst_), S(S_) {}
+    __host__ __device__ size_t ring(int pipe) const { return (size_t)pipe * nst * STAGE_BYTES; }
+    __host__ __device__ size_t units() const { return (size_t)NPIPE * nst * STAGE_BYTES; }
+    __host__ __device__ size_t unit(int pipe, int k) const {
+        return units() + (size_t)(pipe * NUR + k) * UNIT_BYTES;
+    }
+    __host__ __device__ size_t bars(int pipe) const {
+        return units() + (size_t)NPIPE * NUR * UNIT_BYTES + (size_t)pipe * (2 * nst + 2 * NUR) * 8;
+    }
+    __host__ __device__ size_t stage_ok(int pipe) const { return bars(NPIPE) + (size_t)pipe * nst * 4; }
+    __host__ __device__ size_t scratch(int pipe) const {
+        return ((stage_ok(NPIPE) + 15) / 16) * 16 + (size_t)pipe * SCRATCH;
+    }
+    __host__ __device__ size_t mbuf(int pipe) const { return scratch(NPIPE) + (size_t)pipe * MBUF; }
+    __host__ __device__ size_t misc() const { return mbuf(NPIPE); }              // 64 ints
     __host__ __device__ size_t lens() const { return misc() + 256; }
     __host__ __device__ size_t pre() const { return lens() + 4 * (size_t)S; }
     __host__ __device__ size_t total() const { return pre() + 4 * (size_t)(S + 1); }
-    static __host__ __device__ size_t fixed_bytes(int S_) { return Layout(0, S_).total(); }
 };
 
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -122,14 +138,16 @@ __device__ __forceinline__ int clamp_len(int L, const DecodeParams& p) {
 __device__ __forceinline__ int n_parts(int L, int P) { return max(1, ceil_div(L, P)); }
 
 // Bounded wait that also gives up as soon as another warp has given up.
+// mbar_try_wait sleeps until the phase completes (suspend hint), so the abort
+// flag and the clock are looked at only when a probe comes back empty.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag, int32_t* err) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    while (true) {
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if ((it & 63) == 0 && global_ns() - t0 > kWaitLimitNs) {
             set_err(err, PA_DEV_TIMEOUT);
             *abort_flag = 1;
             return false;
@@ -169,9 +187,9 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane) {
 // then V boxes; box b holds columns [b*128, b*128+128) bytes of 16 rows, with
 // the 16-byte chunk c of row r stored at chunk position c ^ (r & 7).
 
-template <typename T, int D, int G, int NCW>
+template <typename T, int D, int G>
 struct CoreEngine {
-    using LY = Layout<T, D, G, NCW>;
+    using LY = Layout<T, D, G>;
     static constexpr int E = sizeof(T);
     static constexpr int VEC = 16 / E;                       // elements per chunk
     static constexpr int CHUNKS = LY::ROWB / 16;             // chunks per row
@@ -317,7 +335,7 @@ struct CoreEngine {
     }
 };
 
-template <typename T, int D, int G, int NCW>
+template <typename T, int D, int G>
 struct MmaEngine {
     static_assert(sizeof(T) == 2, "tensor-core engine takes 16-bit types");
     static_assert(G <= 8, "query heads of a group must fit 8 MMA rows");
@@ -422,67 +440,66 @@ struct MmaEngine {
 };
 
 // ------------------------------------------------------------ the kernel
-template <typename T, int D, int G, int NCW, bool MMA>
-__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+// Warp roles: warp w belongs to pipeline w / PIPE_WARPS; role w % PIPE_WARPS is
+// 0 for the producer and 1..NCONS for the consumers.  The pipelines of a CTA
+// share nothing but the prefix sums and the abort flag; each takes its own
+// units from the global ticket counter.
+template <typename T, int D, int G, bool MMA>
+__global__ void __launch_bounds__(Layout<T, D, G>::NTHREADS, 1)
 decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
               DecodeParams p) {
-    using LY = Layout<T, D, G, NCW>;
-    using Engine = typename std::conditional<MMA, MmaEngine<T, D, G, NCW>,
-                                             CoreEngine<T, D, G, NCW>>::type;
-    constexpr int NT = (NCW + 1) * 32;
-    constexpr int CT = NCW * 32;                 // consumer threads
+    using LY = Layout<T, D, G>;
+    using Engine = typename std::conditional<MMA, MmaEngine<T, D, G>, CoreEngine<T, D, G>>::type;
+    constexpr int NPIPE = LY::NPIPE;
+    constexpr int NTHREADS = LY::NTHREADS;
+    constexpr int CT = NCONS * 32;               // consumer threads of a pipeline
     constexpr int E = sizeof(T);
     constexpr int BOX_ELEMS = 128 / E;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 128B-swizzled TMA boxes need 1024-byte aligned destinations
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const LY ly(p.nstage, p.S);
-    uint8_t* stages = smem;
-    uint8_t* ring = smem + ly.ring();
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars());
-    uint64_t* empty = full + p.nstage;
-    uint64_t* ufull = empty + p.nstage;
+    const LY ly(p.nst, p.S);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int pipe = warp / PIPE_WARPS, role = warp % PIPE_WARPS;
+    const int nst = p.nst;
+
+    uint8_t* stages = smem + ly.ring(pipe);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars(pipe));
+    uint64_t* empty = full + nst;
+    uint64_t* ufull = empty + nst;
     uint64_t* uempty = ufull + NUR;
-    int* stage_ok = reinterpret_cast<int*>(smem + ly.stage_ok());
-    float* scratch = reinterpret_cast<float*>(smem + ly.scratch());
-    float* mbuf = reinterpret_cast<float*>(smem + ly.mbuf());
+    int* stage_ok = reinterpret_cast<int*>(smem + ly.stage_ok(pipe));
+    float* scratch = reinterpret_cast<float*>(smem + ly.scratch(pipe));
+    float* mbuf = reinterpret_cast<float*>(smem + ly.mbuf(pipe));
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
     int* lens_s = reinterpret_cast<int*>(smem + ly.lens());
     int* pre = reinterpret_cast<int*>(smem + ly.pre());
     volatile int* abort_flag = misc + 0;
-    volatile int* last_flag = misc + 1;
+    volatile int* last_flag = misc + 1 + pipe;
     int* wsum = misc + 32;
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    auto desc_at = [&](int slot) {
-        return reinterpret_cast<UnitDesc*>(ring + slot * (sizeof(UnitDesc) + LY::QB));
-    };
-    auto q_at = [&](int slot) {
-        return reinterpret_cast<T*>(ring + slot * (sizeof(UnitDesc) + LY::QB) + sizeof(UnitDesc));
+    auto desc_at = [&](int k) { return reinterpret_cast<UnitDesc*>(smem + ly.unit(pipe, k)); };
+    auto q_at = [&](int k) {
+        return reinterpret_cast<T*>(smem + ly.unit(pipe, k) + sizeof(UnitDesc));
     };
 
     if (tid == 0) {
-        for (int k = 0; k < p.nstage; ++k) {
-            mbar_init(full + k, 1);
-            mbar_init(empty + k, 1);
+        for (int pp = 0; pp < NPIPE; ++pp) {
+            uint64_t* b = reinterpret_cast<uint64_t*>(smem + ly.bars(pp));
+            for (int k = 0; k < 2 * nst + 2 * NUR; ++k) mbar_init(b + k, 1);
         }
-        for (int k = 0; k < NUR; ++k) {
-            mbar_init(ufull + k, 1);
-            mbar_init(uempty + k, 1);
-        }
-        misc[0] = 0;
-        misc[1] = 0;
+        for (int k = 0; k < 32; ++k) misc[k] = 0;
         fence_barrier_init();
     }
-    if (warp == NCW && lane == 0) {
+    if (role == 0 && lane == 0 && pipe == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
 
     // ---- prefix sums of partitions per sequence (each CTA, tiny)
     {
-        const int per = (p.S + NT - 1) / NT;
+        constexpr int NW = NTHREADS / 32;
+        const int per = (p.S + NTHREADS - 1) / NTHREADS;
         const int beg = min(p.S, tid * per), end = min(p.S, beg + per);
         int local = 0;
         for (int k = beg; k < end; ++k) {
@@ -499,14 +516,14 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         if (lane == 31) wsum[warp] = incl;
         __syncthreads();
         if (warp == 0) {
-            int v = (lane < NCW + 1) ? wsum[lane] : 0;
+            const int v = (lane < NW) ? wsum[lane] : 0;
             int iv = v;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const int u = __shfl_up_sync(0xffffffffu, iv, off);
                 if (lane >= off) iv += u;
             }
-            if (lane < NCW + 1) wsum[lane] = iv - v;     // exclusive warp offsets
+            if (lane < NW) wsum[lane] = iv - v;          // exclusive warp offsets
         }
         __syncthreads();
         int run = wsum[warp] + incl - local;
@@ -514,21 +531,58 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
             pre[k] = run;
             run += n_parts(lens_s[k], p.P);
         }
-        if (tid == NT - 1) pre[p.S] = run;
+        if (tid == NTHREADS - 1) pre[p.S] = run;
     }
     __syncthreads();
     const int U = pre[p.S] * p.Hkv;
 
-    if (warp == NCW) {
+    if (role == 0) {
         // ================================================= producer warp
+        // Per unit: the next unit's ticket (global atomic) and its first 64
+        // block ids are fetched while the current unit's stages are issued,
+        // so no global round trip sits between two stages.  The TMA copies
+        // of a stage are issued by several lanes at once.
         const uint64_t policy = policy_evict_first();
         const size_t qrow = (size_t)p.Hq * D * E;
-        int gstage = 0, ucount = 0;
+        const int bs = p.bs, bsl = p.bs_log2;
+        const int npiece = (bs >= TOK) ? 1 : TOK / bs;   // blocks per stage
+        const int prow = (bs >= TOK) ? TOK : bs;         // box rows per block piece
+        struct Plan {
+            int u, s, j, i, t0, t1, nst, n_p, nblk;
+            const int32_t* trow;   // block-table entries of this unit's first block
+            int ids_a, ids_b;      // entries [win, win+32) and [win+32, win+64), one per lane
+        };
+        auto prepare = [&](int u) {
+            Plan q{};
+            q.u = u;
+            if (u >= U) return q;
+            const int x = u / p.Hkv;
+            int lo = 0, hi = p.S;                      // pre[lo] <= x < pre[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (pre[mid] <= x) lo = mid; else hi = mid;
+            }
+            q.s = lo;
+            q.i = x - pre[lo];
+            q.j = u - x * p.Hkv;
+            const int L = lens_s[lo];
+            q.t0 = min(q.i * p.P, L);
+            q.t1 = min(q.t0 + p.P, L);
+            q.nst = (q.t1 - q.t0 + TOK - 1) / TOK;
+            q.n_p = n_parts(L, p.P);
+            const int b0 = q.t0 >> bsl;
+            q.nblk = ((q.t1 + bs - 1) >> bsl) - b0;
+            q.trow = p.tables + (size_t)lo * p.mbps + b0;
+            q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
+            q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
+            return q;
+        };
+        int gstage = 0, st = 0, round = 0, ucount = 0;
+        int ticket = 0;
+        if (lane == 0) ticket = atomicAdd(&p.hdr->next_unit, 1);
+        Plan cur = prepare(__shfl_sync(0xffffffffu, ticket, 0));
         bool ok = true;
         while (ok) {
-            int u = 0;
-            if (lane == 0) u = atomicAdd(&p.hdr->next_unit, 1);
-            u = __shfl_sync(0xffffffffu, u, 0);
             const int slot = ucount % NUR;
             if (ucount >= NUR) {
                 bool w = true;
@@ -536,7 +590,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                 if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
             }
             UnitDesc* d = desc_at(slot);
-            if (u >= U) {
+            if (cur.u >= U) {
                 if (lane == 0) {
                     d->end = 1;
                     mbar_arrive(ufull + slot);
@@ -544,116 +598,117 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                 ++ucount;
                 break;
             }
-            const int x = u / p.Hkv;
-            int lo = 0, hi = p.S;                      // pre[lo] <= x < pre[hi]
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (pre[mid] <= x) lo = mid; else hi = mid;
-            }
-            const int s = lo, i = x - pre[s], j = u - x * p.Hkv;
-            const int L = lens_s[s];
-            const int t0 = min(i * p.P, L), t1 = min(t0 + p.P, L);
-            const int nst = (t1 - t0 + TOK - 1) / TOK;
             if (lane == 0) {
-                d->s = s; d->j = j; d->i = i; d->t0 = t0; d->t1 = t1;
-                d->n_p = n_parts(L, p.P);
-                d->stage_base = gstage; d->n_stages = nst; d->end = 0;
+                d->s = cur.s; d->j = cur.j; d->i = cur.i; d->t0 = cur.t0; d->t1 = cur.t1;
+                d->n_p = cur.n_p;
+                d->stage_base = gstage; d->n_stages = cur.nst; d->end = 0;
                 mbar_arrive_expect_tx(ufull + slot, G * D * E);
                 bulk_g2s(q_at(slot),
-                         reinterpret_cast<const uint8_t*>(p.q) + (size_t)s * qrow + (size_t)j * G * D * E,
+                         reinterpret_cast<const uint8_t*>(p.q) + (size_t)cur.s * qrow +
+                             (size_t)cur.j * G * D * E,
                          G * D * E, ufull + slot);
+                ticket = atomicAdd(&p.hdr->next_unit, 1);     // the unit after this one
             }
             ++ucount;
-            // block ids of this unit, 32 at a time, one lane each
-            const int32_t* trow = p.tables + (size_t)s * p.mbps;
-            const int b0 = t0 / p.bs;
-            const int b_end = (t1 + p.bs - 1) / p.bs;
-            int win = 0;                                // first block id index in `ids`
-            int ids = (lane < b_end - b0) ? __ldg(trow + b0 + lane) : -1;
-            for (int c = 0; c < nst && ok; ++c) {
-                const int tok0 = t0 + c * TOK;
-                const int nv = min(TOK, t1 - tok0);
-                const int st = gstage % p.nstage;
-                if (gstage >= p.nstage) {
+            Plan nxt{};
+            bool have_next = false;
+            int win = 0;                                // table index of ids_a's lane 0
+            const int b0 = cur.t0 >> bsl;
+            for (int c = 0; c < cur.nst; ++c) {
+                const int tok0 = cur.t0 + c * TOK;
+                if (round > 0) {
                     bool w = true;
-                    if (lane == 0) w = wait_or_abort(empty + st, ((gstage / p.nstage) - 1) & 1, abort_flag, p.err);
+                    if (lane == 0) w = wait_or_abort(empty + st, (round - 1) & 1, abort_flag, p.err);
                     if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
                 }
-                // block of each 8- or 16-token piece
-                const int npiece = (p.bs >= TOK) ? 1 : TOK / p.bs;
-                int blk[2] = {-1, -1}, off[2] = {0, 0}, rows[2] = {0, 0};
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    if (k < npiece) {
-                        const int tok = tok0 + k * p.bs;
-                        const int bi = tok / p.bs - b0;
-                        if (bi - win >= 32) {           // advance the id window
-                            win += 32;
-                            ids = (lane + win < b_end - b0) ? __ldg(trow + b0 + win + lane) : -1;
-                        }
-                        const int id = __shfl_sync(0xffffffffu, ids, (bi - win) & 31);
-                        if (tok < t1) {
-                            blk[k] = id;
-                            off[k] = tok % p.bs;
-                            rows[k] = (p.bs >= TOK) ? TOK : p.bs;
-                        }
+                // physical block of each piece (one piece unless bs = 8)
+                int blk0, blk1 = -2;
+                const int off0 = tok0 & (bs - 1);
+                {
+                    const int bi = (tok0 >> bsl) - b0;
+                    if (bi - win >= 32) {
+                        win += 32;
+                        cur.ids_a = cur.ids_b;
+                        cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
                     }
+                    blk0 = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
                 }
-                if (lane == 0) {
-                    bool valid = true;
-                    uint32_t bytes = 0;
-                    for (int k = 0; k < npiece; ++k) {
-                        if (rows[k] == 0) continue;
-                        if (blk[k] < 0 || blk[k] >= p.NB) valid = false;
-                        bytes += 2u * rows[k] * LY::ROWB;
+                if (npiece == 2) {
+                    const int tok = tok0 + bs;
+                    const int bi = (tok >> bsl) - b0;
+                    if (bi - win >= 32) {
+                        win += 32;
+                        cur.ids_a = cur.ids_b;
+                        cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
                     }
+                    const int id = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
+                    if (tok < cur.t1) blk1 = id;
+                }
+                const bool has1 = blk1 != -2;
+                const bool valid = blk0 >= 0 && blk0 < p.NB && (!has1 || (blk1 >= 0 && blk1 < p.NB));
+                uint8_t* Kd = stages + (size_t)st * LY::STAGE_BYTES;
+                if (lane == 0) {
                     stage_ok[st] = valid ? 1 : 0;
-                    uint8_t* Kd = stages + (size_t)st * LY::STAGE_BYTES;
-                    uint8_t* Vd = Kd + LY::KV_BYTES;
                     if (!valid) {
                         set_err(p.err, PA_DEV_BAD_BLOCK);
                         mbar_arrive(full + st);
                     } else {
-                        mbar_arrive_expect_tx(full + st, bytes);
-                        for (int k = 0; k < npiece; ++k) {
-                            if (rows[k] == 0) continue;
-                            const int y = (blk[k] * p.Hkv + j) * p.bs + off[k];
-                            const int rofs = k * p.bs * 128;      // piece row offset in a box
-#pragma unroll
-                            for (int b = 0; b < LY::NBOX; ++b) {
-                                tma_load_2d(Kd + b * BOXB + rofs, &kmap, b * BOX_ELEMS, y, full + st, policy);
-                                tma_load_2d(Vd + b * BOXB + rofs, &vmap, b * BOX_ELEMS, y, full + st, policy);
-                            }
-                        }
+                        mbar_arrive_expect_tx(full + st, (has1 ? 2u : 1u) * 2u * prow * LY::ROWB);
                     }
-                    (void)nv;
+                }
+                __syncwarp();
+                // one TMA box per lane: (piece, K or V, 128-byte column box)
+                const int nops = valid ? (has1 ? 2 : 1) * 2 * LY::NBOX : 0;
+                if (lane < nops) {
+                    const int piece = lane / (2 * LY::NBOX), rem = lane % (2 * LY::NBOX);
+                    const int kv = rem / LY::NBOX, b = rem % LY::NBOX;
+                    const int y = piece ? ((blk1 * p.Hkv + cur.j) << bsl)
+                                        : (((blk0 * p.Hkv + cur.j) << bsl) + off0);
+                    uint8_t* dst = Kd + kv * LY::KV_BYTES + b * BOXB + piece * 8 * 128;
+                    tma_load_2d(dst, kv ? &vmap : &kmap, b * BOX_ELEMS, y, full + st, policy);
                 }
                 ++gstage;
+                if (++st == nst) { st = 0; ++round; }
+                if (!have_next && (c == 3 || c == cur.nst - 1)) {
+                    nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
+                    have_next = true;
+                }
             }
+            if (!ok) break;
+            if (!have_next) nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
+            cur = nxt;
         }
-        // make sure no copy of this CTA is still landing in shared memory
+        // make sure no copy of this pipeline is still landing in shared memory
         if (lane == 0) {
-            const int first = max(0, gstage - p.nstage);
-            for (int g = first; g < gstage; ++g) mbar_wait(full + g % p.nstage, (g / p.nstage) & 1);
+            const int first = max(0, gstage - nst);
+            for (int g = first; g < gstage; ++g) mbar_wait(full + g % nst, (g / nst) & 1);
             const int ufirst = max(0, ucount - NUR);
             for (int k = ufirst; k < ucount; ++k) mbar_wait(ufull + k % NUR, (k / NUR) & 1);
         }
+        __syncwarp();
     } else {
         // ================================================= consumer warps
+        const int cw = role - 1;                 // 0 .. NCONS-1
+        const int ctid = cw * 32 + lane;         // 0 .. CT-1
+        const int bar_id = 1 + pipe;             // named barrier of this pipeline
         Engine eng;
-        float* xs = scratch + warp * 2 * G * TOK;
+        float* xs = scratch + cw * 2 * G * TOK;
         float* ps = xs + G * TOK;
         int ucount = 0;
         while (true) {
             const int slot = ucount % NUR;
-            if (!wait_or_abort(ufull + slot, (ucount / NUR) & 1, abort_flag, p.err)) break;
+            // every lane waits; __all_sync reconverges the warp (the tensor-core
+            // engine's ldmatrix/mma are .aligned and need the whole warp) and
+            // makes the decision the same in every lane
+            if (!__all_sync(0xffffffffu, wait_or_abort(ufull + slot, (ucount / NUR) & 1, abort_flag, p.err)))
+                break;
             const UnitDesc d = *desc_at(slot);
             if (d.end) break;
             eng.begin_unit(q_at(slot), lane, p.scale_log2e);
-            for (int c = warp; c < d.n_stages; c += NCW) {
-                const int g = d.stage_base + c;
-                const int st = g % p.nstage;
-                const bool have = wait_or_abort(full + st, (g / p.nstage) & 1, abort_flag, p.err);
+            int st = (d.stage_base + cw) % nst;
+            uint32_t ph = ((d.stage_base + cw) / nst) & 1;
+            for (int c = cw; c < d.n_stages; c += NCONS) {
+                const bool have = __all_sync(0xffffffffu, wait_or_abort(full + st, ph, abort_flag, p.err));
                 if (have && stage_ok[st]) {
                     const int nv = min(TOK, d.t1 - (d.t0 + c * TOK));
                     uint8_t* Ks = stages + (size_t)st * LY::STAGE_BYTES;
@@ -666,23 +721,24 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty + st);
+                st += NCONS;
+                while (st >= nst) { st -= nst; ph ^= 1u; }
             }
-            // ---- merge the warps' states of this unit
-            float* mb = mbuf + (size_t)(ucount & 1) * NCW * G * (D + 2);
-            eng.dump(mb + (size_t)warp * G * (D + 2), lane);   // m=-inf, l=0, o=0 if no stage
-            named_bar_sync(1, CT);
-            if (tid == 0) mbar_arrive(uempty + slot);   // q and the descriptor are consumed
+            // ---- merge the consumer warps' states of this unit
+            eng.dump(mbuf + (size_t)cw * G * (D + 2), lane);   // m=-inf, l=0, o=0 if no stage
+            named_bar_sync(bar_id, CT);
+            if (ctid == 0) mbar_arrive(uempty + slot);          // q and the descriptor are consumed
             const size_t sj = (size_t)d.s * p.Hkv + d.j;
-            for (int idx = tid; idx < G * D; idx += CT) {
+            for (int idx = ctid; idx < G * D; idx += CT) {
                 const int g = idx / D, dd = idx % D;
                 float M = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < NCW; ++w) M = fmaxf(M, mb[(w * G + g) * (D + 2)]);
+                for (int w = 0; w < NCONS; ++w) M = fmaxf(M, mbuf[(w * G + g) * (D + 2)]);
                 float Lsum = 0.f, O = 0.f;
                 if (M != -INFINITY) {
 #pragma unroll
-                    for (int w = 0; w < NCW; ++w) {
-                        const float* e = mb + (w * G + g) * (D + 2);
+                    for (int w = 0; w < NCONS; ++w) {
+                        const float* e = mbuf + (w * G + g) * (D + 2);
                         const float f = exp2f(e[0] - M);
                         Lsum += e[1] * f;
                         O += e[2 + dd] * f;
@@ -700,20 +756,22 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                     }
                 }
             }
+            named_bar_sync(bar_id, CT);                          // merge buffer free again
             if (d.n_p > 1) {
-                __threadfence();
-                named_bar_sync(1, CT);
-                if (tid == 0) {
+                if (ctid == 0) {
+                    __threadfence();                   // publish the partials before the count
                     const int prev = atomicAdd(p.counters + sj, 1);
                     const int last = (prev == d.n_p - 1);
-                    if (last) p.counters[sj] = 0;      // every partition has arrived
+                    if (last) {
+                        p.counters[sj] = 0;            // every partition has arrived
+                        __threadfence();               // see the other CTAs' partials
+                    }
                     *last_flag = last;
                 }
-                named_bar_sync(1, CT);
+                named_bar_sync(bar_id, CT);
                 if (*last_flag) {
-                    __threadfence();
                     const size_t base = sj * p.n_pmax;
-                    for (int idx = tid; idx < G * D; idx += CT) {
+                    for (int idx = ctid; idx < G * D; idx += CT) {
                         const int g = idx / D, dd = idx % D;
                         float M = -INFINITY;
                         for (int i = 0; i < d.n_p; ++i)
@@ -748,9 +806,11 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                         *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
                     }
                 }
+                named_bar_sync(bar_id, CT);                      // last_flag free again
             }
             ++ucount;
         }
+        __syncwarp();
     }
 
     __syncthreads();
@@ -826,7 +886,8 @@ int dev_info(DevInfo* out) {
     return PA_OK;
 }
 
-constexpr int kMaxStages = 24;
+constexpr int kMaxStages = 8;     // stages per pipeline
+constexpr int kMinStages = 2;     // any count >= 1 is correct; fewer only slows the pipeline
 
 size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
     size_t b = sizeof(WsHeader);
@@ -847,17 +908,22 @@ struct Launch {
     cudaStream_t stream;
 };
 
-template <typename T, int D, int G, int NCW, bool MMA>
+template <typename T, int D, int G, bool MMA>
 int run_decode(Launch& L, const DevInfo& di) {
-    using LY = Layout<T, D, G, NCW>;
-    auto kern = decode_kernel<T, D, G, NCW, MMA>;
-    const size_t fixed = LY::fixed_bytes(L.p.S) + 1024;   // + alignment slack
-    if ((size_t)di.smem_optin < fixed + (size_t)(NCW + 2) * LY::STAGE_BYTES) return PA_ERR_UNSUPPORTED;
-    int nstage = (int)((di.smem_optin - fixed) / LY::STAGE_BYTES);
-    nstage = std::min(nstage, kMaxStages);
-    L.p.nstage = nstage;
-    L.smem = LY(nstage, L.p.S).total() + 1024;
-    L.threads = (NCW + 1) * 32;
+    using LY = Layout<T, D, G>;
+    auto kern = decode_kernel<T, D, G, MMA>;
+    // a stage costs its K/V bytes, two mbarriers and a validity flag; the
+    // rest of the layout is fixed; + 1024 bytes of alignment slack
+    const size_t fixed = LY(0, L.p.S).total() + 1024 + 16;
+    const size_t per_stage = (size_t)LY::NPIPE * (LY::STAGE_BYTES + 2 * 8 + 4);
+    if ((size_t)di.smem_optin < fixed + (size_t)kMinStages * per_stage) return PA_ERR_UNSUPPORTED;
+    int nst = (int)((di.smem_optin - fixed) / per_stage);
+    nst = std::min(nst, kMaxStages);
+    while (nst > kMinStages && LY(nst, L.p.S).total() + 1024 > (size_t)di.smem_optin) --nst;
+    L.p.nst = nst;
+    L.smem = LY(nst, L.p.S).total() + 1024;
+    if (L.smem > (size_t)di.smem_optin) return PA_ERR_UNSUPPORTED;
+    L.threads = LY::NTHREADS;
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -874,9 +940,9 @@ int run_decode(Launch& L, const DevInfo& di) {
 template <typename T, int D, int G>
 int dispatch_engine(Launch& L, const DevInfo& di, bool mma) {
     if constexpr (sizeof(T) == 2) {
-        if (mma) return run_decode<T, D, G, 8, true>(L, di);
+        if (mma) return run_decode<T, D, G, true>(L, di);
     }
-    return run_decode<T, D, G, 8, false>(L, di);
+    return run_decode<T, D, G, false>(L, di);
 }
 
 template <typename T, int D>
@@ -990,6 +1056,7 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     p.Hkv = num_kv_heads;
     p.NB = num_blocks;
     p.bs = block_size;
+    p.bs_log2 = __builtin_ctz((unsigned)block_size);
     p.P = P;
     p.n_pmax = n_pmax;
     p.scale_log2e = scale * 1.4426950408889634f;
@@ -1010,8 +1077,11 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         std::lock_guard<std::mutex> lk(g_mu);
         engine = g_engine;
     }
-    const bool mma = dtype != PA_F32 && engine != PA_ENGINE_CUDA_CORE;
-    if (engine == PA_ENGINE_MMA && dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+    // The tensor-core engine is enabled only on request and only for G = 1:
+    // with G > 1 it failed (launch failure / timeouts) at full size under the
+    // multi-pipeline schedule for a cause not yet found, so it is not run.
+    const bool mma = engine == PA_ENGINE_MMA;
+    if (mma && (dtype == PA_F32 || G != 1)) return PA_ERR_UNSUPPORTED;
     switch (dtype) {
         case PA_F32: return dispatch_dim<float>(L, di, head_dim, G, false);
         case PA_F16: return dispatch_dim<__half>(L, di, head_dim, G, mma);

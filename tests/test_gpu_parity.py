@@ -25,7 +25,7 @@ from tests.harness import (GpuRun, check_close, oracle_sampled, out_f64, sample_
 pytestmark = pytest.mark.gpu
 pa = pytest.importorskip("paged_kv_cache_426_b200")
 
-ENGINES = {"auto": 0, "core": 1}
+ENGINES = {"default": 0}
 
 
 @pytest.fixture(params=list(ENGINES))
@@ -128,7 +128,8 @@ def test_shared_vs_duplicated_prefix_bit_identical():
     b, rb = _decode_outputs(workloads.prefix_f16(duplicate_prefix=True, **kw), 32)
     assert torch.equal(a[0], b[0])
     # the shared layout really holds fewer blocks
-    assert ra.manager.alloc.num_free() > rb.manager.alloc.num_free()
+    used = lambda r: r.manager.alloc.num_blocks - r.manager.alloc.num_free()
+    assert used(ra) < used(rb)
 
 
 @pytest.mark.parametrize("P", [16, 512, 1024, 2048])
@@ -139,11 +140,30 @@ def test_partition_sizes_agree(P):
     check_close(got[0].double().numpy(), ref[0].double().numpy(), "bf16", f"P={P} vs unsplit")
 
 
-def test_engines_agree():
-    w = workloads.gqa8b_bf16(num_seqs=8)
-    a, rec = _decode_outputs(w, 512, 1)
-    b, _ = _decode_outputs(w, 512, 0)
-    check_close(a[0].double().numpy(), b[0].double().numpy(), "bf16", "core vs mma")
+@pytest.mark.parametrize("name,kw", [
+    ("mha", dict()), ("prefix", dict()), ("mha_bf16_d64", dict())])
+def test_mma_engine_g1(name, kw):
+    """The tensor-core engine (accepted for G = 1 only) against the oracle."""
+    prev = pa.pa_set_decode_engine(pa.PA_ENGINE_MMA)
+    try:
+        if name == "mha":
+            run_full_compare(workloads.mha7b_f16(steps=3, num_seqs=5), partition_size=64)
+        elif name == "prefix":
+            w = workloads.prefix_f16(n_req=6, plen=64, suffix_max=40, n_fork=2, heads=4)
+            run_full_compare(w, partition_size=32)
+        else:
+            w = workloads.custom("bf16", [1, 15, 16, 17, 100, 257], 2, 2, 64, 16, seed=5,
+                                 partition_size=64)
+            run_full_compare(w)
+    finally:
+        pa.pa_set_decode_engine(prev)
+
+
+def test_mma_engine_rejects_groups():
+    w = workloads.gqa8b_bf16(num_seqs=2)
+    with pytest.raises(pa.PAError) as e:
+        _decode_outputs(w, 512, 2)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
 
 
 # ---------------------------------------------------------------- edge cases
@@ -196,7 +216,7 @@ def test_bad_block_id_sets_flag_without_fault():
     pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, workspace=ws, err_flag=err)
     torch.cuda.synchronize()
     assert err.item() == pa.PA_DEV_BAD_BLOCK
-    ref = oracle.paged_decode(oracle.as_storage(q.cpu(), "f16"), oracle.as_storage(kc.cpu(), "f16"),
+    ref = oracle.paged_decode(oracle.as_storage(q.cpu()[1:], "f16"), oracle.as_storage(kc.cpu(), "f16"),
                               oracle.as_storage(vc.cpu(), "f16"), tab.cpu().numpy()[1:],
                               lens.cpu().numpy()[1:], 0.1, "f16")
     check_close(out_f64(out[1:], "f16"), ref, "f16", "the valid sequence is unaffected")

@@ -124,6 +124,33 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def profiled_traffic(workload, algo_bytes):
+    """DRAM bytes per decode launch from the committed ncu summary of this
+    workload, scaled to this launch's algorithmic bytes; None if there is no
+    summary or the decode sources changed since it was captured."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch",
+                                                   "algorithmic_bytes_per_launch",
+                                                   "source_sha256_16"):
+            k, v = line.split(":", 1)
+            fields[k] = v.strip()
+    try:
+        want = dict(x.split("=") for x in fields["source_sha256_16"].split())
+        for name, h in want.items():
+            src = os.path.join(ROOT, "paged_kv_cache_426_b200", "csrc", name)
+            if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != h:
+                return None
+        t, a = int(fields["traffic_bytes_per_launch"]), int(fields["algorithmic_bytes_per_launch"])
+    except (KeyError, ValueError, OSError):
+        return None
+    return int(round(t * algo_bytes / a))
+
+
 def dist_setup(n_gpus):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -322,7 +349,8 @@ def run_ours(args, rank, world, local):
         "decode_only": {"gbs": round(dec_gbs, 1), "ms": round(dec_avg_ms, 4),
                         "seqs_per_s": round(S / (dec_avg_ms * 1e-3), 1)},
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(dec_gbs / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(dec_gbs / peak, 4),
+                     "traffic": profiled_traffic(w.name, sum(step_bytes) / len(step_bytes)),
                      "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "pa_decode"},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -409,9 +437,9 @@ def cpu_baseline(w, seconds):
     q = oracle.as_storage(w.step_q[0], w.dtype)
     esize = torch.tensor([], dtype=w.torch_dtype).element_size()
     done, nbytes, t0 = 0, 0, time.perf_counter()
-    order = list(range(len(st.seqs)))
-    while done < len(order):
-        s = order[done]
+    S = len(st.seqs)
+    while True:                 # whole sequences, cycling over the batch, ~`seconds` of work
+        s = done % S
         oracle.paged_decode(q[s:s + 1], rec.key_cache, rec.value_cache, st.block_tables[s:s + 1],
                             st.context_lens[s:s + 1], w.scale, w.dtype)
         nbytes += algorithmic_bytes([int(st.context_lens[s])], w.num_q_heads, w.num_kv_heads,
@@ -423,8 +451,9 @@ def cpu_baseline(w, seconds):
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
-            "sample": f"{done} of {len(order)} sequences of step 0 of {w.name}, float64 numpy "
-                      f"(gather through the block table + softmax attention), {dt:.1f} s",
+            "sample": f"{done} sequence decodes ({done / S:.2f} passes over the {S} sequences of "
+                      f"step 0 of {w.name}), float64 numpy (gather through the block table + "
+                      f"softmax attention), {dt:.1f} s",
             "seqs_per_s": round(done / dt, 3), "host_cpus": len(os.sched_getaffinity(0))}
 
 

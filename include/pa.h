@@ -125,6 +125,30 @@ int pa_decode(void* out, const void* query, const void* key_cache,
               size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
               void* stream);
 
+/* pa_decode_static - pa_decode without a caller-provided workspace, for
+ * callers that cannot allocate device memory (a plugin inside a host that
+ * owns every device allocation, a fixed memory budget, or a latency-critical
+ * path where cudaMalloc's possible device synchronisation is not acceptable).
+ * The pages have no counterpart: this is an interface convenience.
+ * The workspace is a fixed array of PA_DECODE_STATIC_WORKSPACE_BYTES that the
+ * library keeps in device memory on every GPU that loads it, until exit.
+ * Arguments and results are those of pa_decode.  A call whose workspace
+ * (pa_decode_workspace_size) exceeds the array returns PA_ERR_INVALID and
+ * launches nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Each call clears the scheduler words on
+ * `stream` and then runs pa_decode.  All calls on a device share the one
+ * array: calls that overlap on the GPU race and must be serialised by the
+ * caller (e.g. one stream).  Allocates nothing. */
+#define PA_DECODE_STATIC_WORKSPACE_BYTES (16u << 20)
+int pa_decode_static(void* out, const void* query, const void* key_cache,
+                     const void* value_cache, const int32_t* block_tables,
+                     int max_blocks_per_seq, const int32_t* context_lens,
+                     int max_context_len, int num_seqs, int num_q_heads,
+                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                     float scale, int partition_size, pa_dtype dtype,
+                     int32_t* err_flag, void* stream);
+
 /* Decode engine selection (for measurement).  PA_ENGINE_AUTO and
  * PA_ENGINE_CUDA_CORE use CUDA-core dot products.  PA_ENGINE_MMA uses
  * m16n8k16 tensor-core MMAs; it is accepted only for f16/bf16 with

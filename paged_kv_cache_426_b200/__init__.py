@@ -43,6 +43,8 @@ SIGNATURES = {
     "pa_decode_workspace_init": ([_vp, _sz, _vp], _i),
     "pa_decode": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                    _sz, _i, _vp, _vp], _i),
+    "pa_decode_static": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                          _i, _vp, _vp], _i),
     "pa_set_decode_engine": ([_i], _i),
     "pa_copy_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "pa_allocator_create": ([_i, _pi32, _i, C.POINTER(_vp)], _i),
@@ -164,6 +166,23 @@ def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, ma
                         int(partition_size), _ptr(workspace),
                         workspace.numel() * workspace.element_size(), pa_dtype(query),
                         _ptr(err_flag), _stream(stream)), "pa_decode")
+
+
+PA_DECODE_STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def pa_decode_static(out, query, key_cache, value_cache, block_tables, context_lens,
+                     max_context_len, scale, *, partition_size=0, err_flag=None, stream=None):
+    """pa_decode with the library's fixed device workspace (no allocation by
+    anyone); same arguments as pa_decode minus the workspace."""
+    _cuda(out, query, key_cache, value_cache, block_tables, context_lens, err_flag)
+    S, hq, d = query.shape
+    NB, hkv, bs, _ = key_cache.shape
+    check(lib.pa_decode_static(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                               _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                               int(max_context_len), S, hq, hkv, d, bs, NB, float(scale),
+                               int(partition_size), pa_dtype(query), _ptr(err_flag),
+                               _stream(stream)), "pa_decode_static")
 
 
 def pa_set_decode_engine(engine: int) -> int:

@@ -1091,3 +1091,57 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ allocation-free entry point
+// pa_decode_static: pa_decode with its workspace in a fixed array that the
+// library itself holds in device memory, for callers that cannot allocate:
+// plugins running inside a host that owns every device allocation, code whose
+// memory budget is fixed up front, and latency-critical paths where a
+// cudaMalloc (which may synchronise the device) is not acceptable.  The array
+// is reserved on every GPU that loads this library and kept until exit.
+namespace {
+
+constexpr size_t kStaticWsBytes = (size_t)PA_DECODE_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
+
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {};   // device address of g_static_ws, per device
+
+}  // namespace
+
+extern "C" int pa_decode_static(void* out, const void* query, const void* key_cache,
+                                const void* value_cache, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* context_lens,
+                                int max_context_len, int num_seqs, int num_q_heads,
+                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                float scale, int partition_size, pa_dtype dtype,
+                                int32_t* err_flag, void* stream) {
+    if (num_seqs == 0) return PA_OK;
+    size_t need = 0;
+    int st = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                      max_context_len, partition_size, &need);
+    if (st != PA_OK) return st;
+    if (need > kStaticWsBytes) return PA_ERR_INVALID;   // larger than the fixed array
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
+    void* ws = nullptr;
+    {
+        // first call on this device (with it current): look up the array's
+        // device address; host code cannot use g_static_ws's name directly
+        std::lock_guard<std::mutex> lk(g_static_mu);
+        if (!g_static_ptr[dev]) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) return PA_ERR_CUDA;
+            g_static_ptr[dev] = ptr;
+        }
+        ws = g_static_ptr[dev];
+    }
+    // the scheduler words and partition counters must start at zero; a call
+    // that stopped early (PA_DEV_TIMEOUT) may have left them dirty
+    const size_t counters = sizeof(WsHeader) + (((size_t)num_seqs * num_kv_heads * 4 + 255) / 256) * 256;
+    if (cudaMemsetAsync(ws, 0, counters, (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+    return pa_decode(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                     head_dim, block_size, num_blocks, scale, partition_size, ws,
+                     kStaticWsBytes, dtype, err_flag, stream);
+}

@@ -66,6 +66,61 @@ template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, f
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ---------------------------------------------------------------- packed fp32 pairs
+// Two fp32 values in one 64-bit register (low half = first).  sm_100 has
+// packed fp32x2 FMA / MUL: one instruction does both lanes.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Elements of a 32-bit word of storage as fp32 pairs.
+template <typename T> struct Pairs;
+template <> struct Pairs<float> {          // two words make one pair
+    static constexpr int WORDS_PER_PAIR = 2;
+};
+template <> struct Pairs<__half> {
+    static constexpr int WORDS_PER_PAIR = 1;
+    static __device__ __forceinline__ uint64_t from_word(uint32_t w) {
+        __half2 h = *reinterpret_cast<__half2*>(&w);
+        const float2 f = __half22float2(h);
+        return f2_pack(f.x, f.y);
+    }
+};
+template <> struct Pairs<__nv_bfloat16> {
+    static constexpr int WORDS_PER_PAIR = 1;
+    static __device__ __forceinline__ uint64_t from_word(uint32_t w) {
+        return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+};
+// 16 bytes of storage (uint4) -> 16 / (2 * sizeof(T)) fp32 pairs
+template <typename T>
+__device__ __forceinline__ void pairs16(const uint4 raw, uint64_t* out) {
+    if constexpr (sizeof(T) == 4) {
+        out[0] = (uint64_t)raw.x | ((uint64_t)raw.y << 32);
+        out[1] = (uint64_t)raw.z | ((uint64_t)raw.w << 32);
+    } else {
+        out[0] = Pairs<T>::from_word(raw.x);
+        out[1] = Pairs<T>::from_word(raw.y);
+        out[2] = Pairs<T>::from_word(raw.z);
+        out[3] = Pairs<T>::from_word(raw.w);
+    }
+}
+
 // ---------------------------------------------------------------- errors
 __device__ __forceinline__ void set_err(int32_t* err, int code) {
     if (err) atomicCAS(err, 0, code);

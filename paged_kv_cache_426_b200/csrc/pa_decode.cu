@@ -56,8 +56,11 @@
 namespace pa {
 
 constexpr int TOK = 16;           // tokens per pipeline stage
-constexpr int NCONS = 2;          // consumer warps per pipeline (alternate stages)
-constexpr int PIPE_WARPS = 1 + NCONS;
+// consumer warps per pipeline (they take a unit's stages round-robin).  A ring
+// slot stays held while its consumer computes, so extra consumers only pay
+// where compute is the limit: 3 for the CUDA-core engine with query groups
+// (G > 1), otherwise 2.
+template <bool MMA, int G> constexpr int cons_for() { return (!MMA && G > 1) ? 3 : 2; }
 // independent producer/consumer pipelines per CTA: 4, or 2 when a stage is
 // 16 KB (fp32, head_dim 128) so that the rings still fit in shared memory
 template <typename T, int D> constexpr int pipes_for() { return sizeof(T) * D > 256 ? 2 : 4; }
@@ -90,8 +93,10 @@ struct DecodeParams {
 
 // Shared-memory layout (dynamic, 1024-byte aligned base).  Every pipeline has
 // its own stage ring, unit-descriptor ring, barriers, scratch and merge buffer.
-template <typename T, int D, int G>
+template <typename T, int D, int G, int NCONS_ = 3>
 struct Layout {
+    static constexpr int NCONS = NCONS_;
+    static constexpr int PIPE_WARPS = 1 + NCONS;
     static constexpr int NPIPE = pipes_for<T, D>();
     static constexpr int NTHREADS = NPIPE * PIPE_WARPS * 32;
     static constexpr int E = sizeof(T);
@@ -101,7 +106,8 @@ struct Layout {
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int QB = ((G * D * E + 127) / 128) * 128;
     static constexpr int UNIT_BYTES = (int)sizeof(UnitDesc) + QB;
-    static constexpr int SCRATCH = NCONS * 2 * G * TOK * 4;      // per pipe: xs + ps
+    static constexpr int QF = G * D * 4;                         // per pipe: fp32 scaled q
+    static constexpr int SCRATCH = NCONS * 3 * G * TOK * 4 + QF; // per pipe: xs, (p, p) pairs, q
     static constexpr int MBUF = NCONS * G * (D + 2) * 4;         // per pipe
     int nst, S;                                                  // stages per pipe
     __host__ __device__ Layout(int nst_, int S_) : nst(nst_), S(S_) {}
@@ -189,62 +195,86 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane) {
 
 template <typename T, int D, int G>
 struct CoreEngine {
-    using LY = Layout<T, D, G>;
+    using LY = Layout<T, D, G, cons_for<false, G>()>;
     static constexpr int E = sizeof(T);
-    static constexpr int VEC = 16 / E;                       // elements per chunk
+    static constexpr int VEC = 16 / E;                       // elements per 16-byte chunk
+    static constexpr int NP = VEC / 2;                       // fp32 pairs per chunk
     static constexpr int CHUNKS = LY::ROWB / 16;             // chunks per row
     static constexpr int LPT = (G >= 8 && CHUNKS >= 16) ? 16 : 8;
     static constexpr int TPW = 32 / LPT;                     // tokens per warp step
     static constexpr int NCH = CHUNKS / LPT;                 // chunks per lane
     static constexpr int DPL = D / 32;                       // PV columns per lane
+    static constexpr int DPP = DPL / 2;                      // PV column pairs per lane
     static constexpr int NPASS = (G + 1) / 2;
     static_assert(G <= LPT, "group larger than lanes per token");
 
-    float qf[G][NCH * VEC];
-    float o[G][DPL];
+    // All arithmetic on fp32 pairs (fma.rn.f32x2).  q lives in shared memory as
+    // pre-scaled fp32, laid out [g][chunk c][k/2][lane r] in 16-byte units
+    // (two pairs), so the q reads of one step are conflict-free.
+    static constexpr int QUNITS = G * NCH * (NP / 2) * LPT;   // 16-byte units of q
+    uint64_t o2[G][DPP];
     float m_half[NPASS], l_half[NPASS];
+    const uint4* qf = nullptr;
 
-    __device__ void begin_unit(const T* qs, int lane, float scale_log2e) {
-        const int r = lane % LPT;
+    // Cooperative (all consumer threads of the pipeline): storage q -> fp32 scaled,
+    // interleaved.  Caller synchronises before the first stage.
+    static __device__ void stage_q(const T* qs, uint4* qf4, int ctid, int nthreads, float scale) {
+        for (int u = ctid; u < QUNITS; u += nthreads) {
+            const int r = u % LPT, kk = (u / LPT) % (NP / 2), c = (u / (LPT * (NP / 2))) % NCH;
+            const int g = u / (LPT * (NP / 2) * NCH);
+            const int e0 = (r + c * LPT) * VEC + 4 * kk;
+            float4 f;
+            f.x = DT<T>::to_float(qs[g * D + e0 + 0]) * scale;
+            f.y = DT<T>::to_float(qs[g * D + e0 + 1]) * scale;
+            f.z = DT<T>::to_float(qs[g * D + e0 + 2]) * scale;
+            f.w = DT<T>::to_float(qs[g * D + e0 + 3]) * scale;
+            qf4[u] = *reinterpret_cast<uint4*>(&f);
+        }
+    }
+
+    __device__ void begin_unit(const uint4* qf4) {
+        qf = qf4;
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int c = 0; c < NCH; ++c)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e)
-                    qf[g][c * VEC + e] =
-                        DT<T>::to_float(qs[g * D + (r + c * LPT) * VEC + e]) * scale_log2e;
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) o[g][e] = 0.f;
+            for (int k = 0; k < DPP; ++k) o2[g][k] = 0ull;
 #pragma unroll
         for (int k = 0; k < NPASS; ++k) { m_half[k] = -INFINITY; l_half[k] = 0.f; }
     }
 
-    __device__ void stage(const uint8_t* Ks, const uint8_t* Vs, int nv, float* xs, float* ps,
+    // xs: [G][TOK] logits; ps2: [TOK][G] splatted (p, p) pairs.
+    __device__ void stage(const uint8_t* Ks, const uint8_t* Vs, int nv, float* xs, uint64_t* ps2,
                           int lane) {
         const int r = lane % LPT;
         // ---- x_t = <q_g, K_t> (pre-scaled to log2 units)
 #pragma unroll
         for (int step = 0; step < TOK / TPW; ++step) {
             const int tok = step * TPW + lane / LPT;
-            float acc[G];
+            uint64_t acc2[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) acc[g] = 0.f;
+            for (int g = 0; g < G; ++g) acc2[g] = 0ull;
 #pragma unroll
             for (int c = 0; c < NCH; ++c) {
                 const int ch = r + c * LPT;
                 const uint4 raw = *reinterpret_cast<const uint4*>(
                     Ks + (ch >> 3) * BOXB + tok * 128 + (((ch & 7) ^ (tok & 7)) << 4));
-                float x[VEC];
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) Unpack<T>::run(w[k], &x[k * Unpack<T>::N]);
+                uint64_t x2[NP];
+                pairs16<T>(raw, x2);
 #pragma unroll
                 for (int g = 0; g < G; ++g)
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) acc[g] = fmaf(qf[g][c * VEC + e], x[e], acc[g]);
+                    for (int kk = 0; kk < NP / 2; ++kk) {
+                        const uint4 q4 = qf[((g * NCH + c) * (NP / 2) + kk) * LPT + r];
+                        acc2[g] = f2_fma((uint64_t)q4.x | ((uint64_t)q4.y << 32), x2[2 * kk], acc2[g]);
+                        acc2[g] = f2_fma((uint64_t)q4.z | ((uint64_t)q4.w << 32), x2[2 * kk + 1], acc2[g]);
+                    }
+            }
+            float acc[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float lo, hi;
+                f2_unpack(acc2[g], lo, hi);
+                acc[g] = lo + hi;
             }
             const float v = reduce_scatter<G, LPT>(acc, lane);
             constexpr int LPH = LPT / G;           // lanes holding one head's total
@@ -252,7 +282,7 @@ struct CoreEngine {
         }
         __syncwarp();
         // ---- online softmax over the stage's tokens, two heads per pass
-        float alpha[G];
+        uint64_t alpha2[G];
 #pragma unroll
         for (int pass = 0; pass < NPASS; ++pass) {
             const int g = 2 * pass + (lane >> 4);
@@ -272,42 +302,46 @@ struct CoreEngine {
             if (live) {
                 m_half[pass] = mn;
                 l_half[pass] = l_half[pass] * a + sum;
-                ps[t * G + g] = pr;
+                ps2[t * G + g] = f2_pack(pr, pr);
             }
-            alpha[2 * pass] = __shfl_sync(0xffffffffu, a, 0);
-            if (2 * pass + 1 < G) alpha[2 * pass + 1] = __shfl_sync(0xffffffffu, a, 16);
+            const float a0 = __shfl_sync(0xffffffffu, a, 0);
+            alpha2[2 * pass] = f2_pack(a0, a0);
+            if (2 * pass + 1 < G) {
+                const float a1 = __shfl_sync(0xffffffffu, a, 16);
+                alpha2[2 * pass + 1] = f2_pack(a1, a1);
+            }
         }
         __syncwarp();
         // ---- o = alpha o + sum_t p_t V_t
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) o[g][e] *= alpha[g];
+            for (int k = 0; k < DPP; ++k) o2[g][k] = f2_mul(alpha2[g], o2[g][k]);
         const int byte = lane * DPL * E;                  // this lane's columns
         const int box = byte >> 7, cc = (byte & 127) >> 4, sub = byte & 15;
         auto pv_token = [&](int t) {
             const uint8_t* src = Vs + box * BOXB + t * 128 + (((cc ^ (t & 7)) << 4) | sub);
-            float v[DPL];
+            uint64_t v2[DPP];
             if constexpr (DPL * E == 16) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(src);
-                const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) Unpack<T>::run(w[k], &v[k * Unpack<T>::N]);
+                pairs16<T>(*reinterpret_cast<const uint4*>(src), v2);
             } else if constexpr (DPL * E == 8) {
                 const uint2 raw = *reinterpret_cast<const uint2*>(src);
-                Unpack<T>::run(raw.x, &v[0]);
-                Unpack<T>::run(raw.y, &v[Unpack<T>::N]);
+                if constexpr (E == 4) {
+                    v2[0] = (uint64_t)raw.x | ((uint64_t)raw.y << 32);
+                } else {
+                    v2[0] = Pairs<T>::from_word(raw.x);
+                    v2[1] = Pairs<T>::from_word(raw.y);
+                }
             } else {
-                const uint32_t raw = *reinterpret_cast<const uint32_t*>(src);
-                Unpack<T>::run(raw, &v[0]);
+                v2[0] = Pairs<T>::from_word(*reinterpret_cast<const uint32_t*>(src));
             }
-            float pv[G];
+            uint64_t p2[G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) pv[g] = ps[t * G + g];
+            for (int g = 0; g < G; ++g) p2[g] = ps2[t * G + g];
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) o[g][e] = fmaf(pv[g], v[e], o[g][e]);
+                for (int k = 0; k < DPP; ++k) o2[g][k] = f2_fma(p2[g], v2[k], o2[g][k]);
         };
         if (nv == TOK) {
 #pragma unroll
@@ -323,7 +357,12 @@ struct CoreEngine {
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) mb[g * (D + 2) + 2 + lane * DPL + e] = o[g][e];
+            for (int k = 0; k < DPP; ++k) {
+                float lo, hi;
+                f2_unpack(o2[g][k], lo, hi);
+                mb[g * (D + 2) + 2 + lane * DPL + 2 * k] = lo;
+                mb[g * (D + 2) + 2 + lane * DPL + 2 * k + 1] = hi;
+            }
 #pragma unroll
         for (int pass = 0; pass < NPASS; ++pass) {
             const int g = 2 * pass + (lane >> 4);
@@ -445,11 +484,13 @@ struct MmaEngine {
 // share nothing but the prefix sums and the abort flag; each takes its own
 // units from the global ticket counter.
 template <typename T, int D, int G, bool MMA>
-__global__ void __launch_bounds__(Layout<T, D, G>::NTHREADS, 1)
+__global__ void __launch_bounds__(Layout<T, D, G, cons_for<MMA, G>()>::NTHREADS, 1)
 decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
               DecodeParams p) {
-    using LY = Layout<T, D, G>;
+    using LY = Layout<T, D, G, cons_for<MMA, G>()>;
     using Engine = typename std::conditional<MMA, MmaEngine<T, D, G>, CoreEngine<T, D, G>>::type;
+    constexpr int NCONS = LY::NCONS;
+    constexpr int PIPE_WARPS = LY::PIPE_WARPS;
     constexpr int NPIPE = LY::NPIPE;
     constexpr int NTHREADS = LY::NTHREADS;
     constexpr int CT = NCONS * 32;               // consumer threads of a pipeline
@@ -692,8 +733,9 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         const int ctid = cw * 32 + lane;         // 0 .. CT-1
         const int bar_id = 1 + pipe;             // named barrier of this pipeline
         Engine eng;
-        float* xs = scratch + cw * 2 * G * TOK;
-        float* ps = xs + G * TOK;
+        float* xs = scratch + cw * 3 * G * TOK;
+        uint64_t* ps = reinterpret_cast<uint64_t*>(xs + G * TOK);
+        uint4* qf4 = reinterpret_cast<uint4*>(scratch + NCONS * 3 * G * TOK);   // fp32 q (core engine)
         int ucount = 0;
         while (true) {
             const int slot = ucount % NUR;
@@ -704,7 +746,13 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                 break;
             const UnitDesc d = *desc_at(slot);
             if (d.end) break;
-            eng.begin_unit(q_at(slot), lane, p.scale_log2e);
+            if constexpr (MMA) {
+                eng.begin_unit(q_at(slot), lane, p.scale_log2e);
+            } else {
+                Engine::stage_q(q_at(slot), qf4, ctid, CT, p.scale_log2e);
+                named_bar_sync(bar_id, CT);                 // q in fp32 for every consumer warp
+                eng.begin_unit(qf4);
+            }
             int st = (d.stage_base + cw) % nst;
             uint32_t ph = ((d.stage_base + cw) / nst) & 1;
             for (int c = cw; c < d.n_stages; c += NCONS) {
@@ -910,7 +958,7 @@ struct Launch {
 
 template <typename T, int D, int G, bool MMA>
 int run_decode(Launch& L, const DevInfo& di) {
-    using LY = Layout<T, D, G>;
+    using LY = Layout<T, D, G, cons_for<MMA, G>()>;
     auto kern = decode_kernel<T, D, G, MMA>;
     // a stage costs its K/V bytes, two mbarriers and a validity flag; the
     // rest of the layout is fixed; + 1024 bytes of alignment slack

@@ -1,7 +1,7 @@
 """Benchmark: paged decode attention on B200, KV-read GB/s per decode step.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--partition-size P] [--engine auto|core|mma]
+                    [--impl ours|reference] [--partition-size P] [--engine auto|core|tensor]
 
 A step is one decode step of the workload's batch: copy-on-write block
 copies (when the host manager reports any), the cache write of the step's new
@@ -281,7 +281,7 @@ def run_ours(args, rank, world, local):
     w = workloads.make(args.workload, steps=n_steps)
     P = w.partition_size if args.partition_size is None else args.partition_size
     import paged_kv_cache_426_b200 as pa
-    pa.pa_set_decode_engine({"auto": 0, "core": 1, "mma": 2}[args.engine])
+    pa.pa_set_decode_engine({"auto": 0, "core": 1, "tensor": 2}[args.engine])
     sess = Session(w, P, dev)
     _, mgr = sess.prefill()
     plan = sess.plan_steps(mgr, n_steps)
@@ -493,7 +493,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.BUILDERS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition-size", type=int, default=None)
-    ap.add_argument("--engine", default="auto", choices=["auto", "core", "mma"])
+    ap.add_argument("--engine", default="auto", choices=["auto", "core", "tensor"])
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of clock soak")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")

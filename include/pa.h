@@ -149,12 +149,13 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
                      float scale, int partition_size, pa_dtype dtype,
                      int32_t* err_flag, void* stream);
 
-/* Decode engine selection (for measurement).  PA_ENGINE_AUTO and
- * PA_ENGINE_CUDA_CORE use CUDA-core dot products.  PA_ENGINE_MMA uses
- * m16n8k16 tensor-core MMAs; it is accepted only for f16/bf16 with
- * num_q_heads == num_kv_heads (other shapes return PA_ERR_UNSUPPORTED).
- * Process-wide; returns the previous value. */
-enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_MMA = 2 };
+/* Decode engine selection (for measurement).  PA_ENGINE_CUDA_CORE: fp32
+ * dot products on CUDA cores (any dtype).  PA_ENGINE_TENSOR: tcgen05
+ * tensor-core MMAs with accumulators in tensor memory, f16/bf16 only (f32
+ * returns PA_ERR_UNSUPPORTED).  PA_ENGINE_AUTO (the default): the tensor
+ * engine for f16/bf16 with query groups (num_q_heads > num_kv_heads), CUDA
+ * cores otherwise.  Process-wide; returns the previous value. */
+enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_TENSOR = 2 };
 int pa_set_decode_engine(int engine);
 
 /* --------------------------------------------------------------------------

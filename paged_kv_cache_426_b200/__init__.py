@@ -30,7 +30,7 @@ lib = C.CDLL(LIB_PATH)
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_OOM, PA_ERR_STATE = 0, -1, -2, -3, -4, -5
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 PA_DEV_BAD_SLOT, PA_DEV_BAD_BLOCK, PA_DEV_BAD_LEN, PA_DEV_BAD_PAIR, PA_DEV_TIMEOUT = 1, 2, 3, 4, 5
-PA_ENGINE_AUTO, PA_ENGINE_CUDA_CORE, PA_ENGINE_MMA = 0, 1, 2
+PA_ENGINE_AUTO, PA_ENGINE_CUDA_CORE, PA_ENGINE_TENSOR = 0, 1, 2
 
 _vp, _i, _i64, _sz, _f = C.c_void_p, C.c_int, C.c_int64, C.c_size_t, C.c_float
 _pi32, _pi64 = C.POINTER(C.c_int32), C.POINTER(C.c_int64)

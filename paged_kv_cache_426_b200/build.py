@@ -25,7 +25,8 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa_b200.so")
 
 SOURCES = ["pa_host.cpp", "pa_cache_ops.cu", "pa_decode.cu"]
-HEADERS = [os.path.join(CSRC, "pa_common.cuh"), os.path.join(INCLUDE, "pa.h")]
+HEADERS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
+    os.path.join(INCLUDE, "pa.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

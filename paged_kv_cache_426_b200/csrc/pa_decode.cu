@@ -11,40 +11,41 @@
 //  * Work unit = (sequence s, KV head j, partition i) covering tokens
 //    [i*P, min(L_s, (i+1)*P)).  All G query heads of the group are served by
 //    one pass over the group's K/V, so every K/V byte is read from HBM once.
-//  * Persistent CTAs (one per SM).  Each CTA computes the prefix sums of the
-//    partition counts (tiny), then one producer warp takes units from an
-//    atomic counter in the workspace (dynamic load balance, units of at most
-//    P tokens) and streams each unit as 16-token stages into a shared-memory
-//    ring: 2-D tensor TMA copies of 128-byte-wide boxes with 128B swizzle,
-//    one box row per token, so that all later shared-memory reads are free of
-//    bank conflicts.  The block table is read 32 entries at a time by the
+//  * Persistent CTAs (one per SM), each running several independent
+//    pipelines.  Each CTA computes the prefix sums of the partition counts
+//    (tiny); then a pipeline's producer warp takes units from an atomic
+//    counter in the workspace (dynamic load balance, units of at most P
+//    tokens) and streams each unit as 16-token stages into its shared-memory
+//    ring: 2-D tensor TMA copies of 128-byte-wide boxes with 128B swizzle, one
+//    box row per token.  The block table is read 32 entries at a time by the
 //    producer's lanes, ahead of use.  A 16-token stage never crosses a block
 //    (bs >= 16) or covers two (bs = 8).
-//  * Consumer warps take a unit's stages round-robin by logical stage index
-//    and keep a per-warp online softmax (running max m, sum l, output o) in
-//    the log2 domain.  Two compute engines (CUDA cores by default; the
-//    tensor-core one on request, G = 1 only):
-//      CUDA cores: 8 (or 16) lanes per token, 16-byte loads, warp-shuffle
-//        reduce-scatter of the G dot products, then p*V with each lane owning
-//        head_dim/32 output columns of all G heads;
-//      MMA (16-bit types): S = Q K^T and O += P V with m16n8k16 tensor-core
-//        MMAs; the query heads sit in the M dimension (rows >= G are zero),
-//        K and V come from the swizzled stage with ldmatrix(.trans), and the
-//        accumulators of S are reused directly as the A operand of P V.
-//  * At the end of a unit the consumer warps merge their states in shared
-//    memory.  A single-partition sequence writes `out` directly.  Otherwise
-//    the unit writes (m, l, o) to the workspace and bumps a per-(s, j)
-//    counter; the CTA that completes the last partition merges all partials
-//    with their log-sum-exp weights and writes `out` (and re-zeroes the
-//    counter).  No CTA ever waits for another.
+//  * Two compute engines read the same stages:
+//      CUDA cores (fp32, and the default for G = 1): consumer warps take a
+//        unit's stages round-robin and keep a per-warp online softmax in the
+//        log2 domain; 8 (or 16) lanes per token and packed fp32x2 FMAs.
+//      Tensor cores (tcgen05, 16-bit types, the default for G > 1): one
+//        thread issues S = Q K^T (M = 64 rows = query heads, rows >= G
+//        unused, N = 16 tokens) with Q and K read from shared memory through
+//        swizzled matrix descriptors and S accumulated in tensor memory; a
+//        softmax warp turns S into P (16-bit, in tensor memory) and the same
+//        thread issues O += P V with O resident in tensor memory for the
+//        whole unit.  The running max is only moved when it grows by more
+//        than 2^8, so O is rescaled rarely (exact: O, l and m stay
+//        consistent).
+//  * A single-partition sequence writes `out` directly.  Otherwise the unit
+//    writes (m, l, o) to the workspace and bumps a per-(s, j) counter; the
+//    CTA that completes the last partition merges all partials with their
+//    log-sum-exp weights and writes `out` (and re-zeroes the counter).  No
+//    CTA ever waits for another.
 //  * Summation order depends only on logical positions (stage index within
 //    the unit, warp index, partition index), never on physical block ids or
 //    on which CTA ran a unit, so results are bit-identical under any
 //    permutation of the pool and for block sizes 16..128.
 //  * Every wait is bounded (2 s); a timeout sets PA_DEV_TIMEOUT, makes the
-//    other warps give up quickly, waits (bounded) for the CTA's own copies
-//    in flight and returns.  Bad block ids or lengths set err_flag and the
-//    affected tokens are skipped.
+//    other warps give up quickly, waits (bounded) for the CTA's own copies and
+//    MMAs in flight, frees its tensor memory and returns.  Bad block ids or
+//    lengths set err_flag and the affected tokens are skipped.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -52,15 +53,16 @@
 #include <mutex>
 
 #include "pa_common.cuh"
+#include "pa_tcgen05.cuh"
 
 namespace pa {
 
 constexpr int TOK = 16;           // tokens per pipeline stage
-// consumer warps per pipeline (they take a unit's stages round-robin).  A ring
-// slot stays held while its consumer computes, so extra consumers only pay
-// where compute is the limit: 3 for the CUDA-core engine with query groups
+// consumer warps per pipeline of the CUDA-core engine (they take a unit's
+// stages round-robin).  A ring slot stays held while its consumer computes, so
+// extra consumers only pay where compute is the limit: 3 with query groups
 // (G > 1), otherwise 2.
-template <bool MMA, int G> constexpr int cons_for() { return (!MMA && G > 1) ? 3 : 2; }
+template <int G> constexpr int cons_for() { return G > 1 ? 3 : 2; }
 // independent producer/consumer pipelines per CTA: 4, or 2 when a stage is
 // 16 KB (fp32, head_dim 128) so that the rings still fit in shared memory
 template <typename T, int D> constexpr int pipes_for() { return sizeof(T) * D > 256 ? 2 : 4; }
@@ -195,7 +197,7 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int lane) {
 
 template <typename T, int D, int G>
 struct CoreEngine {
-    using LY = Layout<T, D, G, cons_for<false, G>()>;
+    using LY = Layout<T, D, G, cons_for<G>()>;
     static constexpr int E = sizeof(T);
     static constexpr int VEC = 16 / E;                       // elements per 16-byte chunk
     static constexpr int NP = VEC / 2;                       // fp32 pairs per chunk
@@ -374,128 +376,286 @@ struct CoreEngine {
     }
 };
 
-template <typename T, int D, int G>
-struct MmaEngine {
-    static_assert(sizeof(T) == 2, "tensor-core engine takes 16-bit types");
-    static_assert(G <= 8, "query heads of a group must fit 8 MMA rows");
-    static constexpr int KSTEPS = D / 16;
-    static constexpr int NDT = D / 8;          // 8-column output tiles
+// ------------------------------------------------------------ pieces shared by both kernels
 
-    uint32_t qa[KSTEPS][2];    // A fragments of Q (rows lane/4, k low / k high)
-    float oacc[NDT][4];        // O rows lane/4 (and padding rows +8)
-    float m, l;                // state of row lane/4
-
-    __device__ void begin_unit(const T* qs, int lane, float) {
-        const int r = lane >> 2, c = lane & 3;
-        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qs);
-#pragma unroll
-        for (int k = 0; k < KSTEPS; ++k) {
-            qa[k][0] = (r < G) ? q32[(r * D + 16 * k + 2 * c) >> 1] : 0u;
-            qa[k][1] = (r < G) ? q32[(r * D + 16 * k + 8 + 2 * c) >> 1] : 0u;
-        }
-#pragma unroll
-        for (int n = 0; n < NDT; ++n)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) oacc[n][e] = 0.f;
-        m = -INFINITY;
-        l = 0.f;
-    }
-
-    __device__ void stage(const uint8_t* Ks, uint8_t* Vs, int nv, float scale_log2e, int lane) {
-        const uint32_t kbase = smem_u32(Ks), vbase = smem_u32(Vs);
-        if (nv < TOK) {
-            // rows >= nv hold bytes of other tokens (or never-written memory);
-            // zero them so that p = 0 never meets a NaN in the P V product
-            constexpr int ROW16 = D * 2 / 16;
-            for (int idx = lane; idx < (TOK - nv) * ROW16; idx += 32) {
-                const int row = nv + idx / ROW16, ch = idx % ROW16;
-                *reinterpret_cast<uint4*>(Vs + (ch >> 3) * BOXB + row * 128 +
-                                          (((ch & 7) ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
-            }
-            __syncwarp();
-        }
-        // ---- S = Q K^T  (rows: heads, columns: 16 tokens as two n-tiles)
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        const int mi = lane >> 3, lr = lane & 7;
-#pragma unroll
-        for (int k = 0; k < KSTEPS; ++k) {
-            const int row = (mi >> 1) * 8 + lr, ch = 2 * k + (mi & 1);
-            uint32_t b00, b01, b10, b11;
-            ldsm_x4(kbase + (ch >> 3) * BOXB + row * 128 + (((ch & 7) ^ (row & 7)) << 4), b00, b01,
-                    b10, b11);
-            mma16816<T>(s0, qa[k][0], 0u, qa[k][1], 0u, b00, b01);
-            mma16816<T>(s1, qa[k][0], 0u, qa[k][1], 0u, b10, b11);
-        }
-        // ---- online softmax of row lane/4 over this stage's tokens
-        const int c = lane & 3;
-        const int t0 = 2 * c, t1 = 2 * c + 1, t2 = 8 + 2 * c, t3 = 9 + 2 * c;
-        float x0 = (t0 < nv) ? s0[0] * scale_log2e : -INFINITY;
-        float x1 = (t1 < nv) ? s0[1] * scale_log2e : -INFINITY;
-        float x2 = (t2 < nv) ? s1[0] * scale_log2e : -INFINITY;
-        float x3 = (t3 < nv) ? s1[1] * scale_log2e : -INFINITY;
-        float bm = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-        const float mn = fmaxf(m, bm);
-        const float a = exp2f(m - mn);
-        const float p0 = exp2f(x0 - mn), p1 = exp2f(x1 - mn);
-        const float p2 = exp2f(x2 - mn), p3 = exp2f(x3 - mn);
-        float rs = (p0 + p1) + (p2 + p3);
-        rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-        rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-        l = l * a + rs;
-        m = mn;
-#pragma unroll
-        for (int n = 0; n < NDT; ++n) {
-            oacc[n][0] *= a;
-            oacc[n][1] *= a;
-        }
-        const uint32_t pa0 = pack2<T>(p0, p1), pa2 = pack2<T>(p2, p3);
-        // ---- O += P V  (B operand = V [tokens x columns] via ldmatrix.trans)
-#pragma unroll
-        for (int n2 = 0; n2 < NDT / 2; ++n2) {
-            const int row = (mi & 1) * 8 + lr, ch = 2 * n2 + (mi >> 1);
-            uint32_t v0, v1, v2, v3;
-            ldsm_x4_t(vbase + (ch >> 3) * BOXB + row * 128 + (((ch & 7) ^ (row & 7)) << 4), v0, v1,
-                      v2, v3);
-            mma16816<T>(oacc[2 * n2], pa0, 0u, pa2, 0u, v0, v1);
-            mma16816<T>(oacc[2 * n2 + 1], pa0, 0u, pa2, 0u, v2, v3);
-        }
-    }
-
-    __device__ void dump(float* mb, int lane) const {
-        const int r = lane >> 2, c = lane & 3;
-        if (r < G) {
-#pragma unroll
-            for (int n = 0; n < NDT; ++n)
-                *reinterpret_cast<float2*>(&mb[r * (D + 2) + 2 + 8 * n + 2 * c]) =
-                    make_float2(oacc[n][0], oacc[n][1]);
-            if (c == 0) {
-                mb[r * (D + 2) + 0] = m;
-                mb[r * (D + 2) + 1] = l;
-            }
-        }
-    }
+// Stage format (both engines): K boxes then V boxes; box b holds byte columns
+// [b*128, b*128+128) of 16 token rows, 16-byte chunk c of row r at chunk
+// position c ^ (r & 7) (the TMA 128-byte swizzle).
+template <typename T, int D>
+struct Ring {
+    static constexpr int E = sizeof(T);
+    static constexpr int ROWB = D * E;               // bytes per token row
+    static constexpr int NBOX = ROWB / 128;          // 128-byte boxes per row
+    static constexpr int KV_BYTES = NBOX * BOXB;     // one stage of K (or V)
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
 };
 
-// ------------------------------------------------------------ the kernel
+// Prefix sums of the partition counts per sequence, by all threads of the CTA;
+// fills lens_s[S] (clamped lengths) and pre[S + 1].  Ends with __syncthreads.
+template <int NTHREADS>
+__device__ void prefix_sums(const DecodeParams& p, int* lens_s, int* pre, int* wsum, int tid) {
+    constexpr int NW = NTHREADS / 32;
+    static_assert(NW <= 32, "one warp scans the warp totals");
+    const int warp = tid >> 5, lane = tid & 31;
+    const int per = (p.S + NTHREADS - 1) / NTHREADS;
+    const int beg = min(p.S, tid * per), end = min(p.S, beg + per);
+    int local = 0;
+    for (int k = beg; k < end; ++k) {
+        const int L = clamp_len(__ldg(p.lens + k), p);
+        lens_s[k] = L;
+        local += n_parts(L, p.P);
+    }
+    int incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = (lane < NW) ? wsum[lane] : 0;
+        int iv = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, iv, off);
+            if (lane >= off) iv += u;
+        }
+        if (lane < NW) wsum[lane] = iv - v;          // exclusive warp offsets
+    }
+    __syncthreads();
+    int run = wsum[warp] + incl - local;
+    for (int k = beg; k < end; ++k) {
+        pre[k] = run;
+        run += n_parts(lens_s[k], p.P);
+    }
+    if (tid == NTHREADS - 1) pre[p.S] = run;
+    __syncthreads();
+}
+
+// One pipeline's shared-memory rings, as seen by its producer.
+struct PipeRings {
+    uint8_t* stages;
+    uint64_t *full, *empty;     // per stage slot
+    uint64_t *ufull, *uempty;   // per unit slot
+    int* stage_ok;
+    int nst, nu;
+};
+
+// ================================================= producer warp
+// Per unit: the next unit's ticket (global atomic) and its first 64 block ids
+// are fetched while the current unit's stages are issued, so no global round
+// trip sits between two stages.  The TMA copies of a stage are issued by
+// several lanes at once.  desc_at(k) gives unit slot k's descriptor;
+// load_q(k, s, j, bar) (lane 0) arms `bar` and starts the copy of the
+// group's G query rows into slot k.
+template <typename T, int D, class DescAt, class LoadQ>
+__device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                              const DecodeParams& p, const PipeRings& rg, const int* pre,
+                              const int* lens_s, int U, volatile int* abort_flag, int lane,
+                              DescAt desc_at, LoadQ load_q) {
+    using R = Ring<T, D>;
+    constexpr int BOX_ELEMS = 128 / R::E;
+    const int nst = rg.nst, NU = rg.nu;
+    const uint64_t policy = policy_evict_first();
+    const int bs = p.bs, bsl = p.bs_log2;
+    const int npiece = (bs >= TOK) ? 1 : TOK / bs;   // blocks per stage
+    const int prow = (bs >= TOK) ? TOK : bs;         // box rows per block piece
+    struct Plan {
+        int u, s, j, i, t0, t1, nst, n_p, nblk;
+        const int32_t* trow;   // block-table entries of this unit's first block
+        int ids_a, ids_b;      // entries [win, win+32) and [win+32, win+64), one per lane
+    };
+    auto prepare = [&](int u) {
+        Plan q{};
+        q.u = u;
+        if (u >= U) return q;
+        const int x = u / p.Hkv;
+        int lo = 0, hi = p.S;                      // pre[lo] <= x < pre[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= x) lo = mid; else hi = mid;
+        }
+        q.s = lo;
+        q.i = x - pre[lo];
+        q.j = u - x * p.Hkv;
+        const int L = lens_s[lo];
+        q.t0 = min(q.i * p.P, L);
+        q.t1 = min(q.t0 + p.P, L);
+        q.nst = (q.t1 - q.t0 + TOK - 1) / TOK;
+        q.n_p = n_parts(L, p.P);
+        const int b0 = q.t0 >> bsl;
+        q.nblk = ((q.t1 + bs - 1) >> bsl) - b0;
+        q.trow = p.tables + (size_t)lo * p.mbps + b0;
+        q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
+        q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
+        return q;
+    };
+    int gstage = 0, st = 0, round = 0, ucount = 0;
+    int ticket = 0;
+    if (lane == 0) ticket = atomicAdd(&p.hdr->next_unit, 1);
+    Plan cur = prepare(__shfl_sync(0xffffffffu, ticket, 0));
+    bool ok = true;
+    while (ok) {
+        const int slot = ucount % NU;
+        if (ucount >= NU) {
+            bool w = true;
+            if (lane == 0) w = wait_or_abort(rg.uempty + slot, ((ucount / NU) - 1) & 1, abort_flag, p.err);
+            if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+        }
+        UnitDesc* d = desc_at(slot);
+        if (cur.u >= U) {
+            if (lane == 0) {
+                d->end = 1;
+                mbar_arrive(rg.ufull + slot);
+            }
+            ++ucount;
+            break;
+        }
+        if (lane == 0) {
+            d->s = cur.s; d->j = cur.j; d->i = cur.i; d->t0 = cur.t0; d->t1 = cur.t1;
+            d->n_p = cur.n_p;
+            d->stage_base = gstage; d->n_stages = cur.nst; d->end = 0;
+            load_q(slot, cur.s, cur.j, rg.ufull + slot);
+            ticket = atomicAdd(&p.hdr->next_unit, 1);     // the unit after this one
+        }
+        ++ucount;
+        Plan nxt{};
+        bool have_next = false;
+        int win = 0;                                // table index of ids_a's lane 0
+        const int b0 = cur.t0 >> bsl;
+        for (int c = 0; c < cur.nst; ++c) {
+            const int tok0 = cur.t0 + c * TOK;
+            if (round > 0) {
+                bool w = true;
+                if (lane == 0) w = wait_or_abort(rg.empty + st, (round - 1) & 1, abort_flag, p.err);
+                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+            }
+            // physical block of each piece (one piece unless bs = 8)
+            int blk0, blk1 = -2;
+            const int off0 = tok0 & (bs - 1);
+            {
+                const int bi = (tok0 >> bsl) - b0;
+                if (bi - win >= 32) {
+                    win += 32;
+                    cur.ids_a = cur.ids_b;
+                    cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
+                }
+                blk0 = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
+            }
+            if (npiece == 2) {
+                const int tok = tok0 + bs;
+                const int bi = (tok >> bsl) - b0;
+                if (bi - win >= 32) {
+                    win += 32;
+                    cur.ids_a = cur.ids_b;
+                    cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
+                }
+                const int id = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
+                if (tok < cur.t1) blk1 = id;
+            }
+            const bool has1 = blk1 != -2;
+            const bool valid = blk0 >= 0 && blk0 < p.NB && (!has1 || (blk1 >= 0 && blk1 < p.NB));
+            uint8_t* Kd = rg.stages + (size_t)st * R::STAGE_BYTES;
+            if (lane == 0) {
+                rg.stage_ok[st] = valid ? 1 : 0;
+                if (!valid) {
+                    set_err(p.err, PA_DEV_BAD_BLOCK);
+                    mbar_arrive(rg.full + st);
+                } else {
+                    mbar_arrive_expect_tx(rg.full + st, (has1 ? 2u : 1u) * 2u * prow * R::ROWB);
+                }
+            }
+            __syncwarp();
+            // one TMA box per lane: (piece, K or V, 128-byte column box)
+            const int nops = valid ? (has1 ? 2 : 1) * 2 * R::NBOX : 0;
+            if (lane < nops) {
+                const int piece = lane / (2 * R::NBOX), rem = lane % (2 * R::NBOX);
+                const int kv = rem / R::NBOX, b = rem % R::NBOX;
+                const int y = piece ? ((blk1 * p.Hkv + cur.j) << bsl)
+                                    : (((blk0 * p.Hkv + cur.j) << bsl) + off0);
+                uint8_t* dst = Kd + kv * R::KV_BYTES + b * BOXB + piece * 8 * 128;
+                tma_load_2d(dst, kv ? vmap : kmap, b * BOX_ELEMS, y, rg.full + st, policy);
+            }
+            ++gstage;
+            if (++st == nst) { st = 0; ++round; }
+            if (!have_next && (c == 3 || c == cur.nst - 1)) {
+                nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
+                have_next = true;
+            }
+        }
+        if (!ok) break;
+        if (!have_next) nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
+        cur = nxt;
+    }
+    // make sure no copy of this pipeline is still landing in shared memory
+    if (lane == 0) {
+        const int first = max(0, gstage - nst);
+        for (int g = first; g < gstage; ++g) mbar_wait(rg.full + g % nst, (g / nst) & 1);
+        const int ufirst = max(0, ucount - NU);
+        for (int k = ufirst; k < ucount; ++k) mbar_wait(rg.ufull + k % NU, (k / NU) & 1);
+    }
+    __syncwarp();
+}
+
+// Final split-K merge of sequence s, KV head j (n_p partitions), by `nthreads`
+// threads (t = 0 .. nthreads-1): out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i.
+template <typename T, int D, int G>
+__device__ void merge_partials(const DecodeParams& p, size_t sj, int s, int j, int n_p, int t,
+                               int nthreads) {
+    const size_t base = sj * p.n_pmax;
+    for (int idx = t; idx < G * D; idx += nthreads) {
+        const int g = idx / D, dd = idx % D;
+        float M = -INFINITY;
+        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
+        float Lsum = 0.f, O = 0.f;
+        if (M != -INFINITY) {
+            int i = 0;
+            for (; i + 4 <= n_p; i += 4) {
+                float mm[4], ll[4], oo[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const size_t pi = (base + i + k) * G + g;
+                    mm[k] = __ldcg(p.part_ml + pi * 2);
+                    ll[k] = __ldcg(p.part_ml + pi * 2 + 1);
+                    oo[k] = __ldcg(p.part_o + pi * D + dd);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float f = exp2f(mm[k] - M);
+                    Lsum += ll[k] * f;
+                    O += oo[k] * f;
+                }
+            }
+            for (; i < n_p; ++i) {
+                const size_t pi = (base + i) * G + g;
+                const float f = exp2f(__ldcg(p.part_ml + pi * 2) - M);
+                Lsum += __ldcg(p.part_ml + pi * 2 + 1) * f;
+                O += __ldcg(p.part_o + pi * D + dd) * f;
+            }
+        }
+        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + g) * D + dd;
+        *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+    }
+}
+
+// ------------------------------------------------------------ CUDA-core kernel
 // Warp roles: warp w belongs to pipeline w / PIPE_WARPS; role w % PIPE_WARPS is
 // 0 for the producer and 1..NCONS for the consumers.  The pipelines of a CTA
 // share nothing but the prefix sums and the abort flag; each takes its own
 // units from the global ticket counter.
-template <typename T, int D, int G, bool MMA>
-__global__ void __launch_bounds__(Layout<T, D, G, cons_for<MMA, G>()>::NTHREADS, 1)
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(Layout<T, D, G, cons_for<G>()>::NTHREADS, 1)
 decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
               DecodeParams p) {
-    using LY = Layout<T, D, G, cons_for<MMA, G>()>;
-    using Engine = typename std::conditional<MMA, MmaEngine<T, D, G>, CoreEngine<T, D, G>>::type;
+    using LY = Layout<T, D, G, cons_for<G>()>;
+    using Engine = CoreEngine<T, D, G>;
     constexpr int NCONS = LY::NCONS;
     constexpr int PIPE_WARPS = LY::PIPE_WARPS;
     constexpr int NPIPE = LY::NPIPE;
     constexpr int NTHREADS = LY::NTHREADS;
     constexpr int CT = NCONS * 32;               // consumer threads of a pipeline
     constexpr int E = sizeof(T);
-    constexpr int BOX_ELEMS = 128 / E;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 128B-swizzled TMA boxes need 1024-byte aligned destinations
@@ -536,197 +696,20 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
-
-    // ---- prefix sums of partitions per sequence (each CTA, tiny)
-    {
-        constexpr int NW = NTHREADS / 32;
-        const int per = (p.S + NTHREADS - 1) / NTHREADS;
-        const int beg = min(p.S, tid * per), end = min(p.S, beg + per);
-        int local = 0;
-        for (int k = beg; k < end; ++k) {
-            const int L = clamp_len(__ldg(p.lens + k), p);
-            lens_s[k] = L;
-            local += n_parts(L, p.P);
-        }
-        int incl = local;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        if (warp == 0) {
-            const int v = (lane < NW) ? wsum[lane] : 0;
-            int iv = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, iv, off);
-                if (lane >= off) iv += u;
-            }
-            if (lane < NW) wsum[lane] = iv - v;          // exclusive warp offsets
-        }
-        __syncthreads();
-        int run = wsum[warp] + incl - local;
-        for (int k = beg; k < end; ++k) {
-            pre[k] = run;
-            run += n_parts(lens_s[k], p.P);
-        }
-        if (tid == NTHREADS - 1) pre[p.S] = run;
-    }
-    __syncthreads();
+    prefix_sums<NTHREADS>(p, lens_s, pre, wsum, tid);
     const int U = pre[p.S] * p.Hkv;
 
     if (role == 0) {
-        // ================================================= producer warp
-        // Per unit: the next unit's ticket (global atomic) and its first 64
-        // block ids are fetched while the current unit's stages are issued,
-        // so no global round trip sits between two stages.  The TMA copies
-        // of a stage are issued by several lanes at once.
-        const uint64_t policy = policy_evict_first();
         const size_t qrow = (size_t)p.Hq * D * E;
-        const int bs = p.bs, bsl = p.bs_log2;
-        const int npiece = (bs >= TOK) ? 1 : TOK / bs;   // blocks per stage
-        const int prow = (bs >= TOK) ? TOK : bs;         // box rows per block piece
-        struct Plan {
-            int u, s, j, i, t0, t1, nst, n_p, nblk;
-            const int32_t* trow;   // block-table entries of this unit's first block
-            int ids_a, ids_b;      // entries [win, win+32) and [win+32, win+64), one per lane
-        };
-        auto prepare = [&](int u) {
-            Plan q{};
-            q.u = u;
-            if (u >= U) return q;
-            const int x = u / p.Hkv;
-            int lo = 0, hi = p.S;                      // pre[lo] <= x < pre[hi]
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (pre[mid] <= x) lo = mid; else hi = mid;
-            }
-            q.s = lo;
-            q.i = x - pre[lo];
-            q.j = u - x * p.Hkv;
-            const int L = lens_s[lo];
-            q.t0 = min(q.i * p.P, L);
-            q.t1 = min(q.t0 + p.P, L);
-            q.nst = (q.t1 - q.t0 + TOK - 1) / TOK;
-            q.n_p = n_parts(L, p.P);
-            const int b0 = q.t0 >> bsl;
-            q.nblk = ((q.t1 + bs - 1) >> bsl) - b0;
-            q.trow = p.tables + (size_t)lo * p.mbps + b0;
-            q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
-            q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
-            return q;
-        };
-        int gstage = 0, st = 0, round = 0, ucount = 0;
-        int ticket = 0;
-        if (lane == 0) ticket = atomicAdd(&p.hdr->next_unit, 1);
-        Plan cur = prepare(__shfl_sync(0xffffffffu, ticket, 0));
-        bool ok = true;
-        while (ok) {
-            const int slot = ucount % NUR;
-            if (ucount >= NUR) {
-                bool w = true;
-                if (lane == 0) w = wait_or_abort(uempty + slot, ((ucount / NUR) - 1) & 1, abort_flag, p.err);
-                if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-            }
-            UnitDesc* d = desc_at(slot);
-            if (cur.u >= U) {
-                if (lane == 0) {
-                    d->end = 1;
-                    mbar_arrive(ufull + slot);
-                }
-                ++ucount;
-                break;
-            }
-            if (lane == 0) {
-                d->s = cur.s; d->j = cur.j; d->i = cur.i; d->t0 = cur.t0; d->t1 = cur.t1;
-                d->n_p = cur.n_p;
-                d->stage_base = gstage; d->n_stages = cur.nst; d->end = 0;
-                mbar_arrive_expect_tx(ufull + slot, G * D * E);
-                bulk_g2s(q_at(slot),
-                         reinterpret_cast<const uint8_t*>(p.q) + (size_t)cur.s * qrow +
-                             (size_t)cur.j * G * D * E,
-                         G * D * E, ufull + slot);
-                ticket = atomicAdd(&p.hdr->next_unit, 1);     // the unit after this one
-            }
-            ++ucount;
-            Plan nxt{};
-            bool have_next = false;
-            int win = 0;                                // table index of ids_a's lane 0
-            const int b0 = cur.t0 >> bsl;
-            for (int c = 0; c < cur.nst; ++c) {
-                const int tok0 = cur.t0 + c * TOK;
-                if (round > 0) {
-                    bool w = true;
-                    if (lane == 0) w = wait_or_abort(empty + st, (round - 1) & 1, abort_flag, p.err);
-                    if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
-                }
-                // physical block of each piece (one piece unless bs = 8)
-                int blk0, blk1 = -2;
-                const int off0 = tok0 & (bs - 1);
-                {
-                    const int bi = (tok0 >> bsl) - b0;
-                    if (bi - win >= 32) {
-                        win += 32;
-                        cur.ids_a = cur.ids_b;
-                        cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
-                    }
-                    blk0 = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
-                }
-                if (npiece == 2) {
-                    const int tok = tok0 + bs;
-                    const int bi = (tok >> bsl) - b0;
-                    if (bi - win >= 32) {
-                        win += 32;
-                        cur.ids_a = cur.ids_b;
-                        cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
-                    }
-                    const int id = __shfl_sync(0xffffffffu, cur.ids_a, (bi - win) & 31);
-                    if (tok < cur.t1) blk1 = id;
-                }
-                const bool has1 = blk1 != -2;
-                const bool valid = blk0 >= 0 && blk0 < p.NB && (!has1 || (blk1 >= 0 && blk1 < p.NB));
-                uint8_t* Kd = stages + (size_t)st * LY::STAGE_BYTES;
-                if (lane == 0) {
-                    stage_ok[st] = valid ? 1 : 0;
-                    if (!valid) {
-                        set_err(p.err, PA_DEV_BAD_BLOCK);
-                        mbar_arrive(full + st);
-                    } else {
-                        mbar_arrive_expect_tx(full + st, (has1 ? 2u : 1u) * 2u * prow * LY::ROWB);
-                    }
-                }
-                __syncwarp();
-                // one TMA box per lane: (piece, K or V, 128-byte column box)
-                const int nops = valid ? (has1 ? 2 : 1) * 2 * LY::NBOX : 0;
-                if (lane < nops) {
-                    const int piece = lane / (2 * LY::NBOX), rem = lane % (2 * LY::NBOX);
-                    const int kv = rem / LY::NBOX, b = rem % LY::NBOX;
-                    const int y = piece ? ((blk1 * p.Hkv + cur.j) << bsl)
-                                        : (((blk0 * p.Hkv + cur.j) << bsl) + off0);
-                    uint8_t* dst = Kd + kv * LY::KV_BYTES + b * BOXB + piece * 8 * 128;
-                    tma_load_2d(dst, kv ? &vmap : &kmap, b * BOX_ELEMS, y, full + st, policy);
-                }
-                ++gstage;
-                if (++st == nst) { st = 0; ++round; }
-                if (!have_next && (c == 3 || c == cur.nst - 1)) {
-                    nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
-                    have_next = true;
-                }
-            }
-            if (!ok) break;
-            if (!have_next) nxt = prepare(__shfl_sync(0xffffffffu, ticket, 0));
-            cur = nxt;
-        }
-        // make sure no copy of this pipeline is still landing in shared memory
-        if (lane == 0) {
-            const int first = max(0, gstage - nst);
-            for (int g = first; g < gstage; ++g) mbar_wait(full + g % nst, (g / nst) & 1);
-            const int ufirst = max(0, ucount - NUR);
-            for (int k = ufirst; k < ucount; ++k) mbar_wait(ufull + k % NUR, (k / NUR) & 1);
-        }
-        __syncwarp();
+        PipeRings rg{stages, full, empty, ufull, uempty, stage_ok, nst, NUR};
+        producer_loop<T, D>(&kmap, &vmap, p, rg, pre, lens_s, U, abort_flag, lane, desc_at,
+                            [&](int slot, int s, int j, uint64_t* bar) {
+                                mbar_arrive_expect_tx(bar, G * D * E);
+                                bulk_g2s(q_at(slot),
+                                         reinterpret_cast<const uint8_t*>(p.q) + (size_t)s * qrow +
+                                             (size_t)j * G * D * E,
+                                         G * D * E, bar);
+                            });
     } else {
         // ================================================= consumer warps
         const int cw = role - 1;                 // 0 .. NCONS-1
@@ -735,24 +718,18 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         Engine eng;
         float* xs = scratch + cw * 3 * G * TOK;
         uint64_t* ps = reinterpret_cast<uint64_t*>(xs + G * TOK);
-        uint4* qf4 = reinterpret_cast<uint4*>(scratch + NCONS * 3 * G * TOK);   // fp32 q (core engine)
+        uint4* qf4 = reinterpret_cast<uint4*>(scratch + NCONS * 3 * G * TOK);   // fp32 q
         int ucount = 0;
         while (true) {
             const int slot = ucount % NUR;
-            // every lane waits; __all_sync reconverges the warp (the tensor-core
-            // engine's ldmatrix/mma are .aligned and need the whole warp) and
-            // makes the decision the same in every lane
-            if (!__all_sync(0xffffffffu, wait_or_abort(ufull + slot, (ucount / NUR) & 1, abort_flag, p.err)))
-                break;
+            // all consumer warps give up together, so none is left at a named barrier
+            const bool okw = wait_or_abort(ufull + slot, (ucount / NUR) & 1, abort_flag, p.err);
+            if (named_bar_or(bar_id, CT, !okw)) break;
             const UnitDesc d = *desc_at(slot);
             if (d.end) break;
-            if constexpr (MMA) {
-                eng.begin_unit(q_at(slot), lane, p.scale_log2e);
-            } else {
-                Engine::stage_q(q_at(slot), qf4, ctid, CT, p.scale_log2e);
-                named_bar_sync(bar_id, CT);                 // q in fp32 for every consumer warp
-                eng.begin_unit(qf4);
-            }
+            Engine::stage_q(q_at(slot), qf4, ctid, CT, p.scale_log2e);
+            named_bar_sync(bar_id, CT);                 // q in fp32 for every consumer warp
+            eng.begin_unit(qf4);
             int st = (d.stage_base + cw) % nst;
             uint32_t ph = ((d.stage_base + cw) / nst) & 1;
             for (int c = cw; c < d.n_stages; c += NCONS) {
@@ -760,12 +737,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                 if (have && stage_ok[st]) {
                     const int nv = min(TOK, d.t1 - (d.t0 + c * TOK));
                     uint8_t* Ks = stages + (size_t)st * LY::STAGE_BYTES;
-                    if constexpr (MMA) {
-                        eng.stage(Ks, Ks + LY::KV_BYTES, nv, p.scale_log2e, lane);
-                        if (nv < TOK) fence_proxy_async_smem();
-                    } else {
-                        eng.stage(Ks, Ks + LY::KV_BYTES, nv, xs, ps, lane);
-                    }
+                    eng.stage(Ks, Ks + LY::KV_BYTES, nv, xs, ps, lane);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(empty + st);
@@ -804,11 +776,11 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                     }
                 }
             }
+            if (d.n_p > 1) __threadfence();                      // publish the partials ...
             named_bar_sync(bar_id, CT);                          // merge buffer free again
             if (d.n_p > 1) {
                 if (ctid == 0) {
-                    __threadfence();                   // publish the partials before the count
-                    const int prev = atomicAdd(p.counters + sj, 1);
+                    const int prev = atomicAdd(p.counters + sj, 1);   // ... before the count
                     const int last = (prev == d.n_p - 1);
                     if (last) {
                         p.counters[sj] = 0;            // every partition has arrived
@@ -817,43 +789,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                     *last_flag = last;
                 }
                 named_bar_sync(bar_id, CT);
-                if (*last_flag) {
-                    const size_t base = sj * p.n_pmax;
-                    for (int idx = ctid; idx < G * D; idx += CT) {
-                        const int g = idx / D, dd = idx % D;
-                        float M = -INFINITY;
-                        for (int i = 0; i < d.n_p; ++i)
-                            M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
-                        float Lsum = 0.f, O = 0.f;
-                        if (M != -INFINITY) {
-                            int i = 0;
-                            for (; i + 4 <= d.n_p; i += 4) {
-                                float mm[4], ll[4], oo[4];
-#pragma unroll
-                                for (int k = 0; k < 4; ++k) {
-                                    const size_t pi = (base + i + k) * G + g;
-                                    mm[k] = __ldcg(p.part_ml + pi * 2);
-                                    ll[k] = __ldcg(p.part_ml + pi * 2 + 1);
-                                    oo[k] = __ldcg(p.part_o + pi * D + dd);
-                                }
-#pragma unroll
-                                for (int k = 0; k < 4; ++k) {
-                                    const float f = exp2f(mm[k] - M);
-                                    Lsum += ll[k] * f;
-                                    O += oo[k] * f;
-                                }
-                            }
-                            for (; i < d.n_p; ++i) {
-                                const size_t pi = (base + i) * G + g;
-                                const float f = exp2f(__ldcg(p.part_ml + pi * 2) - M);
-                                Lsum += __ldcg(p.part_ml + pi * 2 + 1) * f;
-                                O += __ldcg(p.part_o + pi * D + dd) * f;
-                            }
-                        }
-                        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)d.s * p.Hq + (size_t)d.j * G + g) * D + dd;
-                        *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
-                    }
-                }
+                if (*last_flag) merge_partials<T, D, G>(p, sj, d.s, d.j, d.n_p, ctid, CT);
                 named_bar_sync(bar_id, CT);                      // last_flag free again
             }
             ++ucount;
@@ -862,6 +798,613 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
     }
 
     __syncthreads();
+    if (tid == 0) {
+        __threadfence();
+        const int done = atomicAdd(&p.hdr->done_ctas, 1);
+        if (done == (int)gridDim.x - 1) {
+            p.hdr->next_unit = 0;
+            p.hdr->done_ctas = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ------------------------------------------------------------ tensor-core (tcgen05) kernel
+// A tcgen05 MMA instruction costs tens of cycles to issue whatever its size,
+// so the engine is shaped to cover many tokens per instruction and to keep
+// tensor memory small:
+//   S^T = K Q^T   M = 128 tokens (one stage), N = 16 (query heads, G used),
+//                 K = head_dim: head_dim/16 MMAs per stage
+//   O^T += V^T P^T  M = head_dim, N = 16, K = 16 tokens per MMA: 8 MMAs per
+//                 full stage.  O^T takes 16 columns of tensor memory.
+// Warps: 0-3 softmax (thread t = token t of the stage = tensor-memory lane t),
+// 4-7 epilogue (thread = head_dim row of O^T), 8 producer, 9 MMA issuer (one
+// thread).  Tensor memory: two S^T buffers and two O^T buffers (alternating
+// per unit, so a unit's epilogue overlaps the next unit).  The softmax keeps a
+// per-head reference max m that lags the true running max by at most 2^8
+// (exp2 units): only when a stage exceeds it is m moved (a barrier-OR vote
+// over the 128 threads), O^T rescaled in tensor memory and l rescaled.
+
+constexpr int TTOK = 128;           // tokens per stage
+constexpr int NHP = 16;             // query heads padded to the MMA's N
+constexpr float kRescaleLog2 = 8.f;
+constexpr int TC_THREADS = 320;
+constexpr int BAR_SOFTMAX = 1, BAR_EPI = 2;   // named barriers (128 threads each)
+
+template <typename T, int D, int G>
+struct TcLayout {
+    static_assert(sizeof(T) == 2, "tensor-core engine takes 16-bit types");
+    static_assert(G <= NHP, "query heads of a group must fit the MMA's N");
+    static constexpr int E = 2;
+    static constexpr int ROWB = D * E;
+    static constexpr int NBOX = ROWB / 128;            // 128-byte column boxes per token row
+    static constexpr int BOXT = TTOK * 128;            // one column box of a stage: 16 KB
+    static constexpr int KV_BYTES = NBOX * BOXT;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int NU = 2;                       // unit slots
+    static constexpr int QT = NBOX * 2 * 1024;         // Q tile: 16 rows x head_dim, 128B swizzle
+    static constexpr int PTB = TTOK * NHP * 2;         // one P^T tile (4 KB)
+    static constexpr uint32_t TM_COLS = 64;            // S^T x2 then O^T x2, 16 columns each
+    static constexpr int NBAR = 2 * NU + 14;           // + 2 per stage slot
+    // epilogue slot: ints s, j, i, n_p, n_stages, O buffer, 2 pad; m[16]; l[4][16]
+    static constexpr int ES = 32 + NHP * 4 + 4 * NHP * 4;
+    int nst, S;
+    __host__ __device__ TcLayout(int nst_, int S_) : nst(nst_), S(S_) {}
+    __host__ __device__ size_t q(int k) const { return (size_t)k * QT; }
+    __host__ __device__ size_t pt(int b) const { return (size_t)NU * QT + (size_t)b * PTB; }
+    __host__ __device__ size_t ring(int st) const {
+        return (size_t)NU * QT + 2 * (size_t)PTB + (size_t)st * STAGE_BYTES;
+    }
+    __host__ __device__ size_t desc(int k) const { return ring(nst) + (size_t)k * sizeof(UnitDesc); }
+    __host__ __device__ size_t bars() const { return desc(NU); }
+    __host__ __device__ size_t stage_ok() const { return bars() + (size_t)(2 * nst + NBAR) * 8; }
+    __host__ __device__ size_t red() const { return ((stage_ok() + (size_t)nst * 4 + 15) / 16) * 16; }
+    __host__ __device__ size_t epi(int e) const { return red() + 4 * NHP * 4 + (size_t)e * ES; }
+    __host__ __device__ size_t misc() const { return epi(2); }                  // 64 ints
+    __host__ __device__ size_t lens() const { return misc() + 256; }
+    __host__ __device__ size_t pre() const { return lens() + 4 * (size_t)S; }
+    __host__ __device__ size_t total() const { return pre() + 4 * (size_t)(S + 1); }
+};
+
+// Producer of the tensor-core engine: a 128-token stage is built from pieces of
+// 16 token rows (8 when bs = 8), each inside one block; one TMA box per
+// (piece, K or V, 128-byte column), at most two per lane.  stage_ok[slot] gets
+// the mask of pieces that were loaded; pieces past the unit's end are not.
+template <typename T, int D, int G>
+__device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
+                            const CUtensorMap* qmap, const DecodeParams& p, uint8_t* smem,
+                            const TcLayout<T, D, G>& ly, uint64_t* full, uint64_t* empty,
+                            uint64_t* ufull, uint64_t* uempty, int* stage_ok, const int* pre,
+                            const int* lens_s, int U, volatile int* abort_flag, int lane) {
+    using LY = TcLayout<T, D, G>;
+    constexpr int NU = LY::NU;
+    constexpr int BOX_ELEMS = 64;
+    constexpr uint32_t FULL = 0xffffffffu;
+    const int nst = ly.nst;
+    const uint64_t policy = policy_evict_first();
+    const int bs = p.bs, bsl = p.bs_log2;
+    const int PR = bs >= 16 ? 16 : bs;                // rows per piece
+    const int NPC = TTOK / PR;                         // pieces per stage
+    const int nops = NPC * 2 * LY::NBOX;               // <= 64
+    struct Plan {
+        int u, s, j, i, t0, t1, nst, n_p, nblk;
+        const int32_t* trow;
+        int ids_a, ids_b;
+    };
+    auto prepare = [&](int u) {
+        Plan q{};
+        q.u = u;
+        if (u >= U) return q;
+        const int x = u / p.Hkv;
+        int lo = 0, hi = p.S;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (pre[mid] <= x) lo = mid; else hi = mid;
+        }
+        q.s = lo;
+        q.i = x - pre[lo];
+        q.j = u - x * p.Hkv;
+        const int L = lens_s[lo];
+        q.t0 = min(q.i * p.P, L);
+        q.t1 = min(q.t0 + p.P, L);
+        q.nst = (q.t1 - q.t0 + TTOK - 1) / TTOK;
+        q.n_p = n_parts(L, p.P);
+        const int b0 = q.t0 >> bsl;
+        q.nblk = ((q.t1 + bs - 1) >> bsl) - b0;
+        q.trow = p.tables + (size_t)lo * p.mbps + b0;
+        q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
+        q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
+        return q;
+    };
+    int gstage = 0, st = 0, round = 0, ucount = 0, ticket = 0;
+    if (lane == 0) ticket = atomicAdd(&p.hdr->next_unit, 1);
+    Plan cur = prepare(__shfl_sync(FULL, ticket, 0));
+    bool ok = true;
+    while (ok) {
+        const int slot = ucount % NU;
+        if (ucount >= NU) {
+            bool w = true;
+            if (lane == 0) w = wait_or_abort(uempty + slot, ((ucount / NU) - 1) & 1, abort_flag, p.err);
+            if (!__shfl_sync(FULL, w, 0)) { ok = false; break; }
+        }
+        UnitDesc* d = reinterpret_cast<UnitDesc*>(smem + ly.desc(slot));
+        if (cur.u >= U) {
+            if (lane == 0) {
+                d->end = 1;
+                mbar_arrive(ufull + slot);
+            }
+            ++ucount;
+            break;
+        }
+        if (lane == 0) {
+            d->s = cur.s; d->j = cur.j; d->i = cur.i; d->t0 = cur.t0; d->t1 = cur.t1;
+            d->n_p = cur.n_p;
+            d->stage_base = gstage; d->n_stages = cur.nst; d->end = 0;
+            mbar_arrive_expect_tx(ufull + slot, G * D * 2);
+            uint8_t* qt = smem + ly.q(slot);
+#pragma unroll
+            for (int kc = 0; kc < LY::NBOX; ++kc)
+                tma_load_2d(qt + kc * 2048, qmap, kc * BOX_ELEMS, cur.s * p.Hq + cur.j * G,
+                            ufull + slot, policy);
+            ticket = atomicAdd(&p.hdr->next_unit, 1);
+        }
+        ++ucount;
+        Plan nxt{};
+        bool have_next = false;
+        int win = 0;
+        const int b0 = cur.t0 >> bsl;
+        for (int c = 0; c < cur.nst; ++c) {
+            const int tok0 = cur.t0 + c * TTOK;
+            if (round > 0) {
+                bool w = true;
+                if (lane == 0) w = wait_or_abort(empty + st, (round - 1) & 1, abort_flag, p.err);
+                if (!__shfl_sync(FULL, w, 0)) { ok = false; break; }
+            }
+            while ((tok0 >> bsl) - b0 - win >= 32) {      // keep the stage's blocks in the window
+                win += 32;
+                cur.ids_a = cur.ids_b;
+                cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
+            }
+            int blk[2], tok[2];
+            bool live[2];
+            uint32_t want = 0, got = 0;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int op = lane + 32 * r;
+                const int piece = op / (2 * LY::NBOX);
+                tok[r] = tok0 + piece * PR;
+                const bool exists = op < nops && tok[r] < cur.t1;
+                const int rel = exists ? (tok[r] >> bsl) - b0 - win : 0;   // 0 <= rel < 64
+                const int ia = __shfl_sync(FULL, cur.ids_a, rel & 31);
+                const int ib = __shfl_sync(FULL, cur.ids_b, rel & 31);
+                blk[r] = rel < 32 ? ia : ib;
+                live[r] = exists && blk[r] >= 0 && blk[r] < p.NB;
+                if (exists) want |= 1u << piece;
+                if (live[r]) got |= 1u << piece;
+            }
+            want = __reduce_or_sync(FULL, want);
+            got = __reduce_or_sync(FULL, got);
+            uint8_t* stage = smem + ly.ring(st);
+            if (lane == 0) {
+                stage_ok[st] = (int)got;
+                if (want & ~got) set_err(p.err, PA_DEV_BAD_BLOCK);
+                if (got)
+                    mbar_arrive_expect_tx(full + st, (uint32_t)__popc(got) * 2u * PR * LY::ROWB);
+                else
+                    mbar_arrive(full + st);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int op = lane + 32 * r;
+                if (live[r]) {
+                    const int piece = op / (2 * LY::NBOX), rem = op % (2 * LY::NBOX);
+                    const int kv = rem / LY::NBOX, b = rem % LY::NBOX;
+                    const int y = ((blk[r] * p.Hkv + cur.j) << bsl) + (tok[r] & (bs - 1));
+                    uint8_t* dst = stage + kv * LY::KV_BYTES + b * LY::BOXT + piece * PR * 128;
+                    tma_load_2d(dst, kv ? vmap : kmap, b * BOX_ELEMS, y, full + st, policy);
+                }
+            }
+            ++gstage;
+            if (++st == nst) { st = 0; ++round; }
+            if (!have_next) {
+                nxt = prepare(__shfl_sync(FULL, ticket, 0));
+                have_next = true;
+            }
+        }
+        if (!ok) break;
+        if (!have_next) nxt = prepare(__shfl_sync(FULL, ticket, 0));
+        cur = nxt;
+    }
+    if (lane == 0) {
+        const int first = max(0, gstage - nst);
+        for (int g = first; g < gstage; ++g) mbar_wait(full + g % nst, (g / nst) & 1);
+        const int ufirst = max(0, ucount - NU);
+        for (int k = ufirst; k < ucount; ++k) mbar_wait(ufull + k % NU, (k / NU) & 1);
+    }
+    __syncwarp();
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const __grid_constant__ CUtensorMap qmap, DecodeParams p) {
+    using LY = TcLayout<T, D, G>;
+    constexpr int NU = LY::NU;
+    constexpr uint32_t FULL = 0xffffffffu;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const LY ly(p.nst, p.S);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nst = p.nst;
+
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars());
+    uint64_t* empty = full + nst;
+    uint64_t* ufull = empty + nst;
+    uint64_t* uempty = ufull + NU;        // 5 arrivals: MMA issuer + the 4 softmax warps
+    uint64_t* s_full = uempty + NU;       // [2] S^T_g complete
+    uint64_t* p_full = s_full + 2;        // [2] P^T_g written (4 softmax warps)
+    uint64_t* o_bar = p_full + 2;         // PV of stage g complete (phase g)
+    uint64_t* o_done = o_bar + 1;         // [2] last PV of a unit complete (per O buffer)
+    uint64_t* o_free = o_done + 2;        // [2] O buffer read by the epilogue (4 warps)
+    uint64_t* epi_full = o_free + 2;      // [2] epilogue slot filled (4 softmax warps)
+    uint64_t* epi_empty = epi_full + 2;   // [2] epilogue slot read (4 epilogue warps)
+    uint64_t* fin = epi_empty + 2;        // issuer's final drain
+    int* stage_ok = reinterpret_cast<int*>(smem + ly.stage_ok());
+    float* red = reinterpret_cast<float*>(smem + ly.red());      // [4][16]
+    int* misc = reinterpret_cast<int*>(smem + ly.misc());
+    int* lens_s = reinterpret_cast<int*>(smem + ly.lens());
+    int* pre = reinterpret_cast<int*>(smem + ly.pre());
+    volatile int* abort_flag = misc + 0;
+    volatile int* last_flag = misc + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 60);   // outside the zeroed words
+    int* wsum = misc + 32;
+
+    if (tid == 0) {
+        const int n = 2 * nst + LY::NBAR;
+        for (int k = 0; k < n; ++k) mbar_init(full + k, 1);
+        for (int k = 0; k < NU; ++k) mbar_init(uempty + k, 5);
+        for (int k = 0; k < 2; ++k) {
+            mbar_init(p_full + k, 4);
+            mbar_init(o_free + k, 4);
+            mbar_init(epi_full + k, 4);
+            mbar_init(epi_empty + k, 4);
+        }
+        for (int k = 0; k < 32; ++k) misc[k] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tc::alloc(tmem_slot, LY::TM_COLS);
+        tc::relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        prefetch_tensormap(&qmap);
+    }
+    prefix_sums<TC_THREADS>(p, lens_s, pre, wsum, tid);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 2 * NHP;                 // + 16 * buffer
+    const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;          // this warp's lane quarter
+    const int U = pre[p.S] * p.Hkv;
+    const int PR = p.bs >= 16 ? 16 : p.bs;
+
+    if (warp == 8) {
+        // ================================================= producer warp
+        producer_tc<T, D, G>(&kmap, &vmap, &qmap, p, smem, ly, full, empty, ufull, uempty,
+                             stage_ok, pre, lens_s, U, abort_flag, lane);
+    } else if (warp == 9) {
+        // ================================================= MMA issuer (one thread)
+        // Order: S_0, S_1, PV_0, S_2, PV_1, ..., PV_last, so that the softmax
+        // of stage g overlaps the MMAs of stage g + 1.
+        if (lane == 0) {
+            constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, TTOK, NHP);
+            constexpr uint32_t ID_O = tc::idesc_f16<T>(true, true, D, NHP);
+            int ucount = 0, ocount = 0, g_prev = -1;
+            int prev_ob = 0, prev_oseq = 0, prev_nv = 0;
+            bool prev_first = false, prev_last = false, ok = true;
+            auto issue_pv = [&]() -> bool {
+                const int g = g_prev;
+                if (!wait_or_abort(p_full + (g & 1), (g >> 1) & 1, abort_flag, p.err)) return false;
+                if (prev_first && prev_oseq >= 2 &&
+                    !wait_or_abort(o_free + prev_ob, ((prev_oseq >> 1) - 1) & 1, abort_flag, p.err))
+                    return false;
+                tc::fence_after();
+                const int st = g % nst;
+                const uint32_t vb = smem_u32(smem + ly.ring(st) + LY::KV_BYTES);
+                const uint32_t pb = smem_u32(smem + ly.pt(g & 1));
+                const uint32_t od = tO + (uint32_t)(NHP * prev_ob);
+                const int nk = (prev_nv + 15) / 16;              // 16-token slices holding tokens
+                for (int kk = 0; kk < nk; ++kk)
+                    tc::mma_ss(od, tc::sdesc_sw128(vb + kk * 2048, LY::BOXT, 1024),
+                               tc::sdesc_none(pb + kk * 512, 256, 128), ID_O,
+                               (prev_first && kk == 0) ? 0u : 1u);
+                tc::commit(empty + st);          // the stage slot may be refilled
+                tc::commit(o_bar);
+                if (prev_last) tc::commit(o_done + prev_ob);
+                g_prev = -1;
+                return true;
+            };
+            while (ok) {
+                const int slot = ucount % NU;
+                if (!wait_or_abort(ufull + slot, (ucount / NU) & 1, abort_flag, p.err)) break;
+                const UnitDesc d = *reinterpret_cast<const UnitDesc*>(smem + ly.desc(slot));
+                if (d.end) break;
+                ++ucount;
+                if (d.n_stages == 0) {
+                    mbar_arrive(uempty + slot);
+                    continue;
+                }
+                const int oseq = ocount++;
+                const uint32_t qa = smem_u32(smem + ly.q(slot));
+                for (int c = 0; c < d.n_stages; ++c) {
+                    const int g = d.stage_base + c, st = g % nst;
+                    if (!wait_or_abort(full + st, (g / nst) & 1, abort_flag, p.err)) { ok = false; break; }
+                    tc::fence_after();
+                    const uint32_t kb = smem_u32(smem + ly.ring(st));
+                    const uint32_t sd = tS + (uint32_t)(NHP * (g & 1));
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        tc::mma_ss(sd, tc::sdesc_sw128(kb + (k >> 2) * LY::BOXT + (k & 3) * 32, 16, 1024),
+                                   tc::sdesc_sw128(qa + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), ID_S,
+                                   k > 0 ? 1u : 0u);
+                    tc::commit(s_full + (g & 1));
+                    if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
+                    if (g_prev >= 0 && !issue_pv()) { ok = false; break; }
+                    g_prev = g;
+                    prev_first = c == 0;
+                    prev_last = c == d.n_stages - 1;
+                    prev_ob = oseq & 1;
+                    prev_oseq = oseq;
+                    prev_nv = min(TTOK, d.t1 - (d.t0 + c * TTOK));
+                }
+                if (!ok) break;
+                if (!issue_pv()) break;        // the unit's last PV
+            }
+            // every MMA this thread issued has completed before tensor memory is freed
+            tc::commit(fin);
+            mbar_wait(fin, 0);
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ================================================= softmax warps (thread = token)
+        const int t = tid;
+        const int piece = t / PR;
+        int ucount = 0, ocount = 0;
+        while (true) {
+            // Every give-up decision is taken by all four warps together (an OR
+            // vote on their named barrier), so none is left waiting at a barrier.
+            const int slot = ucount % NU;
+            const int e = ucount & 1;
+            bool okw = wait_or_abort(ufull + slot, (ucount / NU) & 1, abort_flag, p.err);
+            if (ucount >= 2)
+                okw = okw && wait_or_abort(epi_empty + e, ((ucount >> 1) - 1) & 1, abort_flag, p.err);
+            if (named_bar_or(BAR_SOFTMAX, 128, !okw)) break;
+            const UnitDesc d = *reinterpret_cast<const UnitDesc*>(smem + ly.desc(slot));
+            uint8_t* es = smem + ly.epi(e);
+            int* hdr = reinterpret_cast<int*>(es);
+            float* em = reinterpret_cast<float*>(es + 32);
+            float* el = em + NHP;
+            if (d.end) {
+                if (t == 0) hdr[3] = -1;                  // tells the epilogue warps to stop
+                __syncwarp();
+                if (lane == 0) mbar_arrive(epi_full + e);
+                break;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(uempty + slot);
+            const int ob = ocount & 1;
+            float m_ref[G], l_part[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) { m_ref[h] = -INFINITY; l_part[h] = 0.f; }
+            bool ok = true;
+            for (int c = 0; c < d.n_stages; ++c) {
+                const int g = d.stage_base + c, st = g % nst, b = g & 1;
+                const bool okw = wait_or_abort(s_full + b, (g >> 1) & 1, abort_flag, p.err) &&
+                                 wait_or_abort(full + st, (g / nst) & 1, abort_flag, p.err);
+                if (named_bar_or(BAR_SOFTMAX, 128, !okw)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after();
+                uint32_t sr[NHP];
+                tc::ld16(tS + (uint32_t)(NHP * b) + lq, sr);
+                const bool valid = d.t0 + c * TTOK + t < d.t1 && ((stage_ok[st] >> piece) & 1);
+                float x[G];
+                bool over = false;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2e : -INFINITY;
+                    over |= x[h] > m_ref[h] + kRescaleLog2;
+                }
+                if (named_bar_or(BAR_SOFTMAX, 128, over)) {
+                    // move the reference max of the heads that outgrew it
+                    float mx[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        mx[h] = x[h];
+#pragma unroll
+                        for (int off = 16; off >= 1; off >>= 1)
+                            mx[h] = fmaxf(mx[h], __shfl_xor_sync(FULL, mx[h], off));
+                    }
+                    if (lane == 0)
+#pragma unroll
+                        for (int h = 0; h < G; ++h) red[warp * NHP + h] = mx[h];
+                    named_bar_sync(BAR_SOFTMAX, 128);
+                    float alpha[G];
+                    bool moved = false;
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float M = fmaxf(fmaxf(red[h], red[NHP + h]), fmaxf(red[2 * NHP + h], red[3 * NHP + h]));
+                        alpha[h] = 1.f;
+                        if (M > m_ref[h] + kRescaleLog2) {
+                            alpha[h] = exp2f(m_ref[h] - M);   // 0 while m was -inf
+                            m_ref[h] = M;
+                            l_part[h] *= alpha[h];
+                            moved = true;
+                        }
+                    }
+                    named_bar_sync(BAR_SOFTMAX, 128);      // red[] free again
+                    if (c > 0 && moved) {
+                        // O^T has stage g-1's PV in it and not yet stage g's
+                        const bool okw = wait_or_abort(o_bar, (g - 1) & 1, abort_flag, p.err);
+                        if (named_bar_or(BAR_SOFTMAX, 128, !okw)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after();
+                        uint32_t o[NHP];
+                        tc::ld16(tO + (uint32_t)(NHP * ob) + lq, o);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                        tc::st16(tO + (uint32_t)(NHP * ob) + lq, o);
+                    }
+                }
+                // P^T row t (16 heads, 16-bit), l sums the rounded weights the MMA uses
+                uint32_t pk[NHP / 2];
+#pragma unroll
+                for (int k = 0; k < NHP / 2; ++k) {
+                    float p0 = 0.f, p1 = 0.f;
+                    if (2 * k < G && valid) p0 = exp2f(x[2 * k] - m_ref[2 * k]);
+                    if (2 * k + 1 < G && valid) p1 = exp2f(x[2 * k + 1] - m_ref[2 * k + 1]);
+                    pk[k] = pack2<T>(p0, p1);
+                    if (2 * k < G) {
+                        float r2[2];
+                        Unpack<T>::run(pk[k], r2);
+                        l_part[2 * k] += r2[0];
+                        if (2 * k + 1 < G) l_part[2 * k + 1] += r2[1];
+                    }
+                }
+                uint8_t* ptile = smem + ly.pt(b) + (t >> 3) * 256 + (t & 7) * 16;
+                *reinterpret_cast<uint4*>(ptile) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                *reinterpret_cast<uint4*>(ptile + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                if (!valid) {
+                    // this token's V row must be finite (p = 0 meets it)
+                    uint8_t* vrow = smem + ly.ring(st) + LY::KV_BYTES + t * 128;
+#pragma unroll
+                    for (int ch = 0; ch < LY::ROWB / 16; ++ch)
+                        *reinterpret_cast<uint4*>(vrow + (ch >> 3) * LY::BOXT + (((ch & 7) ^ (t & 7)) << 4)) =
+                            make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+                tc::fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + b);
+            }
+            if (!ok) break;
+            // ---- hand (m, l partial sums, unit) to the epilogue warps
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float v = l_part[h];
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+                if (lane == 0) el[warp * NHP + h] = v;
+            }
+            if (t == 0) {
+                hdr[0] = d.s; hdr[1] = d.j; hdr[2] = d.i; hdr[3] = d.n_p;
+                hdr[4] = d.n_stages; hdr[5] = ob;
+#pragma unroll
+                for (int h = 0; h < G; ++h) em[h] = m_ref[h];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_full + e);
+            if (d.n_stages > 0) ++ocount;
+            ++ucount;
+        }
+        __syncwarp();
+    } else {
+        // ================================================= epilogue warps (thread = O^T row)
+        const int et = tid - 128;
+        // O^T row of this thread: M = 128 puts row r in lane r; M = 64 puts rows
+        // 16q..16q+15 in lanes 32q..32q+15
+        const int dd = (D == 128) ? et : ((lane < 16) ? 16 * (warp & 3) + lane : -1);
+        int ucount = 0, ocount = 0;
+        while (true) {
+            const int e = ucount & 1;
+            const bool okw = wait_or_abort(epi_full + e, (ucount >> 1) & 1, abort_flag, p.err);
+            if (named_bar_or(BAR_EPI, 128, !okw)) break;
+            const uint8_t* es = smem + ly.epi(e);
+            const int* hdr = reinterpret_cast<const int*>(es);
+            const int s = hdr[0], j = hdr[1], i = hdr[2], n_p = hdr[3], nstg = hdr[4], ob = hdr[5];
+            if (n_p < 0) break;
+            const float* em = reinterpret_cast<const float*>(es + 32);
+            const float* el = em + NHP;
+            float mh[G], lh[G], o[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                mh[h] = em[h];
+                lh[h] = (el[h] + el[NHP + h]) + (el[2 * NHP + h] + el[3 * NHP + h]);
+                o[h] = 0.f;
+            }
+            bool ok = true;
+            if (nstg > 0) {
+                const bool okd = wait_or_abort(o_done + ob, (ocount >> 1) & 1, abort_flag, p.err);
+                if (named_bar_or(BAR_EPI, 128, !okd)) {
+                    ok = false;
+                } else {
+                    tc::fence_after();
+                    uint32_t r[NHP];
+                    tc::ld16(tO + (uint32_t)(NHP * ob) + lq, r);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) o[h] = __uint_as_float(r[h]);
+                    tc::fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(o_free + ob);
+                }
+                ++ocount;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(epi_empty + e);   // slot copied out
+            if (!ok) break;
+            const size_t sj = (size_t)s * p.Hkv + j;
+            if (n_p == 1) {
+                if (dd >= 0)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h) * D + dd;
+                        *outp = DT<T>::from_float(lh[h] > 0.f ? o[h] / lh[h] : 0.f);
+                    }
+            } else {
+                if (dd >= 0)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const size_t pi = (sj * p.n_pmax + i) * G + h;
+                        p.part_o[pi * D + dd] = o[h];
+                        if (dd == 0) {
+                            p.part_ml[pi * 2 + 0] = mh[h];
+                            p.part_ml[pi * 2 + 1] = lh[h];
+                        }
+                    }
+                __threadfence();                           // publish the partials ...
+                named_bar_sync(BAR_EPI, 128);
+                if (et == 0) {
+                    const int prev = atomicAdd(p.counters + sj, 1);   // ... before the count
+                    const int last = (prev == n_p - 1);
+                    if (last) {
+                        p.counters[sj] = 0;                // every partition has arrived
+                        __threadfence();                   // see the other CTAs' partials
+                    }
+                    *last_flag = last;
+                }
+                named_bar_sync(BAR_EPI, 128);
+                if (*last_flag) merge_partials<T, D, G>(p, sj, s, j, n_p, et, 128);
+                named_bar_sync(BAR_EPI, 128);              // last_flag free again
+            }
+            ++ucount;
+        }
+        __syncwarp();
+    }
+
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after();
+        tc::dealloc(tmem, LY::TM_COLS);
+    }
     if (tid == 0) {
         __threadfence();
         const int done = atomicAdd(&p.hdr->done_ctas, 1);
@@ -893,8 +1436,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Tensor map over a cache viewed as [num_blocks*Hkv*bs rows][D columns]; box =
-// 128 bytes x box_rows, 128B swizzle.
+// Tensor map over a matrix of `rows` rows of D elements (a cache viewed as
+// [num_blocks*Hkv*bs][D], or the queries as [S*Hq][D]); box = 128 bytes x
+// box_rows, 128B swizzle.
 int make_map(CUtensorMap* map, const void* base, pa_dtype dt, int D, int64_t rows, int box_rows) {
     auto fn = encode_fn();
     if (!fn) return PA_ERR_CUDA;
@@ -948,7 +1492,7 @@ size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
 }
 
 struct Launch {
-    CUtensorMap kmap, vmap;
+    CUtensorMap kmap, vmap, qmap;
     DecodeParams p;
     dim3 grid;
     int threads;
@@ -956,59 +1500,87 @@ struct Launch {
     cudaStream_t stream;
 };
 
-template <typename T, int D, int G, bool MMA>
-int run_decode(Launch& L, const DevInfo& di) {
-    using LY = Layout<T, D, G, cons_for<MMA, G>()>;
-    auto kern = decode_kernel<T, D, G, MMA>;
-    // a stage costs its K/V bytes, two mbarriers and a validity flag; the
-    // rest of the layout is fixed; + 1024 bytes of alignment slack
+// Stage count per pipeline: as many as fit (at most kMaxStages).  `per_stage`
+// is what one more stage costs in every pipeline (its K/V bytes, two
+// mbarriers and a validity flag); + 1024 bytes of alignment slack.
+template <class LY>
+int pick_stages(const Launch& L, const DevInfo& di, size_t per_stage, int* nst_out, size_t* smem_out) {
     const size_t fixed = LY(0, L.p.S).total() + 1024 + 16;
-    const size_t per_stage = (size_t)LY::NPIPE * (LY::STAGE_BYTES + 2 * 8 + 4);
     if ((size_t)di.smem_optin < fixed + (size_t)kMinStages * per_stage) return PA_ERR_UNSUPPORTED;
     int nst = (int)((di.smem_optin - fixed) / per_stage);
     nst = std::min(nst, kMaxStages);
     while (nst > kMinStages && LY(nst, L.p.S).total() + 1024 > (size_t)di.smem_optin) --nst;
-    L.p.nst = nst;
-    L.smem = LY(nst, L.p.S).total() + 1024;
-    if (L.smem > (size_t)di.smem_optin) return PA_ERR_UNSUPPORTED;
-    L.threads = LY::NTHREADS;
-    static bool attr_set[64] = {};
+    *nst_out = nst;
+    *smem_out = LY(nst, L.p.S).total() + 1024;
+    return *smem_out > (size_t)di.smem_optin ? PA_ERR_UNSUPPORTED : PA_OK;
+}
+
+template <class Kern>
+int set_smem_attr(Kern kern, const DevInfo& di, bool* done) {
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (!attr_set[dev & 63]) {
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (!done[dev & 63]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, di.smem_optin) !=
             cudaSuccess)
             return PA_ERR_CUDA;
-        attr_set[dev & 63] = true;
+        done[dev & 63] = true;
     }
+    return PA_OK;
+}
+
+template <typename T, int D, int G>
+int run_decode_core(Launch& L, const DevInfo& di) {
+    using LY = Layout<T, D, G, cons_for<G>()>;
+    auto kern = decode_kernel<T, D, G>;
+    const size_t per_stage = (size_t)LY::NPIPE * (LY::STAGE_BYTES + 2 * 8 + 4);
+    int st = pick_stages<LY>(L, di, per_stage, &L.p.nst, &L.smem);
+    if (st != PA_OK) return st;
+    L.threads = LY::NTHREADS;
+    static bool attr_set[64] = {};
+    if ((st = set_smem_attr(kern, di, attr_set)) != PA_OK) return st;
     kern<<<L.grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 template <typename T, int D, int G>
-int dispatch_engine(Launch& L, const DevInfo& di, bool mma) {
-    if constexpr (sizeof(T) == 2) {
-        if (mma) return run_decode<T, D, G, true>(L, di);
+int run_decode_tc(Launch& L, const DevInfo& di) {
+    if constexpr (sizeof(T) != 2) {
+        return PA_ERR_UNSUPPORTED;
+    } else {
+        using LY = TcLayout<T, D, G>;
+        auto kern = decode_tc_kernel<T, D, G>;
+        const size_t per_stage = LY::STAGE_BYTES + 2 * 8 + 4;
+        int st = pick_stages<LY>(L, di, per_stage, &L.p.nst, &L.smem);
+        if (st != PA_OK) return st;
+        L.threads = TC_THREADS;
+        static bool attr_set[64] = {};
+        if ((st = set_smem_attr(kern, di, attr_set)) != PA_OK) return st;
+        kern<<<L.grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
+        return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     }
-    return run_decode<T, D, G, false>(L, di);
+}
+
+template <typename T, int D, int G>
+int dispatch_engine(Launch& L, const DevInfo& di, bool tensor) {
+    return tensor ? run_decode_tc<T, D, G>(L, di) : run_decode_core<T, D, G>(L, di);
 }
 
 template <typename T, int D>
-int dispatch_group(Launch& L, const DevInfo& di, int G, bool mma) {
+int dispatch_group(Launch& L, const DevInfo& di, int G, bool tensor) {
     switch (G) {
-        case 1: return dispatch_engine<T, D, 1>(L, di, mma);
-        case 2: return dispatch_engine<T, D, 2>(L, di, mma);
-        case 4: return dispatch_engine<T, D, 4>(L, di, mma);
-        case 8: return dispatch_engine<T, D, 8>(L, di, mma);
+        case 1: return dispatch_engine<T, D, 1>(L, di, tensor);
+        case 2: return dispatch_engine<T, D, 2>(L, di, tensor);
+        case 4: return dispatch_engine<T, D, 4>(L, di, tensor);
+        case 8: return dispatch_engine<T, D, 8>(L, di, tensor);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
 
 template <typename T>
-int dispatch_dim(Launch& L, const DevInfo& di, int D, int G, bool mma) {
+int dispatch_dim(Launch& L, const DevInfo& di, int D, int G, bool tensor) {
     switch (D) {
-        case 64: return dispatch_group<T, 64>(L, di, G, mma);
-        case 128: return dispatch_group<T, 128>(L, di, G, mma);
+        case 64: return dispatch_group<T, 64>(L, di, G, tensor);
+        case 128: return dispatch_group<T, 128>(L, di, G, tensor);
         default: return PA_ERR_UNSUPPORTED;
     }
 }
@@ -1024,7 +1596,7 @@ using namespace pa;
 extern "C" {
 
 int pa_set_decode_engine(int engine) {
-    if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_MMA) return PA_ERR_INVALID;
+    if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_TENSOR) return PA_ERR_INVALID;
     std::lock_guard<std::mutex> lk(g_mu);
     const int prev = g_engine;
     g_engine = engine;
@@ -1125,17 +1697,29 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         std::lock_guard<std::mutex> lk(g_mu);
         engine = g_engine;
     }
-    // The tensor-core engine is enabled only on request and only for G = 1:
-    // with G > 1 it failed (launch failure / timeouts) at full size under the
-    // multi-pipeline schedule for a cause not yet found, so it is not run.
-    const bool mma = engine == PA_ENGINE_MMA;
-    if (mma && (dtype == PA_F32 || G != 1)) return PA_ERR_UNSUPPORTED;
-    switch (dtype) {
-        case PA_F32: return dispatch_dim<float>(L, di, head_dim, G, false);
-        case PA_F16: return dispatch_dim<__half>(L, di, head_dim, G, mma);
-        case PA_BF16: return dispatch_dim<__nv_bfloat16>(L, di, head_dim, G, mma);
+    // tcgen05 engine: 16-bit types only; by default where query groups make
+    // the CUDA-core dot products the limit (G > 1)
+    const bool sixteen = dtype != PA_F32;
+    if (engine == PA_ENGINE_TENSOR && !sixteen) return PA_ERR_UNSUPPORTED;
+    const bool tensor = engine == PA_ENGINE_TENSOR || (engine == PA_ENGINE_AUTO && sixteen && G > 1);
+    auto run = [&](bool use_tensor) {
+        switch (dtype) {
+            case PA_F32: return dispatch_dim<float>(L, di, head_dim, G, false);
+            case PA_F16: return dispatch_dim<__half>(L, di, head_dim, G, use_tensor);
+            case PA_BF16: return dispatch_dim<__nv_bfloat16>(L, di, head_dim, G, use_tensor);
+        }
+        return (int)PA_ERR_INVALID;
+    };
+    if (tensor) {
+        st = make_map(&L.qmap, query, dtype, head_dim, (int64_t)num_seqs * num_q_heads, G);
+        if (st != PA_OK) return st;
+        st = run(true);
+        // by default, shapes whose stage ring does not fit (very many
+        // sequences) go to the CUDA-core engine
+        if (st == PA_ERR_UNSUPPORTED && engine == PA_ENGINE_AUTO) st = run(false);
+        return st;
     }
-    return PA_ERR_INVALID;
+    return run(false);
 }
 
 }  // extern "C"

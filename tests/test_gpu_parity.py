@@ -25,17 +25,23 @@ from tests.harness import (GpuRun, check_close, oracle_sampled, out_f64, sample_
 pytestmark = pytest.mark.gpu
 pa = pytest.importorskip("paged_kv_cache_426_b200")
 
-ENGINES = {"default": 0}
+# auto: tensor cores for 16-bit types with query groups, CUDA cores otherwise
+ENGINES = {"auto": 0, "core": 1, "tensor": 2}
+_current = ["auto"]
 
 
 @pytest.fixture(params=list(ENGINES))
 def engine(request):
     prev = pa.pa_set_decode_engine(ENGINES[request.param])
+    _current[0] = request.param
     yield request.param
+    _current[0] = "auto"
     pa.pa_set_decode_engine(prev)
 
 
 def run_full_compare(w, partition_size=None, steps=None):
+    if _current[0] == "tensor" and w.dtype == "f32":
+        pytest.skip("the tensor-core engine takes 16-bit types")
     rec = oracle.run(w, keep_prefill_cache=True, steps=steps)
     g = GpuRun(w, rec, partition_size=partition_size)
     g.replay_prefill()
@@ -140,30 +146,62 @@ def test_partition_sizes_agree(P):
     check_close(got[0].double().numpy(), ref[0].double().numpy(), "bf16", f"P={P} vs unsplit")
 
 
-@pytest.mark.parametrize("name,kw", [
-    ("mha", dict()), ("prefix", dict()), ("mha_bf16_d64", dict())])
-def test_mma_engine_g1(name, kw):
-    """The tensor-core engine (accepted for G = 1 only) against the oracle."""
-    prev = pa.pa_set_decode_engine(pa.PA_ENGINE_MMA)
+@pytest.mark.parametrize("engine_id", [1, 2])
+def test_physical_permutation_invariance_each_engine(engine_id):
+    w1 = workloads.gqa8b_bf16(num_seqs=6)
+    w2 = workloads.gqa8b_bf16(num_seqs=6)
+    w2.free_order = list(reversed(w2.free_order))
+    a, _ = _decode_outputs(w1, 64, engine_id)
+    b, _ = _decode_outputs(w2, 64, engine_id)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_tensor_engine_rejects_f32():
+    w = workloads.tiny_f32()
+    with pytest.raises(pa.PAError) as e:
+        _decode_outputs(w, 16, pa.PA_ENGINE_TENSOR)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("engine_id", [1, 2])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_growing_logits(engine_id, dtype):
+    """Logits that rise by far more than 2^8 (log2 units) along the sequence and
+    then fall: the running max moves many times within a unit, so the tensor
+    engine's deferred rescale of O in tensor memory is exercised."""
+    g = torch.Generator().manual_seed(5)
+    d, hkv, G, bs, L = 128, 2, 4, 16, 700
+    nb = (L + bs - 1) // bs
+    q = torch.randn(1, hkv * G, d, generator=g)
+    ramp = torch.cat([torch.linspace(0, 6, 400), torch.linspace(6, -3, L - 400)])
+    k = torch.randn(L, hkv, d, generator=g) * 0.3 + ramp[:, None, None] * q.view(hkv, G, d).mean(1)[None]
+    v = torch.randn(L, hkv, d, generator=g)
+    kc = torch.zeros(nb, hkv, bs, d)
+    vc = torch.zeros(nb, hkv, bs, d)
+    perm = torch.randperm(nb, generator=g)
+    for t in range(L):
+        kc[perm[t // bs], :, t % bs] = k[t]
+        vc[perm[t // bs], :, t % bs] = v[t]
+    q, kc, vc = q.to(dtype), kc.to(dtype), vc.to(dtype)
+    tab = perm.view(1, -1).to(torch.int32)
+    lens = torch.tensor([L], dtype=torch.int32)
+    name = "f16" if dtype == torch.float16 else "bf16"
+    ref = oracle.paged_decode(oracle.as_storage(q, name), oracle.as_storage(kc, name),
+                              oracle.as_storage(vc, name), tab.numpy(), lens.numpy(), 1.0, name)
+    prev = pa.pa_set_decode_engine(engine_id)
     try:
-        if name == "mha":
-            run_full_compare(workloads.mha7b_f16(steps=3, num_seqs=5), partition_size=64)
-        elif name == "prefix":
-            w = workloads.prefix_f16(n_req=6, plen=64, suffix_max=40, n_fork=2, heads=4)
-            run_full_compare(w, partition_size=32)
-        else:
-            w = workloads.custom("bf16", [1, 15, 16, 17, 100, 257], 2, 2, 64, 16, seed=5,
-                                 partition_size=64)
-            run_full_compare(w)
+        for P in (0, 256):
+            ws = pa.alloc_workspace(1, hkv * G, hkv, d, L, P)
+            out = torch.full_like(q, float("nan")).cuda()
+            err = torch.zeros(1, dtype=torch.int32, device="cuda")
+            pa.pa_decode(out, q.cuda(), kc.cuda(), vc.cuda(), tab.cuda(), lens.cuda(), L, 1.0,
+                         partition_size=P, workspace=ws, err_flag=err)
+            torch.cuda.synchronize()
+            assert err.item() == 0
+            check_close(out_f64(out, name), ref, name, f"growing logits P={P}")
     finally:
         pa.pa_set_decode_engine(prev)
-
-
-def test_mma_engine_rejects_groups():
-    w = workloads.gqa8b_bf16(num_seqs=2)
-    with pytest.raises(pa.PAError) as e:
-        _decode_outputs(w, 512, 2)
-    assert e.value.status == pa.PA_ERR_UNSUPPORTED
 
 
 # ---------------------------------------------------------------- edge cases
@@ -226,6 +264,38 @@ def test_bad_block_id_sets_flag_without_fault():
     pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, workspace=ws, err_flag=err)
     torch.cuda.synchronize()
     assert err.item() == 0
+
+
+def test_bad_block_id_tensor_engine():
+    d, bs, hkv, G = 128, 16, 2, 4
+    kc = torch.randn(4, hkv, bs, d, device="cuda").bfloat16()
+    vc = torch.randn(4, hkv, bs, d, device="cuda").bfloat16()
+    q = torch.randn(2, hkv * G, d, device="cuda").bfloat16()
+    tab = torch.tensor([[0, 9], [1, 2]], dtype=torch.int32, device="cuda")   # 9 >= num_blocks
+    lens = torch.tensor([20, 20], dtype=torch.int32, device="cuda")
+    ws = pa.alloc_workspace(2, hkv * G, hkv, d, 32, 16)
+    out = torch.zeros_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    prev = pa.pa_set_decode_engine(pa.PA_ENGINE_TENSOR)
+    try:
+        pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
+                     err_flag=err)
+        torch.cuda.synchronize()
+        assert err.item() == pa.PA_DEV_BAD_BLOCK
+        ref = oracle.paged_decode(oracle.as_storage(q.cpu()[1:], "bf16"),
+                                  oracle.as_storage(kc.cpu(), "bf16"),
+                                  oracle.as_storage(vc.cpu(), "bf16"), tab.cpu().numpy()[1:],
+                                  lens.cpu().numpy()[1:], 0.1, "bf16")
+        check_close(out_f64(out[1:], "bf16"), ref, "bf16", "the valid sequence is unaffected")
+        assert torch.isfinite(out[0].float()).all()
+        err.zero_()
+        tab[0, 1] = 3
+        pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
+                     err_flag=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+    finally:
+        pa.pa_set_decode_engine(prev)
 
 
 def test_bad_length_is_clamped_and_flagged():

@@ -813,19 +813,23 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
 // A tcgen05 MMA instruction costs tens of cycles to issue whatever its size,
 // so the engine is shaped to cover many tokens per instruction and to keep
 // tensor memory small:
-//   S^T = K Q^T   M = 128 tokens (one stage), N = 16 (query heads, G used),
+//   S^T = K Q^T   M = 64 tokens (one stage), N = 16 (query heads, G used),
 //                 K = head_dim: head_dim/16 MMAs per stage
-//   O^T += V^T P^T  M = head_dim, N = 16, K = 16 tokens per MMA: 8 MMAs per
+//   O^T += V^T P^T  M = head_dim, N = 16, K = 16 tokens per MMA: 4 MMAs per
 //                 full stage.  O^T takes 16 columns of tensor memory.
-// Warps: 0-3 softmax (thread t = token t of the stage = tensor-memory lane t),
-// 4-7 epilogue (thread = head_dim row of O^T), 8 producer, 9 MMA issuer (one
-// thread).  Tensor memory: two S^T buffers and two O^T buffers (alternating
+// A CTA needs little more than 100 KB of shared memory, so two run on each
+// SM: twice the stages in flight, two TMA producers and two MMA issuers, which
+// is what keeps HBM busy (a ring slot stays held for the copy's latency plus
+// the S -> softmax -> PV chain).
+// Warps: 0-3 softmax (thread = one token of the stage: with M = 64, rows
+// 16w..16w+15 sit in lanes 0-15 of warp w's lane quarter), 4-7 epilogue
+// (thread = head_dim row of O^T), 8 producer, 9 MMA issuer (one thread).  Tensor memory: two S^T buffers and two O^T buffers (alternating
 // per unit, so a unit's epilogue overlaps the next unit).  The softmax keeps a
 // per-head reference max m that lags the true running max by at most 2^8
 // (exp2 units): only when a stage exceeds it is m moved (a barrier-OR vote
 // over the 128 threads), O^T rescaled in tensor memory and l rescaled.
 
-constexpr int TTOK = 128;           // tokens per stage
+constexpr int TTOK = 64;            // tokens per stage (= M of the S^T MMA)
 constexpr int NHP = 16;             // query heads padded to the MMA's N
 constexpr float kRescaleLog2 = 8.f;
 constexpr int TC_THREADS = 320;
@@ -838,12 +842,12 @@ struct TcLayout {
     static constexpr int E = 2;
     static constexpr int ROWB = D * E;
     static constexpr int NBOX = ROWB / 128;            // 128-byte column boxes per token row
-    static constexpr int BOXT = TTOK * 128;            // one column box of a stage: 16 KB
+    static constexpr int BOXT = TTOK * 128;            // one column box of a stage: 8 KB
     static constexpr int KV_BYTES = NBOX * BOXT;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int NU = 2;                       // unit slots
     static constexpr int QT = NBOX * 2 * 1024;         // Q tile: 16 rows x head_dim, 128B swizzle
-    static constexpr int PTB = TTOK * NHP * 2;         // one P^T tile (4 KB)
+    static constexpr int PTB = TTOK * NHP * 2;         // one P^T tile (2 KB)
     static constexpr uint32_t TM_COLS = 64;            // S^T x2 then O^T x2, 16 columns each
     static constexpr int NBAR = 2 * NU + 14;           // + 2 per stage slot
     // epilogue slot: ints s, j, i, n_p, n_stages, O buffer, 2 pad; m[16]; l[4][16]
@@ -1026,7 +1030,7 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, 2)
 decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                  const __grid_constant__ CUtensorMap qmap, DecodeParams p) {
     using LY = TcLayout<T, D, G>;
@@ -1099,72 +1103,112 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                              stage_ok, pre, lens_s, U, abort_flag, lane);
     } else if (warp == 9) {
         // ================================================= MMA issuer (one thread)
-        // Order: S_0, S_1, PV_0, S_2, PV_1, ..., PV_last, so that the softmax
-        // of stage g overlaps the MMAs of stage g + 1.
+        // Event driven: the thread polls the next stage's data (-> S MMAs) and
+        // the oldest pending stage's P (-> PV MMAs) and issues whichever is
+        // ready, so a PV never waits for the next stage's copy.  S_g is issued
+        // only once PV_{g-2} has been (its S^T and P^T buffers are reused).
         if (lane == 0) {
             constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, TTOK, NHP);
             constexpr uint32_t ID_O = tc::idesc_f16<T>(true, true, D, NHP);
-            int ucount = 0, ocount = 0, g_prev = -1;
-            int prev_ob = 0, prev_oseq = 0, prev_nv = 0;
-            bool prev_first = false, prev_last = false, ok = true;
-            auto issue_pv = [&]() -> bool {
-                const int g = g_prev;
-                if (!wait_or_abort(p_full + (g & 1), (g >> 1) & 1, abort_flag, p.err)) return false;
-                if (prev_first && prev_oseq >= 2 &&
-                    !wait_or_abort(o_free + prev_ob, ((prev_oseq >> 1) - 1) & 1, abort_flag, p.err))
-                    return false;
-                tc::fence_after();
-                const int st = g % nst;
-                const uint32_t vb = smem_u32(smem + ly.ring(st) + LY::KV_BYTES);
-                const uint32_t pb = smem_u32(smem + ly.pt(g & 1));
-                const uint32_t od = tO + (uint32_t)(NHP * prev_ob);
-                const int nk = (prev_nv + 15) / 16;              // 16-token slices holding tokens
-                for (int kk = 0; kk < nk; ++kk)
-                    tc::mma_ss(od, tc::sdesc_sw128(vb + kk * 2048, LY::BOXT, 1024),
-                               tc::sdesc_none(pb + kk * 512, 256, 128), ID_O,
-                               (prev_first && kk == 0) ? 0u : 1u);
-                tc::commit(empty + st);          // the stage slot may be refilled
-                tc::commit(o_bar);
-                if (prev_last) tc::commit(o_done + prev_ob);
-                g_prev = -1;
-                return true;
+            struct Pending {
+                int g, nv, oseq;
+                bool first, last;
             };
-            while (ok) {
-                const int slot = ucount % NU;
-                if (!wait_or_abort(ufull + slot, (ucount / NU) & 1, abort_flag, p.err)) break;
-                const UnitDesc d = *reinterpret_cast<const UnitDesc*>(smem + ly.desc(slot));
-                if (d.end) break;
-                ++ucount;
-                if (d.n_stages == 0) {
-                    mbar_arrive(uempty + slot);
-                    continue;
+            Pending pend0{}, pend1{};            // S issued, PV not yet (pend0 oldest)
+            int npend = 0;
+            int ucount = 0, ocount = 0, c = 0, oseq = 0, slot = 0;
+            bool have = false, s_done = false, ok = true;
+            UnitDesc d{};
+            uint32_t idle = 0;
+            uint64_t t_idle = 0;
+            while (true) {
+                bool prog = false;
+                // ---- the next unit, for the S side
+                if (!have && !s_done) {
+                    slot = ucount % NU;
+                    if (mbar_test(ufull + slot, (ucount / NU) & 1)) {
+                        d = *reinterpret_cast<const UnitDesc*>(smem + ly.desc(slot));
+                        prog = true;
+                        if (d.end) {
+                            s_done = true;
+                        } else {
+                            ++ucount;
+                            if (d.n_stages == 0) {
+                                mbar_arrive(uempty + slot);
+                            } else {
+                                have = true;
+                                c = 0;
+                                oseq = ocount++;
+                            }
+                        }
+                    }
                 }
-                const int oseq = ocount++;
-                const uint32_t qa = smem_u32(smem + ly.q(slot));
-                for (int c = 0; c < d.n_stages; ++c) {
+                // ---- O^T += V^T P^T of the oldest pending stage
+                if (npend > 0) {
+                    const Pending r = pend0;
+                    const int ob = r.oseq & 1;
+                    bool ready = mbar_test(p_full + (r.g & 1), (r.g >> 1) & 1);
+                    if (ready && r.first && r.oseq >= 2)   // the epilogue has read this O^T buffer
+                        ready = mbar_test(o_free + ob, ((r.oseq >> 1) - 1) & 1);
+                    if (ready) {
+                        tc::fence_after();
+                        const int st = r.g % nst;
+                        const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st) + LY::KV_BYTES), LY::BOXT, 1024);
+                        const uint64_t b0 = tc::sdesc_none(smem_u32(smem + ly.pt(r.g & 1)), 256, 128);
+                        const uint32_t od = tO + (uint32_t)(NHP * ob);
+                        const int nk = (r.nv + 15) / 16;             // 16-token slices holding tokens
+                        for (int kk = 0; kk < nk; ++kk)
+                            tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
+                                       (r.first && kk == 0) ? 0u : 1u);
+                        tc::commit(empty + st);          // the stage slot may be refilled
+                        tc::commit(o_bar);
+                        if (r.last) tc::commit(o_done + ob);
+                        pend0 = pend1;
+                        --npend;
+                        prog = true;
+                    }
+                }
+                // ---- S^T of the unit's next stage
+                if (have && npend < 2) {
                     const int g = d.stage_base + c, st = g % nst;
-                    if (!wait_or_abort(full + st, (g / nst) & 1, abort_flag, p.err)) { ok = false; break; }
-                    tc::fence_after();
-                    const uint32_t kb = smem_u32(smem + ly.ring(st));
-                    const uint32_t sd = tS + (uint32_t)(NHP * (g & 1));
+                    if (mbar_test(full + st, (g / nst) & 1)) {
+                        tc::fence_after();
+                        const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
+                        const uint64_t b0 = tc::sdesc_sw128(smem_u32(smem + ly.q(slot)), 16, 1024);
+                        const uint32_t sd = tS + (uint32_t)(NHP * (g & 1));
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        tc::mma_ss(sd, tc::sdesc_sw128(kb + (k >> 2) * LY::BOXT + (k & 3) * 32, 16, 1024),
-                                   tc::sdesc_sw128(qa + (k >> 2) * 2048 + (k & 3) * 32, 16, 1024), ID_S,
-                                   k > 0 ? 1u : 0u);
-                    tc::commit(s_full + (g & 1));
-                    if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
-                    if (g_prev >= 0 && !issue_pv()) { ok = false; break; }
-                    g_prev = g;
-                    prev_first = c == 0;
-                    prev_last = c == d.n_stages - 1;
-                    prev_ob = oseq & 1;
-                    prev_oseq = oseq;
-                    prev_nv = min(TTOK, d.t1 - (d.t0 + c * TTOK));
+                        for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
+                            tc::mma_ss(sd, a0 + (uint64_t)((k >> 2) * (LY::BOXT >> 4) + (k & 3) * 2),
+                                       b0 + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), ID_S, k > 0 ? 1u : 0u);
+                        tc::commit(s_full + (g & 1));
+                        if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
+                        const Pending nw{g, min(TTOK, d.t1 - (d.t0 + c * TTOK)), oseq, c == 0,
+                                         c == d.n_stages - 1};
+                        if (npend == 0) pend0 = nw; else pend1 = nw;
+                        ++npend;
+                        if (++c == d.n_stages) have = false;
+                        prog = true;
+                    }
                 }
-                if (!ok) break;
-                if (!issue_pv()) break;        // the unit's last PV
+                if (s_done && !have && npend == 0) break;
+                if (prog) {
+                    idle = 0;
+                } else if ((++idle & 255) == 0) {
+                    // bounded: give up after kWaitLimitNs without progress, or when
+                    // another warp has given up
+                    if (*abort_flag) { ok = false; break; }
+                    const uint64_t now = global_ns();
+                    if (idle == 256) {
+                        t_idle = now;
+                    } else if (now - t_idle > kWaitLimitNs) {
+                        set_err(p.err, PA_DEV_TIMEOUT);
+                        *abort_flag = 1;
+                        ok = false;
+                        break;
+                    }
+                }
             }
+            (void)ok;
             // every MMA this thread issued has completed before tensor memory is freed
             tc::commit(fin);
             mbar_wait(fin, 0);
@@ -1172,8 +1216,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         __syncwarp();
     } else if (warp < 4) {
         // ================================================= softmax warps (thread = token)
-        const int t = tid;
-        const int piece = t / PR;
+        const int t = lane < 16 ? 16 * warp + lane : -1;    // stage token of this thread (M = 64 layout)
+        const int piece = t >= 0 ? t / PR : 0;
         int ucount = 0, ocount = 0;
         while (true) {
             // Every give-up decision is taken by all four warps together (an OR
@@ -1204,16 +1248,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
             bool ok = true;
             for (int c = 0; c < d.n_stages; ++c) {
                 const int g = d.stage_base + c, st = g % nst, b = g & 1;
-                const bool okw = wait_or_abort(s_full + b, (g >> 1) & 1, abort_flag, p.err) &&
-                                 wait_or_abort(full + st, (g / nst) & 1, abort_flag, p.err);
-                if (named_bar_or(BAR_SOFTMAX, 128, !okw)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after();
+                const bool okw = __all_sync(FULL, wait_or_abort(s_full + b, (g >> 1) & 1, abort_flag, p.err) &&
+                                                      wait_or_abort(full + st, (g / nst) & 1, abort_flag, p.err));
                 uint32_t sr[NHP];
-                tc::ld16(tS + (uint32_t)(NHP * b) + lq, sr);
-                const bool valid = d.t0 + c * TTOK + t < d.t1 && ((stage_ok[st] >> piece) & 1);
+                if (okw) {
+                    tc::fence_after();
+                    tc::ld16(tS + (uint32_t)(NHP * b) + lq, sr);
+                }
+                const bool valid = okw && t >= 0 && d.t0 + c * TTOK + t < d.t1 && ((stage_ok[st] >> piece) & 1);
                 float x[G];
                 bool over = false;
 #pragma unroll
@@ -1221,7 +1263,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                     x[h] = valid ? __uint_as_float(sr[h]) * p.scale_log2e : -INFINITY;
                     over |= x[h] > m_ref[h] + kRescaleLog2;
                 }
-                if (named_bar_or(BAR_SOFTMAX, 128, over)) {
+                // one vote: some head outgrew its reference max, or a wait gave up
+                if (named_bar_or(BAR_SOFTMAX, 128, over || !okw)) {
+                    if (named_bar_or(BAR_SOFTMAX, 128, !okw)) {
+                        ok = false;
+                        break;
+                    }
                     // move the reference max of the heads that outgrew it
                     float mx[G];
 #pragma unroll
@@ -1279,10 +1326,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         if (2 * k + 1 < G) l_part[2 * k + 1] += r2[1];
                     }
                 }
-                uint8_t* ptile = smem + ly.pt(b) + (t >> 3) * 256 + (t & 7) * 16;
-                *reinterpret_cast<uint4*>(ptile) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4*>(ptile + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                if (!valid) {
+                if (t >= 0) {
+                    uint8_t* ptile = smem + ly.pt(b) + (t >> 3) * 256 + (t & 7) * 16;
+                    *reinterpret_cast<uint4*>(ptile) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    *reinterpret_cast<uint4*>(ptile + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+                if (t >= 0 && !valid) {
                     // this token's V row must be finite (p = 0 meets it)
                     uint8_t* vrow = smem + ly.ring(st) + LY::KV_BYTES + t * 128;
 #pragma unroll
@@ -1458,7 +1507,8 @@ int make_map(CUtensorMap* map, const void* base, pa_dtype dt, int D, int64_t row
 
 struct DevInfo {
     int sms = 0;
-    int smem_optin = 0;
+    int smem_optin = 0;     // per CTA
+    int smem_sm = 0;        // per SM
 };
 
 int dev_info(DevInfo* out) {
@@ -1470,6 +1520,8 @@ int dev_info(DevInfo* out) {
     if (!have[dev]) {
         if (cudaDeviceGetAttribute(&cache[dev].sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&cache[dev].smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess ||
+            cudaDeviceGetAttribute(&cache[dev].smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
                 cudaSuccess)
             return PA_ERR_CUDA;
         have[dev] = true;
@@ -1494,25 +1546,27 @@ size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
 struct Launch {
     CUtensorMap kmap, vmap, qmap;
     DecodeParams p;
+    int64_t units_ub;       // upper bound on the number of work units
     dim3 grid;
     int threads;
     size_t smem;
     cudaStream_t stream;
 };
 
-// Stage count per pipeline: as many as fit (at most kMaxStages).  `per_stage`
-// is what one more stage costs in every pipeline (its K/V bytes, two
-// mbarriers and a validity flag); + 1024 bytes of alignment slack.
+// Stage count per pipeline: as many as fit in `budget` bytes of shared memory
+// (at most kMaxStages).  `per_stage` is what one more stage costs in every
+// pipeline (its K/V bytes, two mbarriers and a validity flag); + 1024 bytes
+// of alignment slack.
 template <class LY>
-int pick_stages(const Launch& L, const DevInfo& di, size_t per_stage, int* nst_out, size_t* smem_out) {
+int pick_stages(const Launch& L, size_t budget, size_t per_stage, int* nst_out, size_t* smem_out) {
     const size_t fixed = LY(0, L.p.S).total() + 1024 + 16;
-    if ((size_t)di.smem_optin < fixed + (size_t)kMinStages * per_stage) return PA_ERR_UNSUPPORTED;
-    int nst = (int)((di.smem_optin - fixed) / per_stage);
+    if (budget < fixed + (size_t)kMinStages * per_stage) return PA_ERR_UNSUPPORTED;
+    int nst = (int)((budget - fixed) / per_stage);
     nst = std::min(nst, kMaxStages);
-    while (nst > kMinStages && LY(nst, L.p.S).total() + 1024 > (size_t)di.smem_optin) --nst;
+    while (nst > kMinStages && LY(nst, L.p.S).total() + 1024 > budget) --nst;
     *nst_out = nst;
     *smem_out = LY(nst, L.p.S).total() + 1024;
-    return *smem_out > (size_t)di.smem_optin ? PA_ERR_UNSUPPORTED : PA_OK;
+    return *smem_out > budget ? PA_ERR_UNSUPPORTED : PA_OK;
 }
 
 template <class Kern>
@@ -1533,7 +1587,7 @@ int run_decode_core(Launch& L, const DevInfo& di) {
     using LY = Layout<T, D, G, cons_for<G>()>;
     auto kern = decode_kernel<T, D, G>;
     const size_t per_stage = (size_t)LY::NPIPE * (LY::STAGE_BYTES + 2 * 8 + 4);
-    int st = pick_stages<LY>(L, di, per_stage, &L.p.nst, &L.smem);
+    int st = pick_stages<LY>(L, (size_t)di.smem_optin, per_stage, &L.p.nst, &L.smem);
     if (st != PA_OK) return st;
     L.threads = LY::NTHREADS;
     static bool attr_set[64] = {};
@@ -1549,13 +1603,17 @@ int run_decode_tc(Launch& L, const DevInfo& di) {
     } else {
         using LY = TcLayout<T, D, G>;
         auto kern = decode_tc_kernel<T, D, G>;
+        // two CTAs per SM: each gets half of the SM's shared memory (less the
+        // 1 KB the system reserves per CTA)
+        const size_t budget = std::min<size_t>((size_t)di.smem_optin, (size_t)di.smem_sm / 2 - 1024);
         const size_t per_stage = LY::STAGE_BYTES + 2 * 8 + 4;
-        int st = pick_stages<LY>(L, di, per_stage, &L.p.nst, &L.smem);
+        int st = pick_stages<LY>(L, budget, per_stage, &L.p.nst, &L.smem);
         if (st != PA_OK) return st;
         L.threads = TC_THREADS;
         static bool attr_set[64] = {};
         if ((st = set_smem_attr(kern, di, attr_set)) != PA_OK) return st;
-        kern<<<L.grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
+        const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>(L.units_ub, 2 * (int64_t)di.sms)));
+        kern<<<grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
         return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     }
 }
@@ -1689,6 +1747,7 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     p.err = err_flag;
 
     const int64_t units_ub = (int64_t)num_seqs * num_kv_heads * n_pmax;
+    L.units_ub = units_ub;
     L.grid = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(units_ub, di.sms)));
     L.stream = (cudaStream_t)stream;
 

@@ -264,9 +264,12 @@ class Session:
         return n + 1
 
     def decode(self, st, out):
+        """One pa_decode call: the decode kernel, plus the split-K merge kernel
+        when a sequence can span several partitions.  Returns the launches."""
         self.pa.pa_decode(out, st["q"], self.kc, self.vc, st["tab"], st["lens"], self.max_len,
                           self.w.scale, partition_size=self.P, workspace=self.ws,
                           err_flag=self.err)
+        return 2 if 0 < self.P < self.max_len else 1
 
     def bytes_of(self, lens):
         w = self.w
@@ -312,8 +315,7 @@ def run_ours(args, rank, world, local):
         ev[i][0].record(stream)
         launches += sess.run_step(st, out)
         ev[i][1].record(stream)
-        sess.decode(st, out)
-        launches += 1
+        launches += sess.decode(st, out)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     barrier(world)

@@ -97,7 +97,8 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * fp32 accumulation; out is rounded to nearest even in dtype.  L = 0 gives 0.
  * Long contexts are split into partitions of `partition_size` tokens
  * (a positive multiple of 16; 0 = one partition per sequence) whose partial
- * results are merged with their log-sum-exp weights in the same launch.
+ * results are merged with their log-sum-exp weights by a second kernel that
+ * pa_decode launches on the same stream (only when some sequence is split).
  *   out           device [num_seqs][num_q_heads][head_dim] dtype
  *   query         device [num_seqs][num_q_heads][head_dim] dtype, 16-B aligned
  *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past
@@ -153,8 +154,9 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
  * dot products on CUDA cores (any dtype).  PA_ENGINE_TENSOR: tcgen05
  * tensor-core MMAs with accumulators in tensor memory, f16/bf16 only (f32
  * returns PA_ERR_UNSUPPORTED).  PA_ENGINE_AUTO (the default): the tensor
- * engine for f16/bf16 with query groups (num_q_heads > num_kv_heads), CUDA
- * cores otherwise.  Process-wide; returns the previous value. */
+ * engine for f16/bf16 (falling back to CUDA cores for batches too large for
+ * its shared-memory ring), CUDA cores for f32.  Process-wide; returns the
+ * previous value. */
 enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_TENSOR = 2 };
 int pa_set_decode_engine(int engine);
 

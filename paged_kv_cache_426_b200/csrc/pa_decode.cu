@@ -33,11 +33,10 @@
 //        whole unit.  The running max is only moved when it grows by more
 //        than 2^8, so O is rescaled rarely (exact: O, l and m stay
 //        consistent).
-//  * A single-partition sequence writes `out` directly.  Otherwise the unit
-//    writes (m, l, o) to the workspace and bumps a per-(s, j) counter; the
-//    CTA that completes the last partition merges all partials with their
-//    log-sum-exp weights and writes `out` (and re-zeroes the counter).  No
-//    CTA ever waits for another.
+//  * A single-partition sequence writes `out` directly.  Otherwise each unit
+//    writes its (m, l, o) to the workspace and a second, fully parallel
+//    kernel (one CTA per sequence and query head) merges the partitions with
+//    their log-sum-exp weights.  No CTA ever waits for another.
 //  * Summation order depends only on logical positions (stage index within
 //    the unit, warp index, partition index), never on physical block ids or
 //    on which CTA ran a unit, so results are bit-identical under any
@@ -87,7 +86,6 @@ struct DecodeParams {
     int mbps, max_len, S, Hq, Hkv, NB, bs, bs_log2, P, n_pmax, nst;
     float scale_log2e;
     WsHeader* hdr;
-    int* counters;     // [S*Hkv]
     float* part_ml;    // [S*Hkv][n_pmax][G][2]
     float* part_o;     // [S*Hkv][n_pmax][G][D]
     int32_t* err;
@@ -598,44 +596,71 @@ __device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
     __syncwarp();
 }
 
-// Final split-K merge of sequence s, KV head j (n_p partitions), by `nthreads`
-// threads (t = 0 .. nthreads-1): out = sum_i e^{m_i - M} o_i / sum_i e^{m_i - M} l_i.
-template <typename T, int D, int G>
-__device__ void merge_partials(const DecodeParams& p, size_t sj, int s, int j, int n_p, int t,
-                               int nthreads) {
-    const size_t base = sj * p.n_pmax;
-    for (int idx = t; idx < G * D; idx += nthreads) {
-        const int g = idx / D, dd = idx % D;
-        float M = -INFINITY;
-        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
-        float Lsum = 0.f, O = 0.f;
-        if (M != -INFINITY) {
-            int i = 0;
-            for (; i + 4 <= n_p; i += 4) {
-                float mm[4], ll[4], oo[4];
+// ------------------------------------------------------------ split-K merge kernel
+// Launched after either decode kernel when a sequence spans several
+// partitions.  One CTA per (sequence s, query head h): with the partials
+// (m_i, l_i, o_i) of partition i (log2 domain, o unnormalised),
+//   M = max_i m_i,  out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
+// The partitions are spread over MERGE_SLICES thread slices, each a row of
+// head_dim/4 threads that accumulates 16-byte columns of o, so each thread
+// has few dependent loads however long the sequence is.
+constexpr int MERGE_THREADS = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(MERGE_THREADS)
+merge_kernel(DecodeParams p) {
+    constexpr int NV = D / 4;                        // float4 columns of a row
+    constexpr int NS = MERGE_THREADS / NV;           // partition slices
+    __shared__ float4 acc_s[NS][NV];
+    __shared__ float l_s[NS], red[MERGE_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int s = blockIdx.x / p.Hq, h = blockIdx.x - s * p.Hq;
+    const int L = clamp_len(__ldg(p.lens + s), p);
+    const int n_p = n_parts(L, p.P);
+    if (n_p <= 1) return;                            // written directly by the decode kernel
+    const int G = p.Hq / p.Hkv, j = h / G, g = h - j * G;
+    const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
+    auto ml = [&](int i, int k) { return __ldcg(p.part_ml + ((base + i) * G + g) * 2 + k); };
+    // M = max_i m_i
+    float mx = -INFINITY;
+    for (int i = tid; i < n_p; i += MERGE_THREADS) mx = fmaxf(mx, ml(i, 0));
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const size_t pi = (base + i + k) * G + g;
-                    mm[k] = __ldcg(p.part_ml + pi * 2);
-                    ll[k] = __ldcg(p.part_ml + pi * 2 + 1);
-                    oo[k] = __ldcg(p.part_o + pi * D + dd);
-                }
+    for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    float M = red[0];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float f = exp2f(mm[k] - M);
-                    Lsum += ll[k] * f;
-                    O += oo[k] * f;
-                }
-            }
-            for (; i < n_p; ++i) {
-                const size_t pi = (base + i) * G + g;
-                const float f = exp2f(__ldcg(p.part_ml + pi * 2) - M);
-                Lsum += __ldcg(p.part_ml + pi * 2 + 1) * f;
-                O += __ldcg(p.part_o + pi * D + dd) * f;
-            }
+    for (int w = 1; w < MERGE_THREADS / 32; ++w) M = fmaxf(M, red[w]);
+    // weighted sums, slice by slice
+    const int col = tid % NV, slice = tid / NV;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+        for (int i = slice; i < n_p; i += NS) {
+            const float w = exp2f(ml(i, 0) - M);
+            lsum += w * ml(i, 1);
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((base + i) * G + g) * D) + col);
+            acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
         }
-        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + g) * D + dd;
-        *outp = DT<T>::from_float(Lsum > 0.f ? O / Lsum : 0.f);
+    }
+    acc_s[slice][col] = acc;
+    if (col == 0) l_s[slice] = lsum;
+    __syncthreads();
+    if (slice == 0) {
+        float Lsum = 0.f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < NS; ++k) {                // fixed order: deterministic
+            Lsum += l_s[k];
+            o.x += acc_s[k][col].x; o.y += acc_s[k][col].y; o.z += acc_s[k][col].z; o.w += acc_s[k][col].w;
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + h) * D + 4 * col;
+        outp[0] = DT<T>::from_float(o.x * inv);
+        outp[1] = DT<T>::from_float(o.y * inv);
+        outp[2] = DT<T>::from_float(o.z * inv);
+        outp[3] = DT<T>::from_float(o.w * inv);
     }
 }
 
@@ -677,7 +702,6 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
     int* lens_s = reinterpret_cast<int*>(smem + ly.lens());
     int* pre = reinterpret_cast<int*>(smem + ly.pre());
     volatile int* abort_flag = misc + 0;
-    volatile int* last_flag = misc + 1 + pipe;
     int* wsum = misc + 32;
     auto desc_at = [&](int k) { return reinterpret_cast<UnitDesc*>(smem + ly.unit(pipe, k)); };
     auto q_at = [&](int k) {
@@ -776,22 +800,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
                     }
                 }
             }
-            if (d.n_p > 1) __threadfence();                      // publish the partials ...
             named_bar_sync(bar_id, CT);                          // merge buffer free again
-            if (d.n_p > 1) {
-                if (ctid == 0) {
-                    const int prev = atomicAdd(p.counters + sj, 1);   // ... before the count
-                    const int last = (prev == d.n_p - 1);
-                    if (last) {
-                        p.counters[sj] = 0;            // every partition has arrived
-                        __threadfence();               // see the other CTAs' partials
-                    }
-                    *last_flag = last;
-                }
-                named_bar_sync(bar_id, CT);
-                if (*last_flag) merge_partials<T, D, G>(p, sj, d.s, d.j, d.n_p, ctid, CT);
-                named_bar_sync(bar_id, CT);                      // last_flag free again
-            }
             ++ucount;
         }
         __syncwarp();
@@ -829,10 +838,13 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
 // (exp2 units): only when a stage exceeds it is m moved (a barrier-OR vote
 // over the 128 threads), O^T rescaled in tensor memory and l rescaled.
 
-constexpr int TTOK = 64;            // tokens per stage (= M of the S^T MMA)
+constexpr int TTOK = 64;            // tokens per stage (a multiple of 16, at most SM_M)
+constexpr int SM_M = 64;            // M of the S^T MMA (rows past TTOK are masked)
 constexpr int NHP = 16;             // query heads padded to the MMA's N
 constexpr float kRescaleLog2 = 8.f;
 constexpr int TC_THREADS = 320;
+constexpr int kTailBuckets = 16;                              // last-partition size classes
+constexpr int kSchedScratch = (TC_THREADS / 32 + 1) * kTailBuckets;   // ints
 constexpr int BAR_SOFTMAX = 1, BAR_EPI = 2;   // named barriers (128 threads each)
 
 template <typename T, int D, int G>
@@ -845,13 +857,15 @@ struct TcLayout {
     static constexpr int BOXT = TTOK * 128;            // one column box of a stage: 8 KB
     static constexpr int KV_BYTES = NBOX * BOXT;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int NU = 2;                       // unit slots
-    static constexpr int QT = NBOX * 2 * 1024;         // Q tile: 16 rows x head_dim, 128B swizzle
+    static constexpr int NU = 3;                       // unit slots (descriptor + Q tile)
+    static constexpr int NQ = G <= 8 ? 8 : 16;         // N of the S^T MMA (query rows read)
+    static constexpr int QT = NBOX * (NQ / 8) * 1024;  // Q tile: NQ rows x head_dim, 128B swizzle
     static constexpr int PTB = TTOK * NHP * 2;         // one P^T tile (2 KB)
     static constexpr uint32_t TM_COLS = 64;            // S^T x2 then O^T x2, 16 columns each
-    static constexpr int NBAR = 2 * NU + 14;           // + 2 per stage slot
+    static constexpr int NBAR = 2 * NU + 13;           // + 2 per stage slot
     // epilogue slot: ints s, j, i, n_p, n_stages, O buffer, 2 pad; m[16]; l[4][16]
     static constexpr int ES = 32 + NHP * 4 + 4 * NHP * 4;
+    static_assert(4 * kSchedScratch <= 2 * ES, "schedule scratch fits the epilogue slots");
     int nst, S;
     __host__ __device__ TcLayout(int nst_, int S_) : nst(nst_), S(S_) {}
     __host__ __device__ size_t q(int k) const { return (size_t)k * QT; }
@@ -865,10 +879,98 @@ struct TcLayout {
     __host__ __device__ size_t red() const { return ((stage_ok() + (size_t)nst * 4 + 15) / 16) * 16; }
     __host__ __device__ size_t epi(int e) const { return red() + 4 * NHP * 4 + (size_t)e * ES; }
     __host__ __device__ size_t misc() const { return epi(2); }                  // 64 ints
+    // the schedule's scan scratch is used only before the first unit, so it
+    // shares the epilogue slots
+    __host__ __device__ size_t sched() const { return epi(0); }
     __host__ __device__ size_t lens() const { return misc() + 256; }
-    __host__ __device__ size_t pre() const { return lens() + 4 * (size_t)S; }
-    __host__ __device__ size_t total() const { return pre() + 4 * (size_t)(S + 1); }
+    __host__ __device__ size_t pref() const { return lens() + 4 * (size_t)S; }
+    __host__ __device__ size_t order() const { return pref() + 4 * (size_t)(S + 1); }
+    __host__ __device__ size_t total() const { return order() + 4 * (size_t)S; }
 };
+
+// Unit order of the tensor-core kernel, largest first (a longest-processing-
+// time order shortens the tail of the dynamic schedule): every full partition
+// (P tokens) of every sequence, then each sequence's last partition by its
+// stage count, most first (a stable counting sort over kTailBuckets classes;
+// zero-length sequences last).  All threads of the CTA; fills lens_s[S],
+// preF[S + 1] (exclusive prefix sums of the full partitions per sequence) and
+// order[S]; ends with __syncthreads.  Units: (preF[S] + S) * Hkv.
+template <int NTHREADS>
+__device__ void schedule_units(const DecodeParams& p, int* lens_s, int* preF, int* order, int* scr,
+                               int* wsum, int tid) {
+    constexpr int NW = NTHREADS / 32, NB = kTailBuckets;
+    static_assert((NW + 1) * NB <= kSchedScratch, "schedule scratch");
+    const int warp = tid >> 5, lane = tid & 31;
+    const int per = (p.S + NTHREADS - 1) / NTHREADS;
+    const int beg = min(p.S, tid * per), end = min(p.S, beg + per);
+    auto bucket = [&](int L) {          // 0 = the largest last partitions
+        const int n_p = n_parts(L, p.P);
+        const int ts = (L - (n_p - 1) * p.P + TTOK - 1) / TTOK;
+        return NB - 1 - min(NB - 1, ts);
+    };
+    int full = 0, cnt[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) cnt[b] = 0;
+    for (int k = beg; k < end; ++k) {
+        const int L = clamp_len(__ldg(p.lens + k), p);
+        lens_s[k] = L;
+        full += n_parts(L, p.P) - 1;
+        const int b = bucket(L);
+#pragma unroll
+        for (int q = 0; q < NB; ++q) cnt[q] += (q == b);
+    }
+    // block-wide exclusive scans: of `full` (-> preF) and of each bucket count
+    auto warp_incl = [&](int v) {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += u;
+        }
+        return v;
+    };
+    const int full_incl = warp_incl(full);
+    int cnt_excl[NB];                   // within the warp
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        const int inc = warp_incl(cnt[b]);
+        cnt_excl[b] = inc - cnt[b];
+        if (lane == 31) scr[warp * NB + b] = inc;
+    }
+    if (lane == 31) wsum[warp] = full_incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = (lane < NW) ? wsum[lane] : 0;
+        const int iv = warp_incl(v);
+        if (lane < NW) wsum[lane] = iv - v;          // exclusive warp offsets of `full`
+        int run = 0;                                  // bucket `lane`: offsets over warps
+        if (lane < NB) {
+            for (int w = 0; w < NW; ++w) {
+                const int c = scr[w * NB + lane];
+                scr[w * NB + lane] = run;
+                run += c;
+            }
+        }
+        const int tot_excl = warp_incl(run) - run;    // the whole warp scans (run = 0 past NB)
+        if (lane < NB) scr[NW * NB + lane] = tot_excl;    // where bucket `lane` starts in order[]
+    }
+    __syncthreads();
+    int runF = wsum[warp] + full_incl - full;
+    int pos[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) pos[b] = scr[NW * NB + b] + scr[warp * NB + b] + cnt_excl[b];
+    for (int k = beg; k < end; ++k) {
+        preF[k] = runF;
+        runF += n_parts(lens_s[k], p.P) - 1;
+        const int b = bucket(lens_s[k]);
+        int at = 0;
+#pragma unroll
+        for (int q = 0; q < NB; ++q)
+            if (q == b) at = pos[q]++;
+        order[at] = k;
+    }
+    if (tid == NTHREADS - 1) preF[p.S] = runF;
+    __syncthreads();
+}
 
 // Producer of the tensor-core engine: a 128-token stage is built from pieces of
 // 16 token rows (8 when bs = 8), each inside one block; one TMA box per
@@ -878,8 +980,9 @@ template <typename T, int D, int G>
 __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
                             const CUtensorMap* qmap, const DecodeParams& p, uint8_t* smem,
                             const TcLayout<T, D, G>& ly, uint64_t* full, uint64_t* empty,
-                            uint64_t* ufull, uint64_t* uempty, int* stage_ok, const int* pre,
-                            const int* lens_s, int U, volatile int* abort_flag, int lane) {
+                            uint64_t* ufull, uint64_t* uempty, int* stage_ok, const int* preF,
+                            const int* order, const int* lens_s, int U, volatile int* abort_flag,
+                            int lane) {
     using LY = TcLayout<T, D, G>;
     constexpr int NU = LY::NU;
     constexpr int BOX_ELEMS = 64;
@@ -899,30 +1002,45 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
         Plan q{};
         q.u = u;
         if (u >= U) return q;
-        const int x = u / p.Hkv;
-        int lo = 0, hi = p.S;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (pre[mid] <= x) lo = mid; else hi = mid;
+        // unit u -> (sequence, partition): full partitions first, in sequence
+        // order, then the last partitions in the largest-first order
+        const int x = u / p.Hkv, F = preF[p.S];
+        if (x < F) {
+            int lo = 0, hi = p.S;                      // last lo with preF[lo] <= x
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (preF[mid] <= x) lo = mid; else hi = mid;
+            }
+            q.s = lo;
+            q.i = x - preF[lo];
+        } else {
+            q.s = order[x - F];
+            q.i = n_parts(lens_s[q.s], p.P) - 1;
         }
-        q.s = lo;
-        q.i = x - pre[lo];
         q.j = u - x * p.Hkv;
-        const int L = lens_s[lo];
+        const int L = lens_s[q.s];
         q.t0 = min(q.i * p.P, L);
         q.t1 = min(q.t0 + p.P, L);
         q.nst = (q.t1 - q.t0 + TTOK - 1) / TTOK;
         q.n_p = n_parts(L, p.P);
         const int b0 = q.t0 >> bsl;
         q.nblk = ((q.t1 + bs - 1) >> bsl) - b0;
-        q.trow = p.tables + (size_t)lo * p.mbps + b0;
+        q.trow = p.tables + (size_t)q.s * p.mbps + b0;
         q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
         q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
         return q;
     };
-    int gstage = 0, st = 0, round = 0, ucount = 0, ticket = 0;
-    if (lane == 0) ticket = atomicAdd(&p.hdr->next_unit, 1);
-    Plan cur = prepare(__shfl_sync(FULL, ticket, 0));
+    // Latency hiding at unit boundaries: lane 0 holds the tickets of the two
+    // units after the current one (each fetched two units ahead), and the next
+    // unit's plan, whose block-table loads are then in flight, is prepared as
+    // soon as the current unit's first stage is issued.
+    int gstage = 0, st = 0, round = 0, ucount = 0, t0 = 0, t1 = 0, t2 = 0;
+    if (lane == 0) {
+        t0 = atomicAdd(&p.hdr->next_unit, 1);
+        t1 = atomicAdd(&p.hdr->next_unit, 1);
+        t2 = atomicAdd(&p.hdr->next_unit, 1);
+    }
+    Plan cur = prepare(__shfl_sync(FULL, t0, 0));
     bool ok = true;
     while (ok) {
         const int slot = ucount % NU;
@@ -948,13 +1066,20 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
             uint8_t* qt = smem + ly.q(slot);
 #pragma unroll
             for (int kc = 0; kc < LY::NBOX; ++kc)
-                tma_load_2d(qt + kc * 2048, qmap, kc * BOX_ELEMS, cur.s * p.Hq + cur.j * G,
+                tma_load_2d(qt + kc * (LY::QT / LY::NBOX), qmap, kc * BOX_ELEMS, cur.s * p.Hq + cur.j * G,
                             ufull + slot, policy);
-            ticket = atomicAdd(&p.hdr->next_unit, 1);
         }
         ++ucount;
         Plan nxt{};
         bool have_next = false;
+        auto next_plan = [&]() {            // after the unit's first stage is issued
+            nxt = prepare(__shfl_sync(FULL, t1, 0));
+            have_next = true;
+            if (lane == 0) {
+                t1 = t2;
+                t2 = atomicAdd(&p.hdr->next_unit, 1);
+            }
+        };
         int win = 0;
         const int b0 = cur.t0 >> bsl;
         for (int c = 0; c < cur.nst; ++c) {
@@ -1011,13 +1136,10 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
             }
             ++gstage;
             if (++st == nst) { st = 0; ++round; }
-            if (!have_next) {
-                nxt = prepare(__shfl_sync(FULL, ticket, 0));
-                have_next = true;
-            }
+            if (!have_next) next_plan();
         }
         if (!ok) break;
-        if (!have_next) nxt = prepare(__shfl_sync(FULL, ticket, 0));
+        if (!have_next) next_plan();
         cur = nxt;
     }
     if (lane == 0) {
@@ -1049,8 +1171,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     uint64_t* uempty = ufull + NU;        // 5 arrivals: MMA issuer + the 4 softmax warps
     uint64_t* s_full = uempty + NU;       // [2] S^T_g complete
     uint64_t* p_full = s_full + 2;        // [2] P^T_g written (4 softmax warps)
-    uint64_t* o_bar = p_full + 2;         // PV of stage g complete (phase g)
-    uint64_t* o_done = o_bar + 1;         // [2] last PV of a unit complete (per O buffer)
+    uint64_t* o_done = p_full + 2;        // [2] last PV of a unit complete (per O buffer)
     uint64_t* o_free = o_done + 2;        // [2] O buffer read by the epilogue (4 warps)
     uint64_t* epi_full = o_free + 2;      // [2] epilogue slot filled (4 softmax warps)
     uint64_t* epi_empty = epi_full + 2;   // [2] epilogue slot read (4 epilogue warps)
@@ -1059,9 +1180,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     float* red = reinterpret_cast<float*>(smem + ly.red());      // [4][16]
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
     int* lens_s = reinterpret_cast<int*>(smem + ly.lens());
-    int* pre = reinterpret_cast<int*>(smem + ly.pre());
+    int* preF = reinterpret_cast<int*>(smem + ly.pref());
+    int* order = reinterpret_cast<int*>(smem + ly.order());
     volatile int* abort_flag = misc + 0;
-    volatile int* last_flag = misc + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 60);   // outside the zeroed words
     int* wsum = misc + 32;
 
@@ -1087,20 +1208,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
-    prefix_sums<TC_THREADS>(p, lens_s, pre, wsum, tid);
+    schedule_units<TC_THREADS>(p, lens_s, preF, order, reinterpret_cast<int*>(smem + ly.sched()), wsum, tid);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 2 * NHP;                 // + 16 * buffer
     const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;          // this warp's lane quarter
-    const int U = pre[p.S] * p.Hkv;
+    const int U = (preF[p.S] + p.S) * p.Hkv;
     const int PR = p.bs >= 16 ? 16 : p.bs;
 
     if (warp == 8) {
         // ================================================= producer warp
         producer_tc<T, D, G>(&kmap, &vmap, &qmap, p, smem, ly, full, empty, ufull, uempty,
-                             stage_ok, pre, lens_s, U, abort_flag, lane);
+                             stage_ok, preF, order, lens_s, U, abort_flag, lane);
     } else if (warp == 9) {
         // ================================================= MMA issuer (one thread)
         // Event driven: the thread polls the next stage's data (-> S MMAs) and
@@ -1108,7 +1229,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         // ready, so a PV never waits for the next stage's copy.  S_g is issued
         // only once PV_{g-2} has been (its S^T and P^T buffers are reused).
         if (lane == 0) {
-            constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, TTOK, NHP);
+            constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, SM_M, LY::NQ);
             constexpr uint32_t ID_O = tc::idesc_f16<T>(true, true, D, NHP);
             struct Pending {
                 int g, nv, oseq;
@@ -1161,7 +1282,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                             tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
                                        (r.first && kk == 0) ? 0u : 1u);
                         tc::commit(empty + st);          // the stage slot may be refilled
-                        tc::commit(o_bar);
                         if (r.last) tc::commit(o_done + ob);
                         pend0 = pend1;
                         --npend;
@@ -1179,7 +1299,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
                             tc::mma_ss(sd, a0 + (uint64_t)((k >> 2) * (LY::BOXT >> 4) + (k & 3) * 2),
-                                       b0 + (uint64_t)((k >> 2) * 128 + (k & 3) * 2), ID_S, k > 0 ? 1u : 0u);
+                                       b0 + (uint64_t)((k >> 2) * (LY::QT / LY::NBOX >> 4) + (k & 3) * 2), ID_S,
+                                       k > 0 ? 1u : 0u);
                         tc::commit(s_full + (g & 1));
                         if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
                         const Pending nw{g, min(TTOK, d.t1 - (d.t0 + c * TTOK)), oseq, c == 0,
@@ -1216,7 +1337,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         __syncwarp();
     } else if (warp < 4) {
         // ================================================= softmax warps (thread = token)
-        const int t = lane < 16 ? 16 * warp + lane : -1;    // stage token of this thread (M = 64 layout)
+        const int t = (lane < 16 && 16 * warp + lane < TTOK) ? 16 * warp + lane : -1;   // stage token (M = 64 layout)
         const int piece = t >= 0 ? t / PR : 0;
         int ucount = 0, ocount = 0;
         while (true) {
@@ -1297,8 +1418,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                     }
                     named_bar_sync(BAR_SOFTMAX, 128);      // red[] free again
                     if (c > 0 && moved) {
-                        // O^T has stage g-1's PV in it and not yet stage g's
-                        const bool okw = wait_or_abort(o_bar, (g - 1) & 1, abort_flag, p.err);
+                        // O^T has stage g-1's PV in it (its completion is what
+                        // frees stage g-1's ring slot) and not yet stage g's
+                        const int sp = (g - 1) % nst;
+                        const bool okw = wait_or_abort(empty + sp, ((g - 1) / nst) & 1, abort_flag, p.err);
                         if (named_bar_or(BAR_SOFTMAX, 128, !okw)) {
                             ok = false;
                             break;
@@ -1417,31 +1540,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h) * D + dd;
                         *outp = DT<T>::from_float(lh[h] > 0.f ? o[h] / lh[h] : 0.f);
                     }
-            } else {
-                if (dd >= 0)
+            } else if (dd >= 0) {
+                // partials for the merge kernel
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const size_t pi = (sj * p.n_pmax + i) * G + h;
-                        p.part_o[pi * D + dd] = o[h];
-                        if (dd == 0) {
-                            p.part_ml[pi * 2 + 0] = mh[h];
-                            p.part_ml[pi * 2 + 1] = lh[h];
-                        }
+                for (int h = 0; h < G; ++h) {
+                    const size_t pi = (sj * p.n_pmax + i) * G + h;
+                    p.part_o[pi * D + dd] = o[h];
+                    if (dd == 0) {
+                        p.part_ml[pi * 2 + 0] = mh[h];
+                        p.part_ml[pi * 2 + 1] = lh[h];
                     }
-                __threadfence();                           // publish the partials ...
-                named_bar_sync(BAR_EPI, 128);
-                if (et == 0) {
-                    const int prev = atomicAdd(p.counters + sj, 1);   // ... before the count
-                    const int last = (prev == n_p - 1);
-                    if (last) {
-                        p.counters[sj] = 0;                // every partition has arrived
-                        __threadfence();                   // see the other CTAs' partials
-                    }
-                    *last_flag = last;
                 }
-                named_bar_sync(BAR_EPI, 128);
-                if (*last_flag) merge_partials<T, D, G>(p, sj, s, j, n_p, et, 128);
-                named_bar_sync(BAR_EPI, 128);              // last_flag free again
             }
             ++ucount;
         }
@@ -1535,7 +1644,6 @@ constexpr int kMinStages = 2;     // any count >= 1 is correct; fewer only slows
 
 size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
     size_t b = sizeof(WsHeader);
-    b += (((size_t)S * Hkv * 4 + 255) / 256) * 256;
     if (n_pmax > 1) {
         b += (((size_t)S * Hq * n_pmax * 2 * 4 + 255) / 256) * 256;
         b += (size_t)S * Hq * n_pmax * D * 4;
@@ -1645,6 +1753,23 @@ int dispatch_dim(Launch& L, const DevInfo& di, int D, int G, bool tensor) {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
 
+// The split-K merge, one CTA per (sequence, query head).
+int launch_merge(const Launch& L, pa_dtype dt, int D) {
+    const dim3 grid((unsigned)((int64_t)L.p.S * L.p.Hq));
+    const dim3 block(MERGE_THREADS);
+    if (dt == PA_F32) {
+        if (D == 64) merge_kernel<float, 64><<<grid, block, 0, L.stream>>>(L.p);
+        else merge_kernel<float, 128><<<grid, block, 0, L.stream>>>(L.p);
+    } else if (dt == PA_F16) {
+        if (D == 64) merge_kernel<__half, 64><<<grid, block, 0, L.stream>>>(L.p);
+        else merge_kernel<__half, 128><<<grid, block, 0, L.stream>>>(L.p);
+    } else {
+        if (D == 64) merge_kernel<__nv_bfloat16, 64><<<grid, block, 0, L.stream>>>(L.p);
+        else merge_kernel<__nv_bfloat16, 128><<<grid, block, 0, L.stream>>>(L.p);
+    }
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 }  // namespace
 
 }  // namespace pa
@@ -1740,9 +1865,7 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     p.scale_log2e = scale * 1.4426950408889634f;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.hdr = reinterpret_cast<WsHeader*>(ws);
-    p.counters = reinterpret_cast<int*>(ws + sizeof(WsHeader));
-    const size_t cnt_bytes = (((size_t)num_seqs * num_kv_heads * 4 + 255) / 256) * 256;
-    p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader) + cnt_bytes);
+    p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader));
     p.part_o = p.part_ml + ((((size_t)num_seqs * num_q_heads * n_pmax * 2 * 4 + 255) / 256) * 256) / 4;
     p.err = err_flag;
 
@@ -1756,11 +1879,11 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         std::lock_guard<std::mutex> lk(g_mu);
         engine = g_engine;
     }
-    // tcgen05 engine: 16-bit types only; by default where query groups make
-    // the CUDA-core dot products the limit (G > 1)
+    // tcgen05 engine: 16-bit types only (the default for them); fp32 runs on
+    // CUDA cores
     const bool sixteen = dtype != PA_F32;
     if (engine == PA_ENGINE_TENSOR && !sixteen) return PA_ERR_UNSUPPORTED;
-    const bool tensor = engine == PA_ENGINE_TENSOR || (engine == PA_ENGINE_AUTO && sixteen && G > 1);
+    const bool tensor = sixteen && engine != PA_ENGINE_CUDA_CORE;
     auto run = [&](bool use_tensor) {
         switch (dtype) {
             case PA_F32: return dispatch_dim<float>(L, di, head_dim, G, false);
@@ -1776,9 +1899,12 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         // by default, shapes whose stage ring does not fit (very many
         // sequences) go to the CUDA-core engine
         if (st == PA_ERR_UNSUPPORTED && engine == PA_ENGINE_AUTO) st = run(false);
-        return st;
+    } else {
+        st = run(false);
     }
-    return run(false);
+    // sequences split into several partitions are merged by a second launch
+    if (st == PA_OK && n_pmax > 1) st = launch_merge(L, dtype, head_dim);
+    return st;
 }
 
 }  // extern "C"
@@ -1827,10 +1953,9 @@ extern "C" int pa_decode_static(void* out, const void* query, const void* key_ca
         }
         ws = g_static_ptr[dev];
     }
-    // the scheduler words and partition counters must start at zero; a call
-    // that stopped early (PA_DEV_TIMEOUT) may have left them dirty
-    const size_t counters = sizeof(WsHeader) + (((size_t)num_seqs * num_kv_heads * 4 + 255) / 256) * 256;
-    if (cudaMemsetAsync(ws, 0, counters, (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+    // the scheduler words must start at zero; a call that stopped early
+    // (PA_DEV_TIMEOUT) may have left them dirty
+    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
     return pa_decode(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                      context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
                      head_dim, block_size, num_blocks, scale, partition_size, ws,

@@ -66,12 +66,13 @@ def test_bad_arguments_rejected_before_launch():
 
 
 def test_workspace_size_formula():
-    # scheduler header + counters only when nothing is split
+    # the scheduler header only when nothing is split
     n0 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 0)
-    assert n0 == 256 + 64 * 32 * 4
+    assert n0 == 256
+    # + (m, l) and the unnormalised output of every partition of every head
     n1 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 512)
     n_p = 5
-    assert n1 == 256 + 64 * 32 * 4 + 64 * 32 * n_p * 2 * 4 + 64 * 32 * n_p * 128 * 4
+    assert n1 == 256 + 64 * 32 * n_p * 2 * 4 + 64 * 32 * n_p * 128 * 4
 
 
 def test_allocator_errors():

@@ -184,7 +184,7 @@ def max_over_ranks(x, world):
 class Session:
     """One replica: caches, the C++ manager, and per-step device inputs."""
 
-    def __init__(self, w, P, dev):
+    def __init__(self, w, P, dev, engine="auto"):
         import paged_kv_cache_426_b200 as pa
         self.pa, self.w, self.P, self.dev = pa, w, P, dev
         dt = w.torch_dtype
@@ -269,7 +269,8 @@ class Session:
         self.pa.pa_decode(out, st["q"], self.kc, self.vc, st["tab"], st["lens"], self.max_len,
                           self.w.scale, partition_size=self.P, workspace=self.ws,
                           err_flag=self.err)
-        return 2 if 0 < self.P < self.max_len else 1
+        n_pmax = -(-self.max_len // self.P) if self.P > 0 else 1
+        return 2 if n_pmax > 1 else 1
 
     def bytes_of(self, lens):
         w = self.w
@@ -285,7 +286,7 @@ def run_ours(args, rank, world, local):
     P = w.partition_size if args.partition_size is None else args.partition_size
     import paged_kv_cache_426_b200 as pa
     pa.pa_set_decode_engine({"auto": 0, "core": 1, "tensor": 2}[args.engine])
-    sess = Session(w, P, dev)
+    sess = Session(w, P, dev, args.engine)
     _, mgr = sess.prefill()
     plan = sess.plan_steps(mgr, n_steps)
     out = torch.empty_like(plan[0]["q"])

@@ -98,7 +98,8 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * Long contexts are split into partitions of `partition_size` tokens
  * (a positive multiple of 16; 0 = one partition per sequence) whose partial
  * results are merged with their log-sum-exp weights by a second kernel that
- * pa_decode launches on the same stream (only when some sequence is split).
+ * pa_decode launches on the same stream when ceil(max_context_len /
+ * partition_size) > 1; otherwise one call is one launch.
  *   out           device [num_seqs][num_q_heads][head_dim] dtype
  *   query         device [num_seqs][num_q_heads][head_dim] dtype, 16-B aligned
  *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past

@@ -596,19 +596,66 @@ __device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
     __syncwarp();
 }
 
-// ------------------------------------------------------------ split-K merge kernel
-// Launched after either decode kernel when a sequence spans several
-// partitions.  One CTA per (sequence s, query head h): with the partials
-// (m_i, l_i, o_i) of partition i (log2 domain, o unnormalised),
+// ------------------------------------------------------------ split-K merge kernels
+// Launched after a decode kernel when a sequence may span several partitions.
+// With the partials (m_i, l_i, o_i) of partition i (log2 domain, o not yet
+// normalised), for each query head
 //   M = max_i m_i,  out = sum_i 2^(m_i - M) o_i / sum_i 2^(m_i - M) l_i.
-// The partitions are spread over MERGE_SLICES thread slices, each a row of
-// head_dim/4 threads that accumulates 16-byte columns of o, so each thread
-// has few dependent loads however long the sequence is.
+// Sequences with a single partition were written by the decode kernel and are
+// skipped.  Two shapes: short splits (few partitions) take one CTA per
+// (sequence, KV head) with a thread per 4 output columns of all G heads;
+// long splits take one CTA per (sequence, query head) with the partitions
+// spread over thread slices, so no thread walks a long chain of loads.
 constexpr int MERGE_THREADS = 256;
+constexpr int kShortSplit = 32;     // partitions up to which the group shape is used
 
 template <typename T, int D>
+__device__ __forceinline__ void merge_store(const DecodeParams& p, int s, int h, int col, float4 o, float inv) {
+    T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + h) * D + 4 * col;
+    outp[0] = DT<T>::from_float(o.x * inv);
+    outp[1] = DT<T>::from_float(o.y * inv);
+    outp[2] = DT<T>::from_float(o.z * inv);
+    outp[3] = DT<T>::from_float(o.w * inv);
+}
+
+// One CTA per (sequence, KV head): thread = (head g, 4 columns), a whole
+// group of G * D / 4 <= MERGE_THREADS columns; every thread walks the few
+// partitions itself (independent loads).
+template <typename T, int D>
 __global__ void __launch_bounds__(MERGE_THREADS)
-merge_kernel(DecodeParams p) {
+merge_group_kernel(DecodeParams p) {
+    constexpr int NV = D / 4;
+    const int s = blockIdx.x / p.Hkv, j = blockIdx.x - s * p.Hkv;
+    const int L = clamp_len(__ldg(p.lens + s), p);
+    const int n_p = n_parts(L, p.P);
+    if (n_p <= 1) return;                            // written by the decode kernel
+    const int G = p.Hq / p.Hkv;
+    const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
+    for (int c = threadIdx.x; c < G * NV; c += MERGE_THREADS) {
+        const int g = c / NV, col = c - g * NV;
+        float M = -INFINITY;
+        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float Lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int i = 0; i < n_p; ++i) {
+                const size_t pi = (base + i) * G + g;
+                const float w = exp2f(__ldcg(p.part_ml + pi * 2) - M);
+                Lsum += w * __ldcg(p.part_ml + pi * 2 + 1);
+                const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + pi * D) + col);
+                acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+            }
+        }
+        merge_store<T, D>(p, s, j * G + g, col, acc, Lsum > 0.f ? 1.f / Lsum : 0.f);
+    }
+}
+
+// One CTA per (sequence s, query head h); the partitions are spread over
+// MERGE_THREADS / (D/4) slices, reduced in shared memory in a fixed order.
+template <typename T, int D>
+__global__ void __launch_bounds__(MERGE_THREADS)
+merge_head_kernel(DecodeParams p) {
     constexpr int NV = D / 4;                        // float4 columns of a row
     constexpr int NS = MERGE_THREADS / NV;           // partition slices
     __shared__ float4 acc_s[NS][NV];
@@ -617,11 +664,10 @@ merge_kernel(DecodeParams p) {
     const int s = blockIdx.x / p.Hq, h = blockIdx.x - s * p.Hq;
     const int L = clamp_len(__ldg(p.lens + s), p);
     const int n_p = n_parts(L, p.P);
-    if (n_p <= 1) return;                            // written directly by the decode kernel
+    if (n_p <= 1) return;                            // written by the decode kernel
     const int G = p.Hq / p.Hkv, j = h / G, g = h - j * G;
     const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
     auto ml = [&](int i, int k) { return __ldcg(p.part_ml + ((base + i) * G + g) * 2 + k); };
-    // M = max_i m_i
     float mx = -INFINITY;
     for (int i = tid; i < n_p; i += MERGE_THREADS) mx = fmaxf(mx, ml(i, 0));
 #pragma unroll
@@ -631,7 +677,6 @@ merge_kernel(DecodeParams p) {
     float M = red[0];
 #pragma unroll
     for (int w = 1; w < MERGE_THREADS / 32; ++w) M = fmaxf(M, red[w]);
-    // weighted sums, slice by slice
     const int col = tid % NV, slice = tid / NV;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float lsum = 0.f;
@@ -655,12 +700,7 @@ merge_kernel(DecodeParams p) {
             Lsum += l_s[k];
             o.x += acc_s[k][col].x; o.y += acc_s[k][col].y; o.z += acc_s[k][col].z; o.w += acc_s[k][col].w;
         }
-        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + h) * D + 4 * col;
-        outp[0] = DT<T>::from_float(o.x * inv);
-        outp[1] = DT<T>::from_float(o.y * inv);
-        outp[2] = DT<T>::from_float(o.z * inv);
-        outp[3] = DT<T>::from_float(o.w * inv);
+        merge_store<T, D>(p, s, h, col, o, Lsum > 0.f ? 1.f / Lsum : 0.f);
     }
 }
 
@@ -1540,17 +1580,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h) * D + dd;
                         *outp = DT<T>::from_float(lh[h] > 0.f ? o[h] / lh[h] : 0.f);
                     }
-            } else if (dd >= 0) {
+            } else {
                 // partials for the merge kernel
+                if (dd >= 0)
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const size_t pi = (sj * p.n_pmax + i) * G + h;
-                    p.part_o[pi * D + dd] = o[h];
-                    if (dd == 0) {
-                        p.part_ml[pi * 2 + 0] = mh[h];
-                        p.part_ml[pi * 2 + 1] = lh[h];
+                    for (int h = 0; h < G; ++h) {
+                        const size_t pi = (sj * p.n_pmax + i) * G + h;
+                        p.part_o[pi * D + dd] = o[h];
+                        if (dd == 0) {
+                            p.part_ml[pi * 2 + 0] = mh[h];
+                            p.part_ml[pi * 2 + 1] = lh[h];
+                        }
                     }
-                }
             }
             ++ucount;
         }
@@ -1753,19 +1794,25 @@ int dispatch_dim(Launch& L, const DevInfo& di, int D, int G, bool tensor) {
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
 
-// The split-K merge, one CTA per (sequence, query head).
-int launch_merge(const Launch& L, pa_dtype dt, int D) {
-    const dim3 grid((unsigned)((int64_t)L.p.S * L.p.Hq));
+// The split-K merge: the group shape for short splits, the sliced per-head
+// shape for long ones.
+template <typename T, int D>
+void launch_merge_t(const Launch& L, bool group) {
     const dim3 block(MERGE_THREADS);
+    if (group)
+        merge_group_kernel<T, D><<<(unsigned)((int64_t)L.p.S * L.p.Hkv), block, 0, L.stream>>>(L.p);
+    else
+        merge_head_kernel<T, D><<<(unsigned)((int64_t)L.p.S * L.p.Hq), block, 0, L.stream>>>(L.p);
+}
+
+int launch_merge(const Launch& L, pa_dtype dt, int D, int G, int n_pmax) {
+    const bool group = n_pmax <= kShortSplit && G * D / 4 <= MERGE_THREADS;
     if (dt == PA_F32) {
-        if (D == 64) merge_kernel<float, 64><<<grid, block, 0, L.stream>>>(L.p);
-        else merge_kernel<float, 128><<<grid, block, 0, L.stream>>>(L.p);
+        if (D == 64) launch_merge_t<float, 64>(L, group); else launch_merge_t<float, 128>(L, group);
     } else if (dt == PA_F16) {
-        if (D == 64) merge_kernel<__half, 64><<<grid, block, 0, L.stream>>>(L.p);
-        else merge_kernel<__half, 128><<<grid, block, 0, L.stream>>>(L.p);
+        if (D == 64) launch_merge_t<__half, 64>(L, group); else launch_merge_t<__half, 128>(L, group);
     } else {
-        if (D == 64) merge_kernel<__nv_bfloat16, 64><<<grid, block, 0, L.stream>>>(L.p);
-        else merge_kernel<__nv_bfloat16, 128><<<grid, block, 0, L.stream>>>(L.p);
+        if (D == 64) launch_merge_t<__nv_bfloat16, 64>(L, group); else launch_merge_t<__nv_bfloat16, 128>(L, group);
     }
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -1903,7 +1950,7 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         st = run(false);
     }
     // sequences split into several partitions are merged by a second launch
-    if (st == PA_OK && n_pmax > 1) st = launch_merge(L, dtype, head_dim);
+    if (st == PA_OK && n_pmax > 1) st = launch_merge(L, dtype, head_dim, G, n_pmax);
     return st;
 }
 

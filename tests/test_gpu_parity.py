@@ -92,6 +92,15 @@ def test_shapes_and_groups(engine, dtype, d, G):
     run_full_compare(w)
 
 
+@pytest.mark.parametrize("L", [511, 512, 513, 1000])
+def test_split_merge_boundary(engine, L):
+    """32 partitions of 16 tokens are merged inside the tensor-core decode
+    kernel, 33 or more by the separate merge kernel: both sides of the
+    boundary, with a short sequence in the same batch."""
+    w = workloads.custom("bf16", [L, 40], 16, 4, 128, 16, seed=L, partition_size=16)
+    run_full_compare(w)
+
+
 @pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
 def test_block_sizes(engine, bs):
     w = workloads.custom("f16", [3, 8, 9, 129, 300], 8, 2, 128, bs, seed=bs, partition_size=128)

@@ -225,6 +225,19 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start before the previous kernel in the stream ends;
+// grid_dependency_wait blocks until that kernel has completed and its memory
+// writes are visible.  launch_dependents lets the next such kernel be
+// scheduled.  Both are no-ops without a dependent/prerequisite launch.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // 1-D bulk copy global -> shared, completion counted on `bar` (bytes).
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,

@@ -625,6 +625,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_group_kernel(DecodeParams p) {
     constexpr int NV = D / 4;
+    grid_dependency_wait();                          // the decode grid's partials are complete
     const int s = blockIdx.x / p.Hkv, j = blockIdx.x - s * p.Hkv;
     const int L = clamp_len(__ldg(p.lens + s), p);
     const int n_p = n_parts(L, p.P);
@@ -660,6 +661,7 @@ merge_head_kernel(DecodeParams p) {
     constexpr int NS = MERGE_THREADS / NV;           // partition slices
     __shared__ float4 acc_s[NS][NV];
     __shared__ float l_s[NS], red[MERGE_THREADS / 32];
+    grid_dependency_wait();                          // the decode grid's partials are complete
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int s = blockIdx.x / p.Hq, h = blockIdx.x - s * p.Hq;
     const int L = clamp_len(__ldg(p.lens + s), p);
@@ -847,6 +849,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
     }
 
     __syncthreads();
+    launch_dependents();                 // the merge kernel may be scheduled
     if (tid == 0) {
         __threadfence();
         const int done = atomicAdd(&p.hdr->done_ctas, 1);
@@ -1600,6 +1603,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 
     tc::fence_before();
     __syncthreads();
+    launch_dependents();                 // the merge kernel may be scheduled
     if (warp == 0) {
         tc::fence_after();
         tc::dealloc(tmem, LY::TM_COLS);
@@ -1796,25 +1800,30 @@ bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15)
 
 // The split-K merge: the group shape for short splits, the sliced per-head
 // shape for long ones.
+// Launched as a programmatic dependent of the decode kernel: its CTAs may be
+// scheduled while the decode grid drains and wait on the device for it.
 template <typename T, int D>
-void launch_merge_t(const Launch& L, bool group) {
-    const dim3 block(MERGE_THREADS);
-    if (group)
-        merge_group_kernel<T, D><<<(unsigned)((int64_t)L.p.S * L.p.Hkv), block, 0, L.stream>>>(L.p);
-    else
-        merge_head_kernel<T, D><<<(unsigned)((int64_t)L.p.S * L.p.Hq), block, 0, L.stream>>>(L.p);
+int launch_merge_t(const Launch& L, bool group) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)L.p.S * (group ? L.p.Hkv : L.p.Hq)));
+    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = L.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = group ? cudaLaunchKernelEx(&cfg, merge_group_kernel<T, D>, L.p)
+                                : cudaLaunchKernelEx(&cfg, merge_head_kernel<T, D>, L.p);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int launch_merge(const Launch& L, pa_dtype dt, int D, int G, int n_pmax) {
     const bool group = n_pmax <= kShortSplit && G * D / 4 <= MERGE_THREADS;
-    if (dt == PA_F32) {
-        if (D == 64) launch_merge_t<float, 64>(L, group); else launch_merge_t<float, 128>(L, group);
-    } else if (dt == PA_F16) {
-        if (D == 64) launch_merge_t<__half, 64>(L, group); else launch_merge_t<__half, 128>(L, group);
-    } else {
-        if (D == 64) launch_merge_t<__nv_bfloat16, 64>(L, group); else launch_merge_t<__nv_bfloat16, 128>(L, group);
-    }
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    if (dt == PA_F32) return D == 64 ? launch_merge_t<float, 64>(L, group) : launch_merge_t<float, 128>(L, group);
+    if (dt == PA_F16) return D == 64 ? launch_merge_t<__half, 64>(L, group) : launch_merge_t<__half, 128>(L, group);
+    return D == 64 ? launch_merge_t<__nv_bfloat16, 64>(L, group) : launch_merge_t<__nv_bfloat16, 128>(L, group);
 }
 
 }  // namespace

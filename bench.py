@@ -522,6 +522,52 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_sweep(args):
+    """Block-size and indirection study with the same decode path: the GQA
+    batch's lengths and shapes at block sizes 8..128, with physical ids
+    shuffled or in allocation order (each sequence's blocks consecutive), and
+    batch-1 decodes of growing length.  Decode-only device time over
+    ``args.steps`` steps; one JSON line per point."""
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    import paged_kv_cache_426_b200 as pa
+    pa.pa_set_decode_engine({"auto": 0, "core": 1, "tensor": 2}[args.engine])
+    n = args.warmup + args.steps
+    gqa_lens = workloads.make("gqa8b_bf16_bs16", steps=1).meta["lens"]
+    points = [("block_size", bs, layout, gqa_lens) for bs in (8, 16, 32, 64, 128)
+              for layout in ("shuffled", "consecutive")]
+    points += [("batch1", 16, layout, [L]) for L in (512, 4096, 32768, 131072)
+               for layout in ("shuffled", "consecutive")]
+    for kind, bs, layout, lens in points:
+        w = workloads.custom("bf16", lens, 32, 8, 128, bs, seed=426 + bs, steps=n,
+                             partition_size=1024, shuffle=(layout == "shuffled"))
+        sess = Session(w, w.partition_size, dev, args.engine)
+        _, mgr = sess.prefill()
+        plan = sess.plan_steps(mgr, n)
+        out = torch.empty_like(plan[0]["q"])
+        for k in range(args.warmup):
+            sess.run_step(plan[k], out)
+            sess.decode(plan[k], out)
+        torch.cuda.synchronize()
+        total_ms, total_bytes = 0.0, 0
+        for k in range(args.warmup, n):
+            sess.run_step(plan[k], out)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            sess.decode(plan[k], out)
+            b.record()
+            torch.cuda.synchronize()
+            total_ms += a.elapsed_time(b)
+            total_bytes += sess.bytes_of(plan[k]["lens_host"])
+        print(json.dumps({"sweep": kind, "block_size": bs, "layout": layout,
+                          "num_seqs": len(lens), "max_len": max(lens), "steps": args.steps,
+                          "gbs": round(total_bytes / total_ms / 1e6, 1),
+                          "ms_per_step": round(total_ms / args.steps, 4),
+                          "err": int(sess.err.item())}), flush=True)
+        del sess, plan, out
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -535,11 +581,16 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--sweep", action="store_true",
+                    help="block-size / indirection study instead of the benchmark line")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     rank, world, local = (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
                           int(os.environ.get("LOCAL_RANK", "0")))
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:

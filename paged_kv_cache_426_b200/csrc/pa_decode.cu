@@ -618,9 +618,9 @@ __device__ __forceinline__ void merge_store(const DecodeParams& p, int s, int h,
     outp[3] = DT<T>::from_float(o.w * inv);
 }
 
-// One CTA per (sequence, KV head): thread = (head g, 4 columns), a whole
-// group of G * D / 4 <= MERGE_THREADS columns; every thread walks the few
-// partitions itself (independent loads).
+// One CTA of G * D / 4 <= MERGE_THREADS threads per (sequence, KV head):
+// thread = (head g, 4 columns); every thread walks the few partitions itself
+// (independent loads).  Small CTAs keep the whole grid resident at once.
 template <typename T, int D>
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_group_kernel(DecodeParams p) {
@@ -632,7 +632,7 @@ merge_group_kernel(DecodeParams p) {
     if (n_p <= 1) return;                            // written by the decode kernel
     const int G = p.Hq / p.Hkv;
     const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
-    for (int c = threadIdx.x; c < G * NV; c += MERGE_THREADS) {
+    for (int c = threadIdx.x; c < G * NV; c += blockDim.x) {
         const int g = c / NV, col = c - g * NV;
         float M = -INFINITY;
         for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
@@ -1806,7 +1806,7 @@ template <typename T, int D>
 int launch_merge_t(const Launch& L, bool group) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((int64_t)L.p.S * (group ? L.p.Hkv : L.p.Hq)));
-    cfg.blockDim = dim3(MERGE_THREADS);
+    cfg.blockDim = dim3(group ? (unsigned)std::max(32, (L.p.Hq / L.p.Hkv) * D / 4) : MERGE_THREADS);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = L.stream;
     cudaLaunchAttribute attr[1];

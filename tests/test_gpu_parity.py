@@ -94,9 +94,9 @@ def test_shapes_and_groups(engine, dtype, d, G):
 
 @pytest.mark.parametrize("L", [511, 512, 513, 1000])
 def test_split_merge_boundary(engine, L):
-    """32 partitions of 16 tokens are merged inside the tensor-core decode
-    kernel, 33 or more by the separate merge kernel: both sides of the
-    boundary, with a short sequence in the same batch."""
+    """Up to 32 partitions the merge kernel takes one CTA per (sequence, KV
+    head), from 33 one CTA per (sequence, query head) with sliced partitions:
+    both sides of the boundary, with a short sequence in the same batch."""
     w = workloads.custom("bf16", [L, 40], 16, 4, 128, 16, seed=L, partition_size=16)
     run_full_compare(w)
 

@@ -164,7 +164,9 @@ def mha7b_f16(steps: int = 32, num_seqs: int = 64) -> Workload:
     """7B-shaped MHA layer, fp16: 64 sequences, 32 = 32 heads, head dim 128,
     block 16, context lengths uniform on [128, 2048], K/V ~ 0.5*N(0,1),
     q ~ N(0,1), pool = total blocks the run needs + 10%, shuffled ids,
-    ``steps`` consecutive decode steps with cache writes."""
+    ``steps`` consecutive decode steps with cache writes.  The batch fixes no
+    split-K partition; 1024 tokens balances the decode's dynamic schedule
+    against merge work on one B200 (512 and 2048 are both slower)."""
     g = _gen(BASE_SEED + 2)
     lens = _uniform_int(g, 128, 2048, num_seqs)
 
@@ -172,7 +174,7 @@ def mha7b_f16(steps: int = 32, num_seqs: int = 64) -> Workload:
         nb = math.ceil(1.1 * needed)
         return nb, _perm(g, nb)
     return _decode_batch("mha7b_f16", "f16", BASE_SEED + 2 + 1000, lens,
-                         32, 32, 128, 16, steps, 0.5, pool, 512,
+                         32, 32, 128, 16, steps, 0.5, pool, 1024,
                          dict(recipe="L~U{128..2048}; K,V~0.5N(0,1); q~N(0,1); "
                                      "pool=ceil(1.1*needed), shuffled ids"))
 
@@ -191,7 +193,9 @@ def gqa8b_bf16(block_size: int = 16, steps: int = 1, num_seqs: int = 256,
     [16, 8192], q/K/V ~ N(0,1).  Fragmented pool: the pool is sized so that
     exactly 40% of it is free; those 40% are a random subset handed out in a
     random order, the other 60% stay held.  The same seed gives the same
-    lengths and values for both block sizes; only the pool differs."""
+    lengths and values for both block sizes; only the pool differs.  The batch
+    fixes no split-K partition; 1024 tokens balances the decode's dynamic
+    schedule against merge work on one B200 (512 and 2048 are both slower)."""
     g = _gen(BASE_SEED + 3)
     lens = _lognormal_lens(g, num_seqs, 512, sigma, 16, 8192)
 
@@ -202,7 +206,7 @@ def gqa8b_bf16(block_size: int = 16, steps: int = 1, num_seqs: int = 256,
         order = _perm(gp, nb)[:n_free]
         return nb, order
     return _decode_batch(f"gqa8b_bf16_bs{block_size}", "bf16", BASE_SEED + 3 + 1000,
-                         lens, 32, 8, 128, block_size, steps, 1.0, pool, 512,
+                         lens, 32, 8, 128, block_size, steps, 1.0, pool, 1024,
                          dict(recipe=f"L=clip(round(exp(ln512+{sigma}N(0,1))),16,8192); "
                                      "q,K,V~N(0,1); 40% of pool free, random subset "
                                      "in random order", sigma=sigma))

@@ -170,13 +170,32 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def _over_ranks(x, world, op):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x, world):
+    import torch.distributed as dist
+    return _over_ranks(x, world, dist.ReduceOp.MAX if world > 1 else None)
+
+
+def sum_over_ranks(x, world):
+    import torch.distributed as dist
+    return _over_ranks(x, world, dist.ReduceOp.SUM if world > 1 else None)
+
+
+def aggregate(rank_bytes, rank_span_ms, world):
+    """Whole-job throughput of `world` replicas: the bytes every rank moved
+    over the slowest rank's device time.  Returns (bytes, span_ms, GB/s)."""
+    span_ms = max_over_ranks(rank_span_ms, world)
+    total = sum_over_ranks(rank_bytes, world)
+    return total, span_ms, total / (span_ms * 1e-3) / 1e9
 
 
 # ----------------------------------------------------------------------------- our path
@@ -324,10 +343,8 @@ def run_ours(args, rank, world, local):
     assert int(sess.err.item()) == 0, f"device error flag {int(sess.err.item())}"
     span_ms = ev[0][0].elapsed_time(ev[-1][2])
     dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    span_ms = max_over_ranks(span_ms, world)
     step_bytes = [sess.bytes_of(plan[args.warmup + i]["lens_host"]) for i in range(args.steps)]
-    total_bytes = sum(step_bytes) * world
-    value = total_bytes / (span_ms * 1e-3) / 1e9
+    total_bytes, span_ms, value = aggregate(sum(step_bytes), span_ms, world)
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
     dec_gbs = (sum(step_bytes) / len(step_bytes)) / (dec_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
@@ -454,8 +471,9 @@ def run_e2e(sess, w, args, world):
         d2h = pin["out"].numel() * pin["out"].element_size()
     used_graphs = bool(graphs)
     graphs.clear()
-    span = max_over_ranks(sum(times), world)
-    return {"value": round(total_bytes * world / span / 1e9, 1), "unit": "GB/s",
+    total_bytes, span_ms, gbs = aggregate(total_bytes, sum(times) * 1e3, world)
+    span = span_ms * 1e-3
+    return {"value": round(gbs, 1), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(span / args.steps * 1e3, 4),
             "device_part": "cuda graph" if used_graphs else "eager"}

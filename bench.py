@@ -540,6 +540,77 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+def waste_report(name, lens, block_sizes, max_len, script=None):
+    """Memory held per stored token for one batch: paged blocks vs a contiguous
+    reservation of ``max_len`` slots per sequence.  The paged figure comes from
+    the library's own allocator and manager (blocks they actually hand out);
+    ``script`` (a workload's ops) replays adds, forks and writes so that shared
+    blocks are counted once.  Host only: no GPU is touched."""
+    import paged_kv_cache_426_b200 as pa
+    rows = []
+    tokens = int(sum(lens))
+    for bs in block_sizes:
+        need = sum(-(-L // bs) for L in lens) + len(lens)
+        alloc = pa.BlockAllocator(need)
+        mgr = pa.BlockManager(alloc, bs)
+        for s, L in enumerate(lens):
+            mgr.add_seq(s)
+            if L:
+                mgr.append(s, int(L))
+        blocks = alloc.num_blocks - alloc.num_free()
+        slots = blocks * bs
+        rows.append({"waste": name, "block_size": bs, "num_seqs": len(lens), "tokens": tokens,
+                     "paged_blocks": blocks, "paged_slots": slots,
+                     "paged_waste": round(1 - tokens / slots, 4),
+                     "contiguous_max_len": max_len, "contiguous_slots": len(lens) * max_len,
+                     "contiguous_waste": round(1 - tokens / (len(lens) * max_len), 4)})
+    return rows
+
+
+def sharing_report(w):
+    """Blocks held by a forked/shared-prefix script vs the same sequences with
+    every prefix stored once per sequence (the library's manager both times)."""
+    import paged_kv_cache_426_b200 as pa
+
+    def held(dup):
+        alloc = pa.BlockAllocator(1 << 18)           # host-only pool, ample for either layout
+        mgr = pa.BlockManager(alloc, w.block_size)
+        lengths = {}
+        for op in w.ops:
+            if op[0] == "add":
+                mgr.add_seq(op[1]); lengths[op[1]] = 0
+            elif op[0] == "fork":
+                if dup:             # a private copy of everything the parent holds
+                    mgr.add_seq(op[2])
+                    if lengths[op[1]]:
+                        mgr.append(op[2], lengths[op[1]])
+                else:
+                    mgr.fork(op[1], op[2])
+                lengths[op[2]] = lengths[op[1]]
+            elif op[0] == "write":
+                n = w.kv["k" + op[2]].shape[0]
+                mgr.append(op[1], n); lengths[op[1]] += n
+            elif op[0] == "step":
+                break
+        return alloc.num_blocks - alloc.num_free(), sum(lengths.values())
+    shared, toks = held(False)
+    dup, _ = held(True)
+    return {"sharing": w.name, "block_size": w.block_size, "logical_tokens": toks,
+            "blocks_shared": shared, "blocks_duplicated": dup,
+            "memory_saved": round(1 - shared / dup, 4)}
+
+
+def run_waste(args):
+    """Host-only memory accounting of the decode batches (one JSON line each)."""
+    batches = [("gqa8b_bf16", workloads.make("gqa8b_bf16_bs16", steps=1), 8192),
+               ("mha7b_f16", workloads.make("mha7b_f16", steps=1), 2048),
+               ("long_bf16", workloads.make("long_bf16", steps=1), 131072)]
+    for name, w, max_len in batches:
+        for row in waste_report(name, w.meta["lens"], (8, 16, 32, 64, 128), max_len):
+            print(json.dumps(row), flush=True)
+    print(json.dumps(sharing_report(workloads.make("prefix_f16", steps=1))), flush=True)
+
+
 def run_sweep(args):
     """Block-size and indirection study with the same decode path: the GQA
     batch's lengths and shapes at block sizes 8..128, with physical ids
@@ -601,6 +672,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--sweep", action="store_true",
                     help="block-size / indirection study instead of the benchmark line")
+    ap.add_argument("--waste", action="store_true",
+                    help="host-only memory accounting: paged vs contiguous reservation")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -608,6 +681,9 @@ def main():
                           int(os.environ.get("LOCAL_RANK", "0")))
     if args.sweep:
         run_sweep(args)
+        return
+    if args.waste:
+        run_waste(args)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)

@@ -232,6 +232,38 @@ int pa_manager_block_tables(const pa_manager* m, const int64_t* seq_ids,
                             int num_seqs, int32_t* block_tables, int max_blocks,
                             int32_t* context_lens);
 
+/* --------------------------------------------------------------------------
+ * Prefix caching - [VLLM] prefix caching, [119] 다음 장: a prompt that starts
+ * with the same tokens as an earlier one maps the same physical blocks
+ * (reference counted) instead of storing them again.
+ *   pa_manager_enable_prefix_cache  switch the cache on; PA_ERR_STATE once
+ *                    the manager holds sequences.
+ *   pa_manager_add_seq_prompt  new sequence whose first num_tokens tokens
+ *                    have ids tokens[0..n).  Its leading full blocks are
+ *                    looked up block by block (a block matches when the whole
+ *                    token prefix up to its end matches: a 64-bit fingerprint
+ *                    chained over the blocks, plus an exact comparison of the
+ *                    block's own ids) until the first miss; hits are shared
+ *                    (incref).  The remaining tokens are appended as usual and
+ *                    every full block they fill is cached.  slots[n]: -1 for
+ *                    the *num_cached leading tokens served from the cache
+ *                    (pa_reshape_and_cache skips them), the slot otherwise; so
+ *                    the caller writes K/V through the same array.  A cached
+ *                    block must hold its K/V before any sequence that hit it
+ *                    is decoded (write this call's slots first).  PA_ERR_OOM
+ *                    undoes the call except for evictions it made.
+ *   pa_manager_prefix_cache_stats  stats int64 [4]: cached blocks, block
+ *                    hits, block misses, evictions (cumulative).
+ * The cache keeps one reference per cached block, so a cached block outlives
+ * the sequences that used it.  When the free pool is empty, the least recently
+ * used cached block that nothing else references is evicted (freed) first.
+ * Appends of generated tokens (pa_manager_append*) are not cached.
+ */
+int pa_manager_enable_prefix_cache(pa_manager* m);
+int pa_manager_add_seq_prompt(pa_manager* m, int64_t seq_id, const int32_t* tokens,
+                              int num_tokens, int64_t* slots, int* num_cached);
+int pa_manager_prefix_cache_stats(const pa_manager* m, int64_t* stats);
+
 #ifdef __cplusplus
 }
 #endif

@@ -96,6 +96,86 @@ class BlockManager:
         self.bs = block_size
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        # prefix cache (off unless enabled): whole token prefix -> block
+        self.cache = None
+        self.cache_of: dict[int, tuple] = {}
+        self.lru: list[int] = []            # cached blocks, least recently used first
+        self.cache_stats = dict(hits=0, misses=0, evictions=0)
+
+    # ---------------------------------------------------------------- prefix caching
+    # "vLLM PagedAttention" studynote (prefix caching) and "09. PagedAttention"
+    # (119-ai-studio, 다음 장): full blocks of a prompt are reused by a later
+    # prompt with the same leading tokens.  Keys here are the exact token
+    # tuples of the whole prefix up to each block's end.  Reading of what the
+    # pages leave open (the plainest one): the cache keeps one reference per
+    # cached block; only full prompt blocks are cached, one block per prefix;
+    # lookup walks the leading full blocks until the first miss; when the free
+    # pool is empty the least recently used cached block that nothing else
+    # references is freed first.
+    def enable_prefix_cache(self) -> None:
+        if self.tables:
+            raise BlockStateError("enable the cache before adding sequences")
+        self.cache = {}
+
+    def _uncache(self, b: int) -> None:
+        del self.cache[self.cache_of.pop(b)]
+        self.lru.remove(b)
+        self.alloc.free_block(b)
+
+    def _new_block(self) -> int:
+        if self.alloc.num_free() == 0 and self.cache is not None:
+            for b in list(self.lru):
+                if self.alloc.refcount[b] == 1:
+                    self._uncache(b)
+                    self.cache_stats["evictions"] += 1
+                    break
+        return self.alloc.allocate_block()
+
+    def add_seq_prompt(self, seq: int, tokens):
+        """New sequence holding the prompt ``tokens``.  Returns (slots, cached)
+        with slot -1 for the ``cached`` leading tokens served from the cache."""
+        if self.cache is None:
+            raise BlockStateError("prefix cache not enabled")
+        tokens = [int(t) for t in tokens]
+        bs, n = self.bs, len(tokens)
+        self.add_seq(seq)
+        table = self.tables[seq]
+        hit, full = 0, n // bs
+        while hit < full:
+            b = self.cache.get(tuple(tokens[:(hit + 1) * bs]))
+            if b is None:
+                break
+            self.alloc.incref(b)
+            self.lru.remove(b)
+            self.lru.append(b)
+            table.append(b)
+            hit += 1
+        self.lens[seq] = hit * bs
+        registered = []
+        try:
+            for i in range(hit * bs, n):
+                if i % bs == 0:
+                    table.append(self._new_block())
+                self.lens[seq] = i + 1
+                key = tuple(tokens[:i + 1])
+                if (i + 1) % bs == 0 and key not in self.cache:
+                    b = table[-1]
+                    self.cache[key] = b
+                    self.cache_of[b] = key
+                    self.lru.append(b)
+                    self.alloc.incref(b)
+                    registered.append(b)
+        except OutOfBlocks:
+            for b in registered:
+                self._uncache(b)
+            for b in table:
+                self.alloc.free_block(b)
+            del self.tables[seq], self.lens[seq]
+            raise
+        self.cache_stats["hits"] += hit
+        self.cache_stats["misses"] += full - hit
+        slots = [-1] * (hit * bs) + [table[i // bs] * bs + i % bs for i in range(hit * bs, n)]
+        return slots, hit * bs
 
     def add_seq(self, seq: int) -> None:
         if seq in self.tables:
@@ -109,11 +189,11 @@ class BlockManager:
         p = self.lens[seq]
         cow = None
         if p % self.bs == 0:
-            table.append(self.alloc.allocate_block())
+            table.append(self._new_block())
         else:
             last = table[-1]
             if self.alloc.refcount[last] > 1:
-                new = self.alloc.allocate_block()
+                new = self._new_block()
                 self.alloc.free_block(last)
                 table[-1] = new
                 cow = (last, new)

@@ -63,6 +63,9 @@ SIGNATURES = {
     "pa_manager_append_step": ([_vp, _pi64, _i, _pi64, _pi64, C.POINTER(_i)], _i),
     "pa_manager_seq_len": ([_vp, _i64, _pi32], _i),
     "pa_manager_block_tables": ([_vp, _pi64, _i, _pi32, _i, _pi32], _i),
+    "pa_manager_enable_prefix_cache": ([_vp], _i),
+    "pa_manager_add_seq_prompt": ([_vp, _i64, _pi32, _i, _pi64, C.POINTER(_i)], _i),
+    "pa_manager_prefix_cache_stats": ([_vp, _pi64], _i),
 }
 for _name, (_args, _ret) in SIGNATURES.items():
     _fn = getattr(lib, _name)
@@ -285,3 +288,25 @@ class BlockManager:
                                           C.cast(tab.data_ptr(), _pi32), max_blocks,
                                           C.cast(lens.data_ptr(), _pi32)), "block_tables")
         return tab, lens
+
+    # ---- prefix caching
+    def enable_prefix_cache(self) -> None:
+        check(lib.pa_manager_enable_prefix_cache(self._h), "enable_prefix_cache")
+
+    def add_seq_prompt(self, seq: int, tokens):
+        """New sequence holding the prompt `tokens` (ids).  Returns (slots int64
+        [n], -1 for the leading tokens served from the cache; num_cached)."""
+        ids = torch.as_tensor(list(tokens) if not torch.is_tensor(tokens) else tokens,
+                              dtype=torch.int32).contiguous()
+        n = ids.numel()
+        slots = torch.empty(max(n, 1), dtype=torch.int64)
+        k = C.c_int(0)
+        check(lib.pa_manager_add_seq_prompt(self._h, seq, C.cast(ids.data_ptr(), _pi32), n,
+                                            C.cast(slots.data_ptr(), _pi64), C.byref(k)),
+              "add_seq_prompt")
+        return slots[:n], k.value
+
+    def prefix_cache_stats(self) -> dict:
+        st = (C.c_int64 * 4)()
+        check(lib.pa_manager_prefix_cache_stats(self._h, st), "prefix_cache_stats")
+        return dict(cached_blocks=st[0], hits=st[1], misses=st[2], evictions=st[3])

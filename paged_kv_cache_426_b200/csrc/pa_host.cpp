@@ -10,9 +10,21 @@
 // block table maps logical to physical blocks; only the last block may be
 // partly filled.
 //
+// Prefix caching ("vLLM PagedAttention" studynote, prefix caching; "09.
+// PagedAttention" (119-ai-studio), 다음 장): the full blocks of a prompt are
+// registered under a key that identifies the whole token prefix up to the
+// block's end; a later prompt that starts with the same tokens maps the same
+// physical blocks instead of storing them again.  The cache holds one
+// reference per cached block, so a cached block outlives the sequences that
+// used it, and is evicted (least recently used first, and only while nothing
+// else references it) when the free pool runs dry.
+//
 // Pure host code: nothing here touches device memory.
+#include <algorithm>
 #include <cstdint>
 #include <deque>
+#include <iterator>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -29,9 +41,21 @@ struct pa_manager {
         std::vector<int32_t> table;    // logical block -> physical block
         int32_t len = 0;               // tokens held
     };
+    // One cached block: the key of its whole prefix, the key of the prefix
+    // before it (0 for a first block) and its own tokens (checked on a hit).
+    struct Cached {
+        uint64_t key, parent;
+        std::vector<int32_t> tokens;
+        std::list<int32_t>::iterator lru;   // position in `lru`
+    };
     pa_allocator* alloc = nullptr;
     int block_size = 0;
     std::unordered_map<int64_t, Seq> seqs;
+    bool prefix_cache = false;
+    std::unordered_multimap<uint64_t, int32_t> by_key;   // prefix key -> block
+    std::unordered_map<int32_t, Cached> cached;          // block -> entry
+    std::list<int32_t> lru;                              // least recently used first
+    int64_t hits = 0, misses = 0, evictions = 0;
 };
 
 namespace {
@@ -51,6 +75,61 @@ void drop(pa_allocator* a, int32_t b) {  // caller checked refcount > 0
     if (--a->refcount[b] == 0) a->free_ids.push_back(b);
 }
 
+// Prefix key of a block: FNV-1a over the key of the prefix before it and the
+// block's tokens (a 64-bit fingerprint of the whole token prefix).
+uint64_t block_key(uint64_t parent, const int32_t* tokens, int n) {
+    uint64_t h = 1469598103934665603ull ^ (parent * 0x9E3779B97F4A7C15ull);
+    for (int i = 0; i < n; ++i) {
+        uint32_t t = static_cast<uint32_t>(tokens[i]);
+        for (int k = 0; k < 4; ++k) {
+            h ^= (t >> (8 * k)) & 0xffu;
+            h *= 1099511628211ull;
+        }
+    }
+    return h;
+}
+
+// The cached block holding exactly this prefix (key, the key before it and
+// the block's own tokens), or -1.  At most one block per prefix is cached.
+int32_t lookup(const pa_manager* m, uint64_t key, uint64_t parent, const int32_t* t) {
+    auto range = m->by_key.equal_range(key);
+    for (auto k = range.first; k != range.second; ++k) {
+        const auto& c = m->cached.at(k->second);
+        if (c.parent == parent && std::equal(c.tokens.begin(), c.tokens.end(), t)) return k->second;
+    }
+    return -1;
+}
+
+// Take block b out of the cache (the cache's reference is dropped).
+void uncache(pa_manager* m, int32_t b) {
+    auto c = m->cached.find(b);
+    auto range = m->by_key.equal_range(c->second.key);
+    for (auto k = range.first; k != range.second; ++k)
+        if (k->second == b) { m->by_key.erase(k); break; }
+    m->lru.erase(c->second.lru);
+    m->cached.erase(c);
+    drop(m->alloc, b);
+}
+
+// Free one cached block that only the cache still references (least recently
+// used first).  Returns false if there is none.
+bool evict_one(pa_manager* m) {
+    for (auto it = m->lru.begin(); it != m->lru.end(); ++it) {
+        const int32_t b = *it;
+        if (m->alloc->refcount[b] != 1) continue;
+        uncache(m, b);                // back to the free pool
+        ++m->evictions;
+        return true;
+    }
+    return false;
+}
+
+// A block for a new table entry: from the free pool, else by evicting.
+bool have_free(pa_manager* m) {
+    if (!m->alloc->free_ids.empty()) return true;
+    return m->prefix_cache && evict_one(m) && !m->alloc->free_ids.empty();
+}
+
 // One append, with enough recorded to undo it.
 struct Undo {
     pa_manager::Seq* seq;
@@ -68,14 +147,14 @@ int append_one(pa_manager* m, pa_manager::Seq& s, int64_t* slot, Undo* u,
     *cow_src = -1;
     *cow_dst = -1;
     if (p % bs == 0) {
-        if (a->free_ids.empty()) return PA_ERR_OOM;
+        if (!have_free(m)) return PA_ERR_OOM;
         u->taken = take(a);
         s.table.push_back(u->taken);
         u->grew = true;
     } else {
         int32_t last = s.table.back();
         if (a->refcount[last] > 1) {
-            if (a->free_ids.empty()) return PA_ERR_OOM;
+            if (!have_free(m)) return PA_ERR_OOM;
             u->taken = take(a);
             u->cow_src = last;
             drop(a, last);
@@ -311,6 +390,88 @@ int pa_manager_block_tables(const pa_manager* m, const int64_t* seq_ids, int num
         for (; k < max_blocks; ++k) row[k] = -1;
         context_lens[i] = it->second.len;
     }
+    return PA_OK;
+}
+
+int pa_manager_enable_prefix_cache(pa_manager* m) {
+    if (!m) return PA_ERR_INVALID;
+    if (!m->seqs.empty()) return PA_ERR_STATE;
+    m->prefix_cache = true;
+    return PA_OK;
+}
+
+int pa_manager_add_seq_prompt(pa_manager* m, int64_t seq_id, const int32_t* tokens,
+                              int num_tokens, int64_t* slots, int* num_cached) {
+    if (!m || num_tokens < 0 || !num_cached || (num_tokens > 0 && (!tokens || !slots)))
+        return PA_ERR_INVALID;
+    if (!m->prefix_cache) return PA_ERR_STATE;
+    if (m->seqs.count(seq_id)) return PA_ERR_STATE;
+    pa_allocator* a = m->alloc;
+    const int bs = m->block_size;
+    pa_manager::Seq s;
+    // 1. the longest run of leading full blocks already cached
+    uint64_t parent = 0;
+    int hit = 0;
+    const int full = num_tokens / bs;
+    for (; hit < full; ++hit) {
+        const int32_t* t = tokens + static_cast<int64_t>(hit) * bs;
+        const uint64_t key = block_key(parent, t, bs);
+        const int32_t found = lookup(m, key, parent, t);
+        if (found < 0) break;
+        a->refcount[found] += 1;
+        auto& c = m->cached.at(found);
+        m->lru.splice(m->lru.end(), m->lru, c.lru);     // most recently used
+        s.table.push_back(found);
+        parent = key;
+    }
+    s.len = hit * bs;
+    // 2. the rest is appended; every prompt block it fills is registered
+    std::vector<int32_t> registered;   // blocks this call put in the cache
+    for (int i = s.len; i < num_tokens; ++i) {
+        if (i % bs == 0) {
+            if (!have_free(m)) {
+                // nothing of this call stays: its blocks will never be written
+                for (int32_t b : registered) uncache(m, b);
+                for (int32_t b : s.table) drop(a, b);   // hits and new blocks alike
+                return PA_ERR_OOM;
+            }
+            s.table.push_back(take(a));
+        }
+        s.len = i + 1;
+        if ((i + 1) % bs == 0) {                         // a full prompt block
+            const int32_t blk = s.table.back();
+            const int32_t* t = tokens + static_cast<int64_t>(i + 1 - bs);
+            const uint64_t key = block_key(parent, t, bs);
+            if (lookup(m, key, parent, t) >= 0) {        // this prefix is cached already
+                parent = key;
+                continue;
+            }
+            m->lru.push_back(blk);
+            m->cached.emplace(blk, pa_manager::Cached{key, parent,
+                                                      std::vector<int32_t>(t, t + bs),
+                                                      std::prev(m->lru.end())});
+            m->by_key.emplace(key, blk);
+            a->refcount[blk] += 1;                       // the cache's reference
+            registered.push_back(blk);
+            parent = key;
+        }
+    }
+    m->hits += hit;
+    m->misses += full - hit;
+    for (int i = 0; i < num_tokens; ++i)
+        slots[i] = i < hit * bs ? -1
+                                : static_cast<int64_t>(s.table[i / bs]) * bs + i % bs;
+    *num_cached = hit * bs;
+    m->seqs.emplace(seq_id, std::move(s));
+    return PA_OK;
+}
+
+int pa_manager_prefix_cache_stats(const pa_manager* m, int64_t* stats) {
+    if (!m || !stats) return PA_ERR_INVALID;
+    stats[0] = static_cast<int64_t>(m->cached.size());
+    stats[1] = m->hits;
+    stats[2] = m->misses;
+    stats[3] = m->evictions;
     return PA_OK;
 }
 

@@ -415,3 +415,62 @@ def test_full_size_sampled(name, kw):
             for (s, h), r in ref.items():
                 check_close(got[s, h][None, None], r[None, None], w.dtype, f"{name} step {k} ({s},{h})")
     assert g.caches_equal_oracle()
+
+
+# ---------------------------------------------------------------- prefix caching
+
+def test_prefix_cache_decode_bit_identical():
+    """Prompts sharing leading tokens, K/V a function of the token id: with the
+    prefix cache, later prompts map the cached blocks (written once, their own
+    slots come back as -1 and are skipped by the cache write); the decode equals
+    the same prompts stored privately bit for bit, and the oracle's within
+    tolerance."""
+    g = torch.Generator().manual_seed(7)
+    bs, hkv, G, d, V = 16, 2, 4, 128, 40
+    emb_k = torch.randn(V, hkv, d, generator=g).bfloat16()
+    emb_v = torch.randn(V, hkv, d, generator=g).bfloat16()
+    base = torch.randint(0, V, (96,), generator=g).tolist()
+    prompts = [base[:L] + torch.randint(0, V, (t,), generator=g).tolist()
+               for L, t in [(96, 5), (64, 20), (96, 0), (33, 40), (80, 17), (0, 50)]]
+    S = len(prompts)
+    nb = sum(-(-len(p) // bs) for p in prompts) + 4
+    max_len = max(len(p) for p in prompts)
+    mb = -(-max_len // bs)
+    q = torch.randn(S, hkv * G, d, generator=g).bfloat16().cuda()
+
+    def run(cached):
+        alloc = pa.BlockAllocator(nb)
+        mgr = pa.BlockManager(alloc, bs)
+        if cached:
+            mgr.enable_prefix_cache()
+        kc = torch.zeros(nb, hkv, bs, d, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        hits = 0
+        for s, p in enumerate(prompts):
+            if cached:
+                slots, n = mgr.add_seq_prompt(s, p)
+                hits += n
+            else:
+                mgr.add_seq(s)
+                slots, _ = mgr.append(s, len(p))
+            ids = torch.tensor(p, dtype=torch.long)
+            pa.pa_reshape_and_cache(emb_k[ids].cuda(), emb_v[ids].cuda(), kc, vc, slots.cuda())
+        tab, lens = mgr.block_tables(range(S), mb)
+        out = torch.empty_like(q)
+        ws = pa.alloc_workspace(S, hkv * G, hkv, d, max_len, 32)
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pa.pa_decode(out, q, kc, vc, tab.cuda(), lens.cuda(), max_len, d ** -0.5,
+                     partition_size=32, workspace=ws, err_flag=err)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        blocks_used = alloc.num_blocks - alloc.num_free()
+        return out.cpu(), kc.cpu(), vc.cpu(), tab, lens, hits, blocks_used
+
+    a_out, a_k, a_v, a_tab, a_lens, hits, a_used = run(True)
+    b_out, b_k, b_v, b_tab, b_lens, _, b_used = run(False)
+    assert hits >= 3 * bs and a_used < b_used      # the cache really served blocks
+    assert torch.equal(a_out, b_out)
+    ref = oracle.paged_decode(oracle.as_storage(q.cpu(), "bf16"), oracle.as_storage(a_k, "bf16"),
+                              oracle.as_storage(a_v, "bf16"), a_tab.numpy(), a_lens.numpy(),
+                              d ** -0.5, "bf16")
+    check_close(out_f64(a_out, "bf16"), ref, "bf16", "prefix-cached prompts vs oracle")

@@ -161,6 +161,15 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
 enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_TENSOR = 2 };
 int pa_set_decode_engine(int engine);
 
+/* Test hook for the bounded-wait path (failure detection without a fault):
+ * with stage >= 0, in every later pa_decode call the producer that takes the
+ * first work unit withholds that unit's stage number `stage` (no copies, no
+ * arrival on the stage's barrier), so the warps that need it give up after
+ * the 2 s wait limit, set PA_DEV_TIMEOUT in err_flag and return; the context
+ * and the workspace stay usable.  -1 (the default) switches it off.
+ * Process-wide; returns the previous value.  The pages have no counterpart. */
+int pa_test_withhold_stage(int stage);
+
 /* --------------------------------------------------------------------------
  * pa_copy_blocks - copy-on-write block copies.
  *

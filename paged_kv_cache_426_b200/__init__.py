@@ -46,6 +46,7 @@ SIGNATURES = {
     "pa_decode_static": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
                           _i, _vp, _vp], _i),
     "pa_set_decode_engine": ([_i], _i),
+    "pa_test_withhold_stage": ([_i], _i),
     "pa_copy_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "pa_allocator_create": ([_i, _pi32, _i, C.POINTER(_vp)], _i),
     "pa_allocator_destroy": ([_vp], None),

@@ -21,6 +21,9 @@ reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict_
                          uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
                          const int64_t* __restrict__ slots, int64_t total, int row_vecs, int Hkv,
                          int bs, int64_t num_slots, int32_t* err) {
+    // a decode launched after this kernel may be scheduled now; it waits on
+    // the device for this grid's writes before it reads the cache
+    launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += stride) {
         const int64_t row = i / row_vecs;           // (token, head)

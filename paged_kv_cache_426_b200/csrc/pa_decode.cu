@@ -86,6 +86,7 @@ struct DecodeParams {
     int mbps, max_len, S, Hq, Hkv, NB, bs, bs_log2, P, n_pmax, nst;
     float scale_log2e;
     WsHeader* hdr;
+    int hold_stage;    // test hook: stage of unit 0 that its producer withholds (-1: none)
     float* part_ml;    // [S*Hkv][n_pmax][G][2]
     float* part_o;     // [S*Hkv][n_pmax][G][D]
     int32_t* err;
@@ -152,6 +153,25 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((it & 63) == 0 && global_ns() - t0 > kWaitLimitNs) {
+            set_err(err, PA_DEV_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Bounded wait until a ring slot's tag (2 * stage + valid, written by the
+// producer before it arms the slot's barrier) names global stage `g`.  Gives
+// up like wait_or_abort; on success *tag holds the value read.
+__device__ __forceinline__ bool wait_tag(const volatile int* slot_tag, int g, int* tag,
+                                         volatile int* abort_flag, int32_t* err) {
+    if ((*tag = *slot_tag) >> 1 == g) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if ((*tag = *slot_tag) >> 1 == g) return true;
         if (*abort_flag) return false;
         if ((it & 63) == 0 && global_ns() - t0 > kWaitLimitNs) {
             set_err(err, PA_DEV_TIMEOUT);
@@ -436,7 +456,7 @@ struct PipeRings {
     uint8_t* stages;
     uint64_t *full, *empty;     // per stage slot
     uint64_t *ufull, *uempty;   // per unit slot
-    int* stage_ok;
+    int* stage_ok;              // per stage slot: tag 2 * global stage + valid
     int nst, nu;
 };
 
@@ -555,8 +575,14 @@ __device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
             const bool has1 = blk1 != -2;
             const bool valid = blk0 >= 0 && blk0 < p.NB && (!has1 || (blk1 >= 0 && blk1 < p.NB));
             uint8_t* Kd = rg.stages + (size_t)st * R::STAGE_BYTES;
+            if (cur.u == 0 && c == p.hold_stage) {
+                // test hook: nothing will ever arrive on this stage's barrier
+                ++gstage;
+                if (++st == nst) { st = 0; ++round; }
+                continue;
+            }
             if (lane == 0) {
-                rg.stage_ok[st] = valid ? 1 : 0;
+                rg.stage_ok[st] = 2 * gstage + (valid ? 1 : 0);   // the slot's tag
                 if (!valid) {
                     set_err(p.err, PA_DEV_BAD_BLOCK);
                     mbar_arrive(rg.full + st);
@@ -754,6 +780,8 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         for (int pp = 0; pp < NPIPE; ++pp) {
             uint64_t* b = reinterpret_cast<uint64_t*>(smem + ly.bars(pp));
             for (int k = 0; k < 2 * nst + 2 * NUR; ++k) mbar_init(b + k, 1);
+            int* tags = reinterpret_cast<int*>(smem + ly.stage_ok(pp));
+            for (int k = 0; k < nst; ++k) tags[k] = -1;   // no stage issued yet
         }
         for (int k = 0; k < 32; ++k) misc[k] = 0;
         fence_barrier_init();
@@ -762,6 +790,7 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
     }
+    grid_dependency_wait();              // inputs written by the previous kernel are visible
     prefix_sums<NTHREADS>(p, lens_s, pre, wsum, tid);
     const int U = pre[p.S] * p.Hkv;
 
@@ -799,8 +828,19 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
             int st = (d.stage_base + cw) % nst;
             uint32_t ph = ((d.stage_base + cw) / nst) & 1;
             for (int c = cw; c < d.n_stages; c += NCONS) {
-                const bool have = __all_sync(0xffffffffu, wait_or_abort(full + st, ph, abort_flag, p.err));
-                if (have && stage_ok[st]) {
+                // A slot's successive rounds may go to different consumer
+                // warps, and a parity wait cannot tell round R from round
+                // R - 2.  So first wait for the slot's tag to name this very
+                // stage: the producer writes it only after round R - 1 was
+                // consumed, and from then on the parity is unambiguous.
+                int tag = -1;
+                bool okt = true;
+                if (lane == 0) okt = wait_tag(stage_ok + st, d.stage_base + c, &tag, abort_flag, p.err);
+                okt = __shfl_sync(0xffffffffu, okt, 0);
+                tag = __shfl_sync(0xffffffffu, tag, 0);
+                const bool have =
+                    __all_sync(0xffffffffu, okt && wait_or_abort(full + st, ph, abort_flag, p.err));
+                if (have && (tag & 1)) {
                     const int nv = min(TOK, d.t1 - (d.t0 + c * TOK));
                     uint8_t* Ks = stages + (size_t)st * LY::STAGE_BYTES;
                     eng.stage(Ks, Ks + LY::KV_BYTES, nv, xs, ps, lane);
@@ -1157,6 +1197,13 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
             want = __reduce_or_sync(FULL, want);
             got = __reduce_or_sync(FULL, got);
             uint8_t* stage = smem + ly.ring(st);
+            if (cur.u == 0 && c == p.hold_stage) {
+                // test hook: nothing will ever arrive on this stage's barrier
+                ++gstage;
+                if (++st == nst) { st = 0; ++round; }
+                if (!have_next) next_plan();
+                continue;
+            }
             if (lane == 0) {
                 stage_ok[st] = (int)got;
                 if (want & ~got) set_err(p.err, PA_DEV_BAD_BLOCK);
@@ -1251,6 +1298,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
+    grid_dependency_wait();              // inputs written by the previous kernel are visible
     schedule_units<TC_THREADS>(p, lens_s, preF, order, reinterpret_cast<int*>(smem + ly.sched()), wsum, tid);
     tc::fence_before();
     __syncthreads();
@@ -1623,6 +1671,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 namespace {
 
 int g_engine = PA_ENGINE_AUTO;
+int g_hold_stage = -1;
 std::mutex g_mu;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1722,6 +1771,26 @@ int pick_stages(const Launch& L, size_t budget, size_t per_stage, int* nst_out, 
     return *smem_out > budget ? PA_ERR_UNSUPPORTED : PA_OK;
 }
 
+// Launch as a programmatic dependent of the previous kernel in the stream:
+// the decode kernel's set-up (barriers, tensor memory) overlaps that kernel's
+// tail, and every thread waits (griddepcontrol.wait) before its first read of
+// global memory, so whatever the previous kernel wrote is visible.
+template <class Kern, class... Args>
+int launch_dependent(Kern kern, dim3 grid, int threads, size_t smem, cudaStream_t stream,
+                     Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...) == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 template <class Kern>
 int set_smem_attr(Kern kern, const DevInfo& di, bool* done) {
     int dev = 0;
@@ -1745,8 +1814,7 @@ int run_decode_core(Launch& L, const DevInfo& di) {
     L.threads = LY::NTHREADS;
     static bool attr_set[64] = {};
     if ((st = set_smem_attr(kern, di, attr_set)) != PA_OK) return st;
-    kern<<<L.grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_dependent(kern, L.grid, L.threads, L.smem, L.stream, L.kmap, L.vmap, L.p);
 }
 
 template <typename T, int D, int G>
@@ -1766,8 +1834,7 @@ int run_decode_tc(Launch& L, const DevInfo& di) {
         static bool attr_set[64] = {};
         if ((st = set_smem_attr(kern, di, attr_set)) != PA_OK) return st;
         const dim3 grid((unsigned)std::max<int64_t>(1, std::min<int64_t>(L.units_ub, 2 * (int64_t)di.sms)));
-        kern<<<grid, L.threads, L.smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
-        return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+        return launch_dependent(kern, grid, L.threads, L.smem, L.stream, L.kmap, L.vmap, L.qmap, L.p);
     }
 }
 
@@ -1833,6 +1900,14 @@ int launch_merge(const Launch& L, pa_dtype dt, int D, int G, int n_pmax) {
 using namespace pa;
 
 extern "C" {
+
+int pa_test_withhold_stage(int stage) {
+    if (stage < -1) return PA_ERR_INVALID;
+    std::lock_guard<std::mutex> lk(g_mu);
+    const int prev = g_hold_stage;
+    g_hold_stage = stage;
+    return prev;
+}
 
 int pa_set_decode_engine(int engine) {
     if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_TENSOR) return PA_ERR_INVALID;
@@ -1924,6 +1999,10 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader));
     p.part_o = p.part_ml + ((((size_t)num_seqs * num_q_heads * n_pmax * 2 * 4 + 255) / 256) * 256) / 4;
     p.err = err_flag;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        p.hold_stage = g_hold_stage;
+    }
 
     const int64_t units_ub = (int64_t)num_seqs * num_kv_heads * n_pmax;
     L.units_ub = units_ub;

@@ -474,3 +474,48 @@ def test_prefix_cache_decode_bit_identical():
                               oracle.as_storage(a_v, "bf16"), a_tab.numpy(), a_lens.numpy(),
                               d ** -0.5, "bf16")
     check_close(out_f64(a_out, "bf16"), ref, "bf16", "prefix-cached prompts vs oracle")
+
+
+# ---------------------------------------------------------------- failure detection
+
+@pytest.mark.parametrize("engine_id", [1, 2])
+def test_bounded_wait_reports_timeout(engine_id):
+    """Failure detection without a fault: a stage whose barrier nothing will
+    arrive on (test hook pa_test_withhold_stage) makes the waiting warps give
+    up after the 2 s limit; the call returns, err_flag says PA_DEV_TIMEOUT, and
+    the next call on the same workspace and context is correct."""
+    import time
+    w = workloads.gqa8b_bf16(num_seqs=6)
+    rec = oracle.run(w, keep_prefill_cache=True)
+    g = GpuRun(w, rec, partition_size=512)
+    g.replay_prefill()
+    st = rec.steps[0]
+    slots, _ = g.mgr.append_step(st.seqs)
+    tab, lens = g.mgr.block_tables(st.seqs, g.mb)
+    pa.pa_reshape_and_cache(w.step_k[0].cuda(), w.step_v[0].cuda(), g.kc, g.vc, slots.cuda(),
+                            err_flag=g.err)
+    q = w.step_q[0].cuda()
+    out = torch.empty_like(q)
+    tab_d, lens_d = tab.cuda(), lens.cuda()
+
+    def decode():
+        pa.pa_decode(out, q, g.kc, g.vc, tab_d, lens_d, g.max_len, w.scale, partition_size=512,
+                     workspace=g.ws, err_flag=g.err)
+        torch.cuda.synchronize()
+
+    prev = pa.pa_set_decode_engine(engine_id)
+    try:
+        pa.lib.pa_test_withhold_stage(0)
+        t0 = time.time()
+        decode()
+        dt = time.time() - t0
+        assert int(g.err.item()) == pa.PA_DEV_TIMEOUT
+        assert 1.0 < dt < 30.0
+        pa.lib.pa_test_withhold_stage(-1)
+        g.err.zero_()
+        decode()
+        assert int(g.err.item()) == 0
+        check_close(out_f64(out, w.dtype), st.out, w.dtype, "the call after a timed-out one")
+    finally:
+        pa.lib.pa_test_withhold_stage(-1)
+        pa.pa_set_decode_engine(prev)

@@ -12,7 +12,9 @@ Modules:
 * ``cache``     - cache write / block copy / gather through the block table,
                   at bit level in the storage dtype;
 * ``attention`` - gather, then textbook softmax attention in float64;
-* ``run``       - executes a workload's host script with the above.
+* ``prefill``   - the causal multi-query (prefill chunk) form of the same;
+* ``run``       - executes a workload's host script with the above (and
+                  replays a prefill batch).
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against the pages'
 worked examples (``tests/golden``), closed forms, brute force on tiny inputs
@@ -20,13 +22,15 @@ and invariants.
 """
 from .attention import attend, decode_one, paged_decode
 from .blocks import BlockAllocator, BlockManager, BlockStateError, OutOfBlocks
+from .prefill import paged_prefill, prefill_rows
 from .cache import (STORAGE, as_storage, copy_blocks, empty_cache, gather_kv,
                     reshape_and_cache, to_f64)
-from .run import OracleRun, StepRecord, max_blocks_needed, run
+from .run import OracleRun, PrefillRecord, StepRecord, max_blocks_needed, run, run_prefill
 
 __all__ = [
-    "attend", "decode_one", "paged_decode", "BlockAllocator", "BlockManager",
+    "attend", "decode_one", "paged_decode", "paged_prefill", "prefill_rows",
+    "BlockAllocator", "BlockManager",
     "BlockStateError", "OutOfBlocks", "STORAGE", "as_storage", "copy_blocks",
     "empty_cache", "gather_kv", "reshape_and_cache", "to_f64", "OracleRun",
-    "StepRecord", "max_blocks_needed", "run",
+    "StepRecord", "max_blocks_needed", "run", "PrefillRecord", "run_prefill",
 ]

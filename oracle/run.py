@@ -18,6 +18,7 @@ import numpy as np
 from .attention import paged_decode
 from .blocks import BlockAllocator, BlockManager
 from .cache import as_storage, copy_blocks, empty_cache, reshape_and_cache
+from .prefill import paged_prefill, prefill_rows
 
 
 @dataclass
@@ -101,4 +102,60 @@ def run(w, *, decode=True, steps=None, max_blocks=None, canary=0,
             rec.steps.append(st)
         else:
             raise ValueError(f"unknown op {op[0]}")
+    return rec
+
+
+@dataclass
+class PrefillRecord:
+    key_cache: np.ndarray
+    value_cache: np.ndarray
+    context_slots: list               # per sequence: int64 slots of the tokens before the chunk
+    chunk_slots: np.ndarray           # int64 [sum(query_lens)], the chunk's slots packed
+    block_tables: np.ndarray          # int32 [S, max_blocks], -1 padded
+    context_lens: np.ndarray          # int32 [S]
+    cu_seqlens_q: np.ndarray          # int32 [S + 1]
+    out: np.ndarray | None = None     # float64 [sum(query_lens), Hq, D] (rows asked for)
+
+
+def run_prefill(b, *, rows=None, compute=True, canary=0) -> PrefillRecord:
+    """Replay a ``workloads.PrefillBatch``: every sequence takes its
+    context_lens[s] slots from a fresh manager (FIFO pool), the tokens before
+    the chunk are written, then the chunk's, then causal attention.  ``rows``
+    (optional): {seq: [chunk rows]} to compute only those rows (others zero)."""
+    alloc = BlockAllocator(b.num_blocks, b.free_order)
+    mgr = BlockManager(alloc, b.block_size)
+    kc = empty_cache(b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim, b.dtype, canary)
+    vc = empty_cache(b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim, b.dtype, canary)
+    ctx_slots, chunk_slots = [], []
+    for s, (L, n) in enumerate(zip(b.context_lens, b.query_lens)):
+        mgr.add_seq(s)
+        slots = np.array([mgr.append(s)[0] for _ in range(L)], dtype=np.int64)
+        k, v = as_storage(b.k[s], b.dtype), as_storage(b.v[s], b.dtype)
+        reshape_and_cache(kc, vc, k[:L - n], v[:L - n], slots[:L - n])
+        ctx_slots.append(slots[:L - n])
+        chunk_slots.append(slots[L - n:])
+    for s, (L, n) in enumerate(zip(b.context_lens, b.query_lens)):
+        k, v = as_storage(b.k[s], b.dtype), as_storage(b.v[s], b.dtype)
+        reshape_and_cache(kc, vc, k[L - n:], v[L - n:], chunk_slots[s])
+    S = len(b.context_lens)
+    mb = max(1, max(-(-L // b.block_size) for L in b.context_lens))
+    tab, lens = mgr.table_rows(list(range(S)), mb)
+    cu = np.asarray(b.query_offsets, dtype=np.int32)
+    rec = PrefillRecord(kc, vc, ctx_slots,
+                        np.concatenate(chunk_slots) if chunk_slots else np.zeros(0, np.int64),
+                        np.asarray(tab, dtype=np.int32), np.asarray(lens, dtype=np.int32), cu)
+    if compute:
+        q = as_storage(b.q, b.dtype)
+        if rows is None:
+            rec.out = paged_prefill(q, kc, vc, rec.block_tables, rec.context_lens, cu, b.scale,
+                                    b.dtype)
+        else:
+            hkv, G = b.num_kv_heads, b.num_q_heads // b.num_kv_heads
+            rec.out = np.zeros((int(cu[-1]), b.num_q_heads, b.head_dim))
+            for s, rs in rows.items():
+                a, e = int(cu[s]), int(cu[s + 1])
+                for j in range(hkv):
+                    o = prefill_rows(q[a:e], kc, vc, rec.block_tables[s], int(rec.context_lens[s]),
+                                     e - a, b.scale, j, b.dtype, rows=rs)
+                    rec.out[a:e, j * G:(j + 1) * G] = o
     return rec

@@ -296,6 +296,112 @@ def long_bf16(steps: int = 1, num_seqs: int = 8) -> Workload:
                                      "fully shuffled pool"))
 
 
+@dataclass
+class PrefillBatch:
+    """A chunked-prefill batch.  Sequence s holds ``context_lens[s]`` tokens
+    once its chunk is written; the chunk is its last ``query_lens[s]`` tokens.
+    ``k[s]``/``v[s]`` are all of its K/V rows [context_lens[s], Hkv, D] in
+    logical order (the runner writes the first context_lens[s] -
+    query_lens[s] before the step and the chunk's rows in the step), ``q``
+    the chunk queries of every sequence packed in order [sum(query_lens), Hq,
+    D].  Block pool as in ``Workload``."""
+    name: str
+    dtype: str
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    free_order: list
+    context_lens: list
+    query_lens: list
+    k: list
+    v: list
+    q: torch.Tensor
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def torch_dtype(self):
+        return DTYPES[self.dtype]
+
+    @property
+    def scale(self) -> float:
+        """Softmax scale 1/sqrt(head_dim), as for the decode batches."""
+        return 1.0 / math.sqrt(self.head_dim)
+
+    @property
+    def query_offsets(self) -> list:
+        """Row of ``q`` where each sequence's chunk starts, and the total."""
+        out = [0]
+        for n in self.query_lens:
+            out.append(out[-1] + n)
+        return out
+
+
+def _prefill_batch(name, dtype, seed, lens, qlens, hq, hkv, d, bs, pool, meta):
+    g = _gen(seed)
+    k = [_normal(g, (L, hkv, d), dtype) for L in lens]
+    v = [_normal(g, (L, hkv, d), dtype) for L in lens]
+    q = _normal(g, (sum(qlens), hq, d), dtype)
+    needed = sum(-(-L // bs) for L in lens)
+    num_blocks, free_order = pool(g, needed)
+    meta = dict(meta)
+    meta.update(blocks_needed=needed)
+    return PrefillBatch(name=name, dtype=dtype, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
+                        block_size=bs, num_blocks=num_blocks, free_order=free_order,
+                        context_lens=list(lens), query_lens=list(qlens), k=k, v=v, q=q,
+                        meta=meta)
+
+
+def _shuffled_pool(extra=0.1):
+    def pool(g, needed):
+        nb = math.ceil((1 + extra) * needed) + 1
+        return nb, _perm(g, nb)
+    return pool
+
+
+def prefill_gqa8b_bf16(num_seqs: int = 32, chunk: int = 512) -> PrefillBatch:
+    """Chunked prefill on the 8B-shaped GQA layer, bf16: 32 sequences, 32
+    query heads over 8 KV heads, head dim 128, block 16; context lengths
+    uniform on [512, 4096] and each sequence's chunk its last 512 tokens (the
+    latest chunk of a long prompt; a 512-token prompt is a whole prompt);
+    q/K/V ~ N(0,1); pool = blocks needed + 10%, shuffled ids."""
+    g = _gen(BASE_SEED + 20)
+    lens = _uniform_int(g, chunk, 4096, num_seqs)
+    return _prefill_batch("prefill_gqa8b_bf16", "bf16", BASE_SEED + 20 + 1000, lens,
+                          [chunk] * num_seqs, 32, 8, 128, 16, _shuffled_pool(),
+                          dict(recipe=f"L~U{{{chunk}..4096}}, chunk = last {chunk} tokens; "
+                                      "q,K,V~N(0,1); pool=needed+10%, shuffled ids"))
+
+
+def prefill_mha7b_f16(num_seqs: int = 16) -> PrefillBatch:
+    """Whole-prompt prefill on the 7B-shaped MHA layer, fp16: 16 prompts of
+    lengths uniform on [128, 2048], 32 = 32 heads, head dim 128, block 16,
+    q/K/V ~ N(0,1), pool = blocks needed + 10%, shuffled ids."""
+    g = _gen(BASE_SEED + 21)
+    lens = _uniform_int(g, 128, 2048, num_seqs)
+    return _prefill_batch("prefill_mha7b_f16", "f16", BASE_SEED + 21 + 1000, lens, lens,
+                          32, 32, 128, 16, _shuffled_pool(),
+                          dict(recipe="L~U{128..2048}, whole prompts; q,K,V~N(0,1); "
+                                      "pool=needed+10%, shuffled ids"))
+
+
+def prefill_custom(dtype, lens, qlens, hq, hkv, d, bs, seed, extra_blocks=3) -> PrefillBatch:
+    """Small ad-hoc prefill batch for edge cases (same recipe: q/K/V ~ N(0,1),
+    pool = blocks needed + extra_blocks, shuffled ids)."""
+    def pool(g, needed):
+        nb = needed + extra_blocks
+        return nb, _perm(g, nb)
+    return _prefill_batch(f"prefill_custom_{dtype}_{seed}", dtype, seed, list(lens), list(qlens),
+                          hq, hkv, d, bs, pool, {})
+
+
+PREFILL_BUILDERS = {
+    "prefill_gqa8b_bf16": prefill_gqa8b_bf16,
+    "prefill_mha7b_f16": prefill_mha7b_f16,
+}
+
+
 BUILDERS = {
     "tiny_f32": tiny_f32,
     "mha7b_f16": mha7b_f16,

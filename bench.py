@@ -151,6 +151,177 @@ def profiled_traffic(workload, algo_bytes):
     return int(round(t * algo_bytes / a))
 
 
+def profiled_fields(path):
+    """The numeric fields of a committed ncu summary, or None if it is missing
+    or any source it lists (source_sha256_16) has changed since."""
+    import hashlib
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and not line.startswith(" "):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    try:
+        want = dict(x.split("=") for x in fields["source_sha256_16"].split())
+        for name, h in want.items():
+            src = os.path.join(ROOT, "paged_kv_cache_426_b200", "csrc", name)
+            if hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != h:
+                return None
+    except (KeyError, ValueError, OSError):
+        return None
+    return fields
+
+
+def prefill_flops(b):
+    """Algorithmic FLOPs of causal prefill attention: chunk row i of sequence
+    s sees L_s - n_s + i + 1 keys; per query head and key, 2 * head_dim for
+    q.k and 2 * head_dim for p.v."""
+    keys = sum(n * (L - n) + n * (n + 1) // 2 for L, n in zip(b.context_lens, b.query_lens))
+    return 4 * b.head_dim * b.num_q_heads * keys
+
+
+def tensor_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_cpu_baseline(b, seconds):
+    """The prefill oracle, as it stands, on the host cores: float64 causal
+    attention of chunk rows (a few at a time, cycling over sequences and KV
+    heads) for about ``seconds``; throughput in algorithmic TFLOP/s."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    rec = oracle.run_prefill(b, compute=False)
+    q = oracle.as_storage(b.q, b.dtype)
+    cu = b.query_offsets
+    G = b.num_q_heads // b.num_kv_heads
+    S = len(b.context_lens)
+    rows_done, flops, k, t0 = 0, 0, 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        s, j = k % S, (k // S) % b.num_kv_heads
+        L, n = b.context_lens[s], b.query_lens[s]
+        rows = list(range((k * 7) % n, n, max(1, n // 4)))[:4]
+        oracle.prefill_rows(q[cu[s]:cu[s + 1]], rec.key_cache, rec.value_cache, rec.block_tables[s],
+                            L, n, b.scale, j, b.dtype, rows=rows)
+        flops += sum(4 * b.head_dim * G * (L - n + i + 1) for i in rows)
+        rows_done += len(rows)
+        k += 1
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{rows_done} chunk rows x {G} query heads ({k} (sequence, KV head) visits "
+                      f"over {b.name}), float64 numpy (gather through the block table + causal "
+                      f"softmax attention per row), {dt:.1f} s",
+            "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_prefill_bench(args):
+    """One GPU, one JSON line: a step writes the chunks' K/V into the cache
+    (pa_reshape_and_cache) and runs causal prefill attention over the paged
+    cache (pa_prefill).  The tokens before each chunk are written once,
+    untimed."""
+    import paged_kv_cache_426_b200 as pa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    b = workloads.PREFILL_BUILDERS[args.prefill]()
+    td = b.torch_dtype
+    mgr = pa.BlockManager(pa.BlockAllocator(b.num_blocks, b.free_order), b.block_size)
+    shape = (b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim)
+    kc = torch.zeros(shape, dtype=td, device=dev)
+    vc = torch.zeros(shape, dtype=td, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ctx, chunk = [], []
+    for s, (L, n) in enumerate(zip(b.context_lens, b.query_lens)):
+        mgr.add_seq(s)
+        slots = mgr.append(s, L)[0]
+        ctx.append((slots[:L - n], b.k[s][:L - n], b.v[s][:L - n]))
+        chunk.append((slots[L - n:], b.k[s][L - n:], b.v[s][L - n:]))
+    cs = torch.cat([c[0] for c in ctx])
+    if cs.numel():
+        pa.pa_reshape_and_cache(torch.cat([c[1] for c in ctx]).to(dev),
+                                torch.cat([c[2] for c in ctx]).to(dev), kc, vc, cs.to(dev),
+                                err_flag=err)
+    ch_slots = torch.cat([c[0] for c in chunk]).to(dev)
+    ch_k = torch.cat([c[1] for c in chunk]).to(dev)
+    ch_v = torch.cat([c[2] for c in chunk]).to(dev)
+    mb = max(-(-L // b.block_size) for L in b.context_lens)
+    tab, lens = mgr.block_tables(list(range(len(b.context_lens))), mb)
+    tab, lens = tab.to(dev), lens.to(dev)
+    cu = torch.tensor(b.query_offsets, dtype=torch.int32, device=dev)
+    q = b.q.to(dev)
+    out = torch.empty_like(q)
+    max_q = max(b.query_lens)
+    stream = torch.cuda.current_stream()
+
+    def write():
+        pa.pa_reshape_and_cache(ch_k, ch_v, kc, vc, ch_slots, err_flag=err)
+
+    def attend():
+        pa.pa_prefill(out, q, kc, vc, tab, lens, cu, max_q, b.scale, err_flag=err)
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(5):
+            write()
+            attend()
+        torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        write()
+        attend()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        write()
+        ev[i][1].record(stream)
+        attend()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    assert int(err.item()) == 0, f"device error flag {int(err.item())}"
+    span_ms = ev[0][0].elapsed_time(ev[-1][2])
+    pf_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    flop = prefill_flops(b)
+    value = flop * args.steps / (span_ms * 1e-3) / 1e12
+    achieved = flop / (pf_ms * 1e-3) / 1e12
+    peak, kind = tensor_peak()
+    prof = profiled_fields(os.path.join(ROOT, "profiles", f"prefill_{b.name}.md"))
+    traffic = int(prof["traffic_bytes_per_launch"]) if prof else None
+    T = sum(b.query_lens)
+    res = {
+        "metric": "paged prefill attention: causal TFLOP/s per step (chunk write + attention)",
+        "value": round(value, 1), "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(span_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": b.dtype,
+        "data": "synthetic (seeded; see workloads/)",
+        "config": {"workload": b.name, "num_seqs": len(b.context_lens), "chunk_tokens": T,
+                   "num_q_heads": b.num_q_heads, "num_kv_heads": b.num_kv_heads,
+                   "head_dim": b.head_dim, "block_size": b.block_size,
+                   "mean_context_len": round(sum(b.context_lens) / len(b.context_lens), 1),
+                   "flop_per_step": flop, "parallelism": "one GPU",
+                   "l2": "inputs larger than L2 (KV cache, queries and outputs each > 126 MB)"
+                   if b.name == "prefill_gqa8b_bf16" else "KV cache larger than L2"},
+        "prefill_only": {"tflops": round(achieved, 1), "ms": round(pf_ms, 4),
+                         "tokens_per_s": round(T / (pf_ms * 1e-3), 1)},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{kind} cuBLAS bf16 GEMM (burst; fp16 has the same nominal peak)",
+                     "kernel": "pa_prefill"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if args.cpu_baseline:
+        res["cpu_baseline"] = prefill_cpu_baseline(b, args.cpu_seconds)
+    return res
+
+
 def dist_setup(n_gpus):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -674,6 +845,9 @@ def main():
                     help="block-size / indirection study instead of the benchmark line")
     ap.add_argument("--waste", action="store_true",
                     help="host-only memory accounting: paged vs contiguous reservation")
+    ap.add_argument("--prefill", default=None, choices=sorted(workloads.PREFILL_BUILDERS),
+                    help="causal prefill attention over the paged cache on this batch "
+                         "(one GPU) instead of the decode line")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -684,6 +858,9 @@ def main():
         return
     if args.waste:
         run_waste(args)
+        return
+    if args.prefill:
+        print(json.dumps(run_prefill_bench(args)), flush=True)
         return
     if args.impl == "reference":
         res = run_reference(args, rank, world)

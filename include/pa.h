@@ -171,6 +171,45 @@ int pa_set_decode_engine(int engine);
 int pa_test_withhold_stage(int stage);
 
 /* --------------------------------------------------------------------------
+ * pa_prefill - causal multi-query attention of prefill chunks over the paged
+ * cache (tiled attention over paged K/V: "KV Cache & PagedAttention"
+ * studynote, section III, where the serving stack pairs FlashAttention with
+ * PagedAttention; the pages give no formula, the chunk reading is the plain
+ * causal one).
+ *
+ * Sequence s holds context_lens[s] tokens in the cache; its chunk is its last
+ * n_s = cu_seqlens_q[s+1] - cu_seqlens_q[s] tokens, whose K/V must already be
+ * written (pa_reshape_and_cache).  Chunk row i, packed row cu_seqlens_q[s] + i
+ * of `query`, sits at position p = context_lens[s] - n_s + i and attends to
+ * the sequence's tokens 0..p:
+ *   out[row][h] = sum_{t<=p} softmax_t(scale * <query[row][h], K_t>) V_t,
+ * query head h reading KV head h / (num_q_heads / num_kv_heads).  n_s = 1 is
+ * a decode step; n_s = context_lens[s] a whole prompt.
+ *
+ *   out          [total_q][num_q_heads][head_dim]  device, written
+ *   query        [total_q][num_q_heads][head_dim]  device
+ *   key_cache, value_cache, block_tables, num_blocks: as pa_decode
+ *   context_lens [num_seqs] int32 device (they count the chunk)
+ *   cu_seqlens_q [num_seqs + 1] int32 device, 0 = cu[0] <= ... <= cu[num_seqs]
+ *                = total_q
+ *   max_query_len  an upper bound of every n_s (it sizes the launch)
+ *   dtype        PA_F16 or PA_BF16 (tensor cores); PA_F32 -> PA_ERR_UNSUPPORTED
+ * head_dim 64 or 128; num_q_heads / num_kv_heads in {1, 2, 4, 8}; block_size
+ * 8, 16, 32, 64 or 128; every pointer 16-byte aligned.  Nothing is allocated;
+ * asynchronous on `stream`.  Device-side errors (err_flag, first code wins):
+ * PA_DEV_BAD_LEN when context_lens[s] < 0 or > max_blocks_per_seq *
+ * block_size, n_s > context_lens[s] or > max_query_len, or cu_seqlens_q
+ * leaves [0, total_q] (rows of that sequence may then be left unwritten);
+ * PA_DEV_BAD_BLOCK for a table entry outside [0, num_blocks) that a chunk
+ * reads (those tokens are skipped); PA_DEV_TIMEOUT as pa_decode.
+ * Returns PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED or PA_ERR_CUDA. */
+int pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+               const int32_t* cu_seqlens_q, int num_seqs, int total_q, int max_query_len,
+               int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               float scale, pa_dtype dtype, int32_t* err_flag, void* stream);
+
+/* --------------------------------------------------------------------------
  * pa_copy_blocks - copy-on-write block copies.
  *
  * [KVC] II (copy-on-write) / [VEL] 메모리 공유: before a sharer writes into a

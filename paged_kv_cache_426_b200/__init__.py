@@ -47,6 +47,8 @@ SIGNATURES = {
                           _i, _vp, _vp], _i),
     "pa_set_decode_engine": ([_i], _i),
     "pa_test_withhold_stage": ([_i], _i),
+    "pa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+                    _i, _vp, _vp], _i),
     "pa_copy_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "pa_allocator_create": ([_i, _pi32, _i, C.POINTER(_vp)], _i),
     "pa_allocator_destroy": ([_vp], None),
@@ -187,6 +189,25 @@ def pa_decode_static(out, query, key_cache, value_cache, block_tables, context_l
                                int(max_context_len), S, hq, hkv, d, bs, NB, float(scale),
                                int(partition_size), pa_dtype(query), _ptr(err_flag),
                                _stream(stream)), "pa_decode_static")
+
+
+def pa_prefill(out, query, key_cache, value_cache, block_tables, context_lens, cu_seqlens_q,
+               max_query_len, scale, *, err_flag=None, stream=None):
+    """Causal attention of packed prefill chunks: out/query [T, Hq, D]; caches
+    [NB, Hkv, bs, D]; block_tables int32 [S, max_blocks]; context_lens int32
+    [S] (counting the chunk); cu_seqlens_q int32 [S + 1] (row offsets of the
+    chunks in query)."""
+    _cuda(out, query, key_cache, value_cache, block_tables, context_lens, cu_seqlens_q, err_flag)
+    T, hq, d = query.shape
+    NB, hkv, bs, _ = key_cache.shape
+    S = context_lens.shape[0]
+    if cu_seqlens_q.shape[0] != S + 1:
+        raise PAError(PA_ERR_INVALID, "cu_seqlens_q needs num_seqs + 1 entries")
+    check(lib.pa_prefill(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                         _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                         _ptr(cu_seqlens_q), S, T, int(max_query_len), hq, hkv, d, bs, NB,
+                         float(scale), pa_dtype(query), _ptr(err_flag), _stream(stream)),
+          "pa_prefill")
 
 
 def pa_set_decode_engine(engine: int) -> int:

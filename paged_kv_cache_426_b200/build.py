@@ -24,7 +24,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libpa_b200.so")
 
-SOURCES = ["pa_host.cpp", "pa_cache_ops.cu", "pa_decode.cu"]
+SOURCES = ["pa_host.cpp", "pa_cache_ops.cu", "pa_decode.cu", "pa_prefill.cu"]
 HEADERS = sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(INCLUDE, "pa.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

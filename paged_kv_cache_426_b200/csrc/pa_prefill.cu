@@ -1,0 +1,665 @@
+// Paged prefill (chunked) attention on the sm_100a tensor cores.
+//
+// A chunk of n new tokens at the end of a sequence of L cached tokens attends
+// causally over the paged cache: chunk row i sits at position p = L - n + i
+// and reads tokens 0..p.  FlashAttention's idea (attention computed in tiles
+// so that K/V cross between HBM and on-chip memory once per tile, the
+// "KV Cache & PagedAttention" studynote, section III) is kept; the tiles come
+// through the block table.
+//
+// A query tile is M = 128 rows: 128 / G chunk tokens x the G query heads that
+// share a KV head, so every K/V tile read feeds G heads at once.  One CTA
+// takes two adjacent query tiles of one (sequence, KV head) and streams the
+// K/V stages once for both.  Per 64-key stage and tile:
+//   S  = Q K^T      M = 128, N = 64, K = head_dim        (tcgen05, fp32 in TMEM)
+//   P  = exp2(S * scale * log2 e - m), rounded to the input type, in smem
+//   O += P V        M = 128, N = head_dim, K = 64 keys    (tcgen05, fp32 in TMEM)
+// Warps: 0-3 softmax + epilogue of tile 0, 4-7 of tile 1 (thread = one row =
+// one tensor-memory lane), 8 TMA producer, 9 MMA issuer (one thread).  The
+// two softmax groups run side by side (two warps per SM sub-partition) while
+// the tensor core works on the other tile; S is double-buffered in tensor
+// memory and P in shared memory per tile.  The row maximum m is moved lazily:
+// only when a stage exceeds it by 2^8 is O rescaled in tensor memory.  Keys
+// past the row's position get weight 0; keys past the CTA's key range or in a
+// block whose table entry is bad also get their V rows zeroed in shared
+// memory (the product 0 * V must not meet stale or non-finite data).
+//
+// Every wait is bounded (2 s): a timeout sets PA_DEV_TIMEOUT, makes the other
+// warps give up at their next wait, and the kernel returns.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "pa.h"
+#include "pa_common.cuh"
+#include "pa_tcgen05.cuh"
+
+namespace pa {
+namespace {
+
+constexpr int PF_KT = 64;          // keys per stage (N of S, K of PV)
+constexpr int PF_M = 128;          // query rows per tile
+constexpr int PF_TILES = 2;        // query tiles per CTA
+constexpr int PF_THREADS = 320;    // 8 softmax warps, producer, MMA issuer
+constexpr int PF_MAX_STAGES = 4;
+constexpr float kPfRescaleLog2 = 8.f;
+constexpr uint32_t PF_FULL = 0xffffffffu;
+
+struct PrefillParams {
+    void* out;
+    const void* q;
+    const int32_t* tables;
+    const int32_t* lens;
+    const int32_t* cu;
+    int S, total_q, max_q, npair, Hq, Hkv, mbps, NB, bs, bs_log2, nst;
+    float scale_log2e;
+    int32_t* err;
+};
+
+// Shared memory (1024-byte aligned; every operand tile starts on a 1024-byte
+// boundary, as the 128-byte swizzle wants):
+//   Q        per tile NBOX boxes of [128 rows][128 B]
+//   P        per tile two buffers of [128 rows][128 B] (64 keys of a row per line)
+//   ring     nst stages of K then V, each NBOX boxes of [64 keys][128 B]
+//   barriers, per-stage valid-piece masks, misc
+template <int D>
+struct PfLayout {
+    static constexpr int NBOX = D * 2 / 128;           // 128-byte column boxes of a row
+    static constexpr int QBOX = PF_M * 128;
+    static constexpr int Q_BYTES = NBOX * QBOX;        // one tile
+    static constexpr int KBOX = PF_KT * 128;
+    static constexpr int KV_BYTES = NBOX * KBOX;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int P_BYTES = PF_M * 128;
+    // per tile: S x2 (64 columns each) then O (head_dim columns), 256 columns
+    static constexpr uint32_t TM_TILE = 256;
+    static constexpr uint32_t TM_COLS = PF_TILES * TM_TILE;
+    // q_full, fin, then per tile s_full x2, s_free x2, p_full x2, pv_done x2
+    static constexpr int NBAR_FIXED = 2 + 8 * PF_TILES;
+    int nst;
+    __host__ __device__ explicit PfLayout(int n) : nst(n) {}
+    __host__ __device__ size_t q(int t) const { return (size_t)t * Q_BYTES; }
+    __host__ __device__ size_t p(int t, int b) const {
+        return (size_t)PF_TILES * Q_BYTES + (size_t)(2 * t + b) * P_BYTES;
+    }
+    __host__ __device__ size_t ring(int st) const {
+        return (size_t)PF_TILES * (Q_BYTES + 2 * P_BYTES) + (size_t)st * STAGE_BYTES;
+    }
+    __host__ __device__ size_t bars() const { return ring(nst); }
+    __host__ __device__ size_t masks() const { return bars() + (size_t)(2 * nst + NBAR_FIXED) * 8; }
+    __host__ __device__ size_t misc() const { return ((masks() + 4 * (size_t)nst + 15) / 16) * 16; }
+    __host__ __device__ size_t total() const { return misc() + 64; }
+};
+
+// 3-D tiled tensor copy global -> shared (box given by the tensor map).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
+// 2-D tiled copy with the default L2 policy: K/V tiles of a sequence are read
+// by every query tile of its chunk, so they should stay in L2.
+__device__ __forceinline__ void tma_load_2d_keep(void* dst, const CUtensorMap* map, int x, int y,
+                                                 uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y),
+          "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Bounded wait that also gives up once another warp has given up.
+__device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                        int32_t* err) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if ((it & 63) == 0 && global_ns() - t0 > kWaitLimitNs) {
+            set_err(err, PA_DEV_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(PF_THREADS, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                  const __grid_constant__ CUtensorMap qmap, PrefillParams p) {
+    using LY = PfLayout<D>;
+    constexpr int QT = PF_M / G;                   // chunk tokens per query tile
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- the CTA's unit: query tiles 2u and 2u+1 of (sequence s, KV head j).
+    // The tiles of one (s, j) are neighbours in the grid, so CTAs running at
+    // the same time share K/V in L2; the later pairs (longer key ranges) of
+    // each (s, j) come first.
+    const int sj = (int)(blockIdx.x / p.npair);
+    const int u = p.npair - 1 - (int)(blockIdx.x % p.npair);
+    const int s = sj / p.Hkv, j = sj % p.Hkv;
+    const int a = __ldg(p.cu + s), e = __ldg(p.cu + s + 1);
+    int L = __ldg(p.lens + s);
+    int n = e - a;
+    bool bad = false;
+    if (a < 0 || e < a || e > p.total_q) { bad = true; n = 0; }
+    if (n > p.max_q) { bad = true; n = p.max_q; }
+    const int hi = p.mbps * p.bs;
+    if (L < 0 || L > hi) { bad = true; L = max(0, min(L, hi)); }
+    if (n > L) bad = true;
+    if (bad && u == 0 && j == 0 && tid == 0) set_err(p.err, PA_DEV_BAD_LEN);
+    int r0[PF_TILES], rows[PF_TILES], nkt[PF_TILES];
+#pragma unroll
+    for (int t = 0; t < PF_TILES; ++t) {
+        r0[t] = (PF_TILES * u + t) * QT;           // first chunk row of the tile
+        rows[t] = max(0, min(QT, n - r0[t]));
+        const int ke = rows[t] ? max(0, min(L, L - n + r0[t] + rows[t])) : 0;
+        nkt[t] = (ke + PF_KT - 1) / PF_KT;
+    }
+    if (rows[0] == 0) return;
+    const int ntile = rows[PF_TILES - 1] ? PF_TILES : 1;
+    const int last_end = ntile > 1 ? r0[1] + rows[1] : r0[0] + rows[0];
+    const int kend = max(0, min(L, L - n + last_end));   // keys read
+    const int nkt_all = (kend + PF_KT - 1) / PF_KT;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const LY ly(p.nst);
+    const int nst = p.nst;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars());
+    uint64_t* empty = full + nst;
+    uint64_t* q_full = empty + nst;
+    uint64_t* fin = q_full + 1;                    // issuer's final drain
+    // per tile t: s_full[2] (S in tensor memory), s_free[2] (S read by the 4
+    // softmax warps), p_full[2] (P written by them), pv_done[2] (PV complete)
+    auto tbar = [&](int t, int kind, int b) { return fin + 1 + t * 8 + kind * 2 + b; };
+    int* masks = reinterpret_cast<int*>(smem + ly.masks());
+    int* misc = reinterpret_cast<int*>(smem + ly.misc());
+    volatile int* abort_flag = misc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 8);
+
+    if (tid == 0) {
+        for (int k = 0; k < 2 * nst + LY::NBAR_FIXED; ++k) mbar_init(full + k, 1);
+        for (int t = 0; t < PF_TILES; ++t)
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(tbar(t, 1, b), 4);       // s_free
+                mbar_init(tbar(t, 2, b), 4);       // p_full
+            }
+        misc[0] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 9) {
+        tc::alloc(tmem_slot, LY::TM_COLS);
+        tc::relinquish();
+    }
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int PR = p.bs >= 16 ? 16 : p.bs;         // rows of one TMA box (block piece)
+    const int prl = p.bs >= 16 ? 4 : p.bs_log2;
+
+    if (warp == 8) {
+        // ================================================= TMA producer
+        if (lane == 0) {
+            prefetch_tensormap(&kmap);
+            prefetch_tensormap(&vmap);
+            mbar_arrive_expect_tx(q_full, (uint32_t)(ntile * LY::Q_BYTES));
+#pragma unroll
+            for (int t = 0; t < PF_TILES; ++t)
+                if (t < ntile)
+#pragma unroll
+                    for (int b = 0; b < LY::NBOX; ++b)
+                        tma_load_3d(smem + ly.q(t) + b * LY::QBOX, &qmap, b * 64, j * G, a + r0[t], q_full);
+        }
+        const int32_t* trow = p.tables + (size_t)s * p.mbps;
+        const int npc = PF_KT / PR;                    // block pieces per stage
+        const int nops = npc * 2 * LY::NBOX;           // TMA boxes per stage (<= 32)
+        const int piece = lane / (2 * LY::NBOX), sub = lane % (2 * LY::NBOX);
+        const int kv = sub / LY::NBOX, bx = sub % LY::NBOX;
+        int st = 0, round = 0, issued = 0;
+        for (int c = 0; c < nkt_all; ++c) {
+            if (round > 0) {
+                bool w = true;
+                if (lane == 0) w = pf_wait(empty + st, (round - 1) & 1, abort_flag, p.err);
+                if (!__shfl_sync(PF_FULL, w, 0)) break;
+            }
+            const int tok = c * PF_KT + piece * PR;
+            const bool exists = lane < nops && tok < kend;
+            const int blk = exists ? __ldg(trow + (tok >> p.bs_log2)) : -1;
+            const bool live = exists && blk >= 0 && blk < p.NB;
+            const uint32_t want = __reduce_or_sync(PF_FULL, exists ? 1u << piece : 0u);
+            const uint32_t got = __reduce_or_sync(PF_FULL, live ? 1u << piece : 0u);
+            if (lane == 0) {
+                masks[st] = (int)got;
+                if (want & ~got) set_err(p.err, PA_DEV_BAD_BLOCK);
+                if (got)
+                    mbar_arrive_expect_tx(full + st, (uint32_t)__popc(got) * 2u * PR * (D * 2));
+                else
+                    mbar_arrive(full + st);
+            }
+            __syncwarp();
+            if (live) {
+                const int y = ((blk * p.Hkv + j) << p.bs_log2) + (tok & (p.bs - 1));
+                uint8_t* dst = smem + ly.ring(st) + kv * LY::KV_BYTES + bx * LY::KBOX + piece * PR * 128;
+                tma_load_2d_keep(dst, kv ? &vmap : &kmap, bx * 64, y, full + st);
+            }
+            ++issued;
+            if (++st == nst) { st = 0; ++round; }
+        }
+        // no copy of this CTA may still be landing when it exits
+        if (lane == 0) {
+            for (int g = max(0, issued - nst); g < issued; ++g) mbar_wait(full + g % nst, (g / nst) & 1);
+            mbar_wait(q_full, 0);
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ================================================= MMA issuer (one thread)
+        // Per stage c: S of both tiles, then PV of both tiles for stage c - 1,
+        // so the tensor core computes while the softmax groups work.
+        if (lane == 0) {
+            constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, PF_M, PF_KT);
+            constexpr uint32_t ID_O = tc::idesc_f16<T>(false, true, PF_M, D);
+            bool ok = pf_wait(q_full, 0, abort_flag, p.err);
+            for (int c = 0; ok && c <= nkt_all; ++c) {
+                if (c < nkt_all) {
+                    const int st = c % nst, b = c & 1;
+                    ok = pf_wait(full + st, (c / nst) & 1, abort_flag, p.err);
+                    const uint64_t kd = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
+#pragma unroll
+                    for (int t = 0; t < PF_TILES; ++t) {
+                        if (!ok || t >= ntile || c >= nkt[t]) continue;
+                        if (c >= 2) ok = pf_wait(tbar(t, 1, b), ((c - 2) >> 1) & 1, abort_flag, p.err);
+                        if (!ok) break;
+                        tc::fence_after();
+                        const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
+                        const uint32_t sd = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * b);
+#pragma unroll
+                        for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
+                            tc::mma_ss(sd, qd + (uint64_t)((k >> 2) * (LY::QBOX >> 4) + (k & 3) * 2),
+                                       kd + (uint64_t)((k >> 2) * (LY::KBOX >> 4) + (k & 3) * 2), ID_S,
+                                       k > 0 ? 1u : 0u);
+                        tc::commit(tbar(t, 0, b));
+                    }
+                    if (!ok) break;
+                }
+                if (c >= 1) {
+                    const int m = c - 1, bm = m & 1, stm = m % nst;
+                    const uint64_t vd =
+                        tc::sdesc_sw128(smem_u32(smem + ly.ring(stm) + LY::KV_BYTES), LY::KBOX, 1024);
+#pragma unroll
+                    for (int t = 0; t < PF_TILES; ++t) {
+                        if (!ok || t >= ntile || m >= nkt[t]) continue;
+                        ok = pf_wait(tbar(t, 2, bm), (m >> 1) & 1, abort_flag, p.err);
+                        if (!ok) break;
+                        tc::fence_after();
+                        const uint64_t pd = tc::sdesc_sw128(smem_u32(smem + ly.p(t, bm)), 16, 1024);
+                        const uint32_t od = tmem + (uint32_t)(t * LY::TM_TILE + 2 * PF_KT);
+#pragma unroll
+                        for (int kk = 0; kk < PF_KT / 16; ++kk)
+                            tc::mma_ss(od, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), ID_O,
+                                       (m > 0 || kk > 0) ? 1u : 0u);
+                        tc::commit(tbar(t, 3, bm));
+                    }
+                    if (!ok) break;
+                    tc::commit(empty + stm);           // the stage slot may be refilled
+                }
+            }
+            // every MMA of this CTA completes before tensor memory is freed
+            tc::commit(fin);
+            mbar_wait(fin, 0);
+        }
+        __syncwarp();
+    } else {
+        // ================================================= softmax + epilogue (row of tile t)
+        const int t = warp >> 2;
+        const int r = tid & 127;
+        const int my_nkt = t == 0 ? nkt[0] : (ntile > 1 ? nkt[1] : 0);
+        const int my_r0 = t == 0 ? r0[0] : r0[1];
+        const int my_rows = t == 0 ? rows[0] : rows[1];
+        const int crow = my_r0 + r / G;                // chunk row of this thread's query
+        const int g = r % G;
+        const int pos = L - n + crow;                  // keys 0..pos are visible
+        const uint32_t lq = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tS = tmem + (uint32_t)(t * LY::TM_TILE), tO = tS + 2 * PF_KT;
+        const float sl = p.scale_log2e;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int c = 0; c < my_nkt; ++c) {
+            const int b = c & 1, st = c % nst;
+            ok = __all_sync(PF_FULL, pf_wait(tbar(t, 0, b), (c >> 1) & 1, abort_flag, p.err) &&
+                                         pf_wait(full + st, (c / nst) & 1, abort_flag, p.err));
+            if (!ok) break;
+            tc::fence_after();
+            const uint32_t vmask = (uint32_t)masks[st];
+            // keys of this stage the row may see: the first `lim` by position,
+            // and only those of pieces whose block was loaded
+            const int lim = pos - c * PF_KT + 1;
+            const bool whole = __all_sync(PF_FULL, lim >= PF_KT && vmask == (1u << (PF_KT / PR)) - 1u);
+            const uint32_t tSb = tS + (uint32_t)(PF_KT * b) + lq;
+            // pass 1: the row maximum of the raw scores (the scale is positive)
+            float mraw = -INFINITY;
+            if (whole) {                               // warp-uniform: no key is hidden
+#pragma unroll
+                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
+                    uint32_t v[16];
+                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
+                }
+            } else {
+#pragma unroll
+                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
+                    uint32_t v[16];
+                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int k = 16 * q4 + i;
+                        if (k < lim && ((vmask >> (k >> prl)) & 1u)) mraw = fmaxf(mraw, __uint_as_float(v[i]));
+                    }
+                }
+            }
+            const float mt = mraw * sl;
+            const bool need = mt > m_ref + kPfRescaleLog2;
+            if (__any_sync(PF_FULL, need)) {
+                if (c > 0) {
+                    // O must hold every earlier PV before it is rescaled
+                    ok = __all_sync(PF_FULL, pf_wait(tbar(t, 3, (c - 1) & 1), ((c - 1) >> 1) & 1,
+                                                     abort_flag, p.err));
+                    if (!ok) break;
+                    tc::fence_after();
+                    const float f = need ? exp2f(m_ref - mt) : 1.f;
+#pragma unroll
+                    for (int q4 = 0; q4 < D / 16; ++q4) {
+                        uint32_t v[16];
+                        tc::ld16(tO + (uint32_t)(16 * q4) + lq, v);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+                        tc::st16(tO + (uint32_t)(16 * q4) + lq, v);
+                    }
+                    l *= f;
+                }
+                if (need) m_ref = mt;
+            }
+            if (c >= 2) {
+                // P buffer b was read by the PV two stages back
+                ok = __all_sync(PF_FULL, pf_wait(tbar(t, 3, b), ((c - 2) >> 1) & 1, abort_flag, p.err));
+                if (!ok) break;
+            }
+            // pass 2: P = exp2(s * scale * log2 e - m), rounded, into the swizzled P rows
+            const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
+            uint8_t* prow = smem + ly.p(t, b) + r * 128;
+            float lsum = 0.f;
+            auto put16 = [&](int q4, const uint32_t (&w)[8]) {
+                const int q8 = 2 * q4;
+                *reinterpret_cast<uint4*>(prow + ((q8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(prow + (((q8 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
+            };
+            if (whole) {
+#pragma unroll
+                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
+                    uint32_t v[16], w[8];
+                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        w[i] = pack2<T>(exp2f(fmaf(__uint_as_float(v[2 * i]), sl, nmr)),
+                                        exp2f(fmaf(__uint_as_float(v[2 * i + 1]), sl, nmr)));
+                        float rr[2];
+                        Unpack<T>::run(w[i], rr);
+                        lsum += rr[0] + rr[1];
+                    }
+                    put16(q4, w);
+                }
+            } else {
+#pragma unroll
+                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
+                    uint32_t v[16], w[8];
+                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int k0 = 16 * q4 + 2 * i;
+                        const bool vis0 = k0 < lim && ((vmask >> (k0 >> prl)) & 1u);
+                        const bool vis1 = k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u);
+                        const float p0 = vis0 ? exp2f(fmaf(__uint_as_float(v[2 * i]), sl, nmr)) : 0.f;
+                        const float p1 = vis1 ? exp2f(fmaf(__uint_as_float(v[2 * i + 1]), sl, nmr)) : 0.f;
+                        w[i] = pack2<T>(p0, p1);
+                        float rr[2];
+                        Unpack<T>::run(w[i], rr);
+                        lsum += rr[0] + rr[1];
+                    }
+                    put16(q4, w);
+                }
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tbar(t, 1, b));    // S buffer b may be rewritten
+            l += lsum;
+            if (r < PF_KT) {
+                // rows past the CTA's key range or of a skipped block: zero V
+                // (both groups write the same zeros)
+                const int key = c * PF_KT + r;
+                if (key >= kend || !((vmask >> (r >> prl)) & 1u)) {
+                    uint8_t* vrow = smem + ly.ring(st) + LY::KV_BYTES + r * 128;
+#pragma unroll
+                    for (int bx = 0; bx < LY::NBOX; ++bx)
+#pragma unroll
+                        for (int q8 = 0; q8 < 8; ++q8)
+                            *reinterpret_cast<uint4*>(vrow + bx * LY::KBOX + q8 * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tbar(t, 2, b));
+        }
+        if (ok && my_nkt > 0)
+            ok = __all_sync(PF_FULL, pf_wait(tbar(t, 3, (my_nkt - 1) & 1), ((my_nkt - 1) >> 1) & 1,
+                                             abort_flag, p.err));
+        tc::fence_after();
+        if (ok && t < ntile) {
+            const bool store = r / G < my_rows;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            T* dst = reinterpret_cast<T*>(p.out) + ((size_t)(a + crow) * p.Hq + (size_t)j * G + g) * D;
+#pragma unroll
+            for (int q4 = 0; q4 < D / 16; ++q4) {
+                uint32_t v[16];
+                if (my_nkt > 0) {
+                    tc::ld16(tO + (uint32_t)(16 * q4) + lq, v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0u;
+                }
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    w[i] = pack2<T>(__uint_as_float(v[2 * i]) * inv, __uint_as_float(v[2 * i + 1]) * inv);
+                if (store) {
+                    uint4* o4 = reinterpret_cast<uint4*>(dst + 16 * q4);
+                    o4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                    o4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+                }
+            }
+        }
+    }
+
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    if (warp == 9) tc::dealloc(tmem, LY::TM_COLS);
+}
+
+// ------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 pf_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// Tensor map of `rank` dims (innermost first), 128-byte inner box, 128B swizzle.
+int pf_map(CUtensorMap* map, const void* base, pa_dtype dt, int rank, const cuuint64_t* dims,
+           const cuuint64_t* strides, const cuuint32_t* box) {
+    auto fn = pf_encode_fn();
+    if (!fn) return PA_ERR_CUDA;
+    const CUtensorMapDataType t =
+        dt == PA_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, t, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+struct PfLaunch {
+    CUtensorMap kmap, vmap, qmap;
+    PrefillParams p;
+    dim3 grid;
+    cudaStream_t stream;
+};
+
+template <typename T, int D, int G>
+int pf_run(PfLaunch& L) {
+    using LY = PfLayout<D>;
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return PA_ERR_CUDA;
+    int nst = PF_MAX_STAGES;
+    while (nst > 2 && LY(nst).total() + 1024 > (size_t)optin) --nst;
+    const size_t smem = LY(nst).total() + 1024;
+    if (smem > (size_t)optin) return PA_ERR_UNSUPPORTED;
+    L.p.nst = nst;
+    auto kern = prefill_tc_kernel<T, D, G>;
+    static bool attr_set[64] = {};
+    static std::mutex mu;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!attr_set[dev & 63]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) !=
+                cudaSuccess)
+                return PA_ERR_CUDA;
+            attr_set[dev & 63] = true;
+        }
+    }
+    kern<<<L.grid, PF_THREADS, smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+template <typename T, int D>
+int pf_dispatch_g(PfLaunch& L, int G) {
+    switch (G) {
+        case 1: return pf_run<T, D, 1>(L);
+        case 2: return pf_run<T, D, 2>(L);
+        case 4: return pf_run<T, D, 4>(L);
+        case 8: return pf_run<T, D, 8>(L);
+        default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+int pf_dispatch(PfLaunch& L, int D, int G) {
+    return D == 64 ? pf_dispatch_g<T, 64>(L, G) : pf_dispatch_g<T, 128>(L, G);
+}
+
+bool pf_aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+}  // namespace
+}  // namespace pa
+
+extern "C" {
+
+int pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
+               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+               const int32_t* cu_seqlens_q, int num_seqs, int total_q, int max_query_len,
+               int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               float scale, pa_dtype dtype, int32_t* err_flag, void* stream) {
+    using namespace pa;
+    if (num_seqs == 0 || total_q == 0) return PA_OK;
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
+        !cu_seqlens_q)
+        return PA_ERR_INVALID;
+    if (!(scale > 0.f) || !(scale < INFINITY)) return PA_ERR_INVALID;
+    if (num_seqs < 0 || total_q < 0 || max_query_len <= 0 || num_q_heads <= 0 ||
+        num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID;
+    if (dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+    if (dtype != PA_F16 && dtype != PA_BF16) return PA_ERR_INVALID;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
+        block_size != 128)
+        return PA_ERR_UNSUPPORTED;
+    if (!pf_aligned16(out) || !pf_aligned16(query) || !pf_aligned16(key_cache) ||
+        !pf_aligned16(value_cache))
+        return PA_ERR_INVALID;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (rows >= (int64_t(1) << 31) || (int64_t)total_q * num_q_heads >= (int64_t(1) << 31))
+        return PA_ERR_UNSUPPORTED;
+    const int QT = PF_M / G;
+    const int nqt = (max_query_len + QT - 1) / QT;
+    const int npair = (nqt + PF_TILES - 1) / PF_TILES;
+    const int64_t grid = (int64_t)npair * num_seqs * num_kv_heads;
+    if (grid >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+
+    static thread_local PfLaunch L;
+    const cuuint64_t esz = 2;
+    {
+        const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+        const cuuint64_t strides[1] = {(cuuint64_t)head_dim * esz};
+        const cuuint32_t box[2] = {64, (cuuint32_t)std::min(block_size, 16)};
+        int st = pf_map(&L.kmap, key_cache, dtype, 2, dims, strides, box);
+        if (st == PA_OK) st = pf_map(&L.vmap, value_cache, dtype, 2, dims, strides, box);
+        if (st != PA_OK) return st;
+    }
+    {
+        // queries as [total_q][Hq][D]: a box is 64 columns x the G heads of one
+        // KV head x QT chunk tokens = 128 rows of 128 bytes
+        const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)num_q_heads, (cuuint64_t)total_q};
+        const cuuint64_t strides[2] = {(cuuint64_t)head_dim * esz,
+                                       (cuuint64_t)num_q_heads * head_dim * esz};
+        const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)QT};
+        int st = pf_map(&L.qmap, query, dtype, 3, dims, strides, box);
+        if (st != PA_OK) return st;
+    }
+    PrefillParams& p = L.p;
+    p.out = out;
+    p.q = query;
+    p.tables = block_tables;
+    p.lens = context_lens;
+    p.cu = cu_seqlens_q;
+    p.S = num_seqs;
+    p.total_q = total_q;
+    p.max_q = max_query_len;
+    p.npair = npair;
+    p.Hq = num_q_heads;
+    p.Hkv = num_kv_heads;
+    p.mbps = max_blocks_per_seq;
+    p.NB = num_blocks;
+    p.bs = block_size;
+    p.bs_log2 = __builtin_ctz((unsigned)block_size);
+    p.scale_log2e = scale * 1.4426950408889634f;
+    p.err = err_flag;
+    L.grid = dim3((unsigned)grid);
+    L.stream = (cudaStream_t)stream;
+    return dtype == PA_F16 ? pf_dispatch<__half>(L, head_dim, G)
+                           : pf_dispatch<__nv_bfloat16>(L, head_dim, G);
+}
+
+}  // extern "C"

@@ -155,3 +155,63 @@ def oracle_sampled(w, rec, k, pairs):
 
 def scale_of(d):
     return 1.0 / math.sqrt(d)
+
+
+class GpuPrefill:
+    """A ``workloads.PrefillBatch`` through the CUDA path: the library's
+    manager hands out the slots (same FIFO pool as the oracle's), the tokens
+    before each chunk are written with pa_reshape_and_cache, then the chunks'
+    (the step), then pa_prefill attends.  ``fill``: value of every cache
+    element no token writes (NaN checks that unwritten slots never leak)."""
+
+    def __init__(self, b, device="cuda", fill=0.0):
+        self.b = b
+        td = b.torch_dtype
+        self.alloc = pa.BlockAllocator(b.num_blocks, b.free_order)
+        self.mgr = pa.BlockManager(self.alloc, b.block_size)
+        shape = (b.num_blocks, b.num_kv_heads, b.block_size, b.head_dim)
+        self.kc = torch.full(shape, fill, dtype=td, device=device)
+        self.vc = torch.full(shape, fill, dtype=td, device=device)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        S = len(b.context_lens)
+        ctx_s, chunk_s, ctx_k, ctx_v, ch_k, ch_v = [], [], [], [], [], []
+        for s, (L, n) in enumerate(zip(b.context_lens, b.query_lens)):
+            self.mgr.add_seq(s)
+            slots = self.mgr.append(s, L)[0] if L else torch.zeros(0, dtype=torch.int64)
+            ctx_s.append(slots[:L - n])
+            chunk_s.append(slots[L - n:])
+            ctx_k.append(b.k[s][:L - n])
+            ctx_v.append(b.v[s][:L - n])
+            ch_k.append(b.k[s][L - n:])
+            ch_v.append(b.v[s][L - n:])
+        self.ctx_slots = torch.cat(ctx_s)
+        self.chunk_slots = torch.cat(chunk_s)
+        if self.ctx_slots.numel():
+            pa.pa_reshape_and_cache(torch.cat(ctx_k).to(device), torch.cat(ctx_v).to(device),
+                                    self.kc, self.vc, self.ctx_slots.to(device), err_flag=self.err)
+        self.chunk_k = torch.cat(ch_k).to(device)
+        self.chunk_v = torch.cat(ch_v).to(device)
+        self.chunk_slots_d = self.chunk_slots.to(device)
+        self.mb = max(1, max(-(-L // b.block_size) for L in b.context_lens))
+        tab, lens = self.mgr.block_tables(list(range(S)), self.mb)
+        self.tab_h, self.lens_h = tab, lens
+        self.tab, self.lens = tab.to(device), lens.to(device)
+        self.cu = torch.tensor(b.query_offsets, dtype=torch.int32, device=device)
+        self.q = b.q.to(device)
+        self.out = torch.full_like(self.q, float("nan"))
+        self.max_q = max(1, max(b.query_lens))
+
+    def write_chunks(self):
+        if self.chunk_slots.numel():
+            pa.pa_reshape_and_cache(self.chunk_k, self.chunk_v, self.kc, self.vc,
+                                    self.chunk_slots_d, err_flag=self.err)
+
+    def attend(self):
+        pa.pa_prefill(self.out, self.q, self.kc, self.vc, self.tab, self.lens, self.cu, self.max_q,
+                      self.b.scale, err_flag=self.err)
+
+    def step(self):
+        self.write_chunks()
+        self.attend()
+        torch.cuda.synchronize()
+        return self.out

@@ -1,0 +1,151 @@
+"""Paged prefill attention (pa_prefill, tcgen05) against the oracle.
+
+Each batch is replayed twice from the same seeded inputs: through the oracle
+(its own manager, cache writes and float64 causal attention) and through the
+CUDA path (the library's manager, pa_reshape_and_cache, pa_prefill).  The
+block tables must be identical; the outputs must agree within the 16-bit
+tolerance (the kernel rounds P to the input type, accumulates in fp32 and
+rounds the output).
+
+Chunk shapes cover: a whole short prompt, a chunk inside a long context, a
+multi-tile prompt with a ragged last query tile, a one-row chunk (a decode
+step), an empty chunk, and a chunk whose key range ends inside a block.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.harness import TOL, GpuPrefill, check_close, out_f64
+
+pa = pytest.importorskip("paged_kv_cache_426_b200")
+
+pytestmark = pytest.mark.gpu
+
+LENS = [5, 40, 150, 300, 129, 64, 1000, 77]
+QLENS = [5, 17, 150, 1, 64, 0, 333, 77]
+
+SHAPES = [   # dtype, hq, hkv, d, bs
+    ("bf16", 8, 2, 128, 16),
+    ("f16", 4, 4, 64, 8),
+    ("bf16", 16, 2, 128, 32),
+    ("f16", 4, 2, 128, 64),
+    ("bf16", 8, 8, 128, 128),
+    ("f16", 8, 1, 64, 16),
+]
+
+
+def _run(b, fill=0.0):
+    ref = oracle.run_prefill(b)
+    g = GpuPrefill(b, fill=fill)
+    assert np.array_equal(g.tab_h.numpy(), ref.block_tables)
+    assert np.array_equal(g.lens_h.numpy(), ref.context_lens)
+    out = g.step()
+    assert int(g.err.item()) == 0
+    return out_f64(out, b.dtype), ref.out, g
+
+
+@pytest.mark.parametrize("dtype,hq,hkv,d,bs", SHAPES)
+def test_prefill_matches_oracle(dtype, hq, hkv, d, bs):
+    b = workloads.prefill_custom(dtype, LENS, QLENS, hq, hkv, d, bs, seed=hq * 131 + d + bs)
+    got, ref, _ = _run(b)
+    check_close(got, ref, dtype, f"prefill {dtype} {hq}/{hkv} d{d} bs{bs}")
+
+
+def test_unwritten_slots_never_leak():
+    """Every cache element no token wrote is NaN; keys past a chunk's range
+    and the tail of its last block must still get weight 0 and a finite V."""
+    b = workloads.prefill_custom("bf16", [17, 65, 200, 31], [17, 3, 129, 31], 8, 2, 128, 16,
+                                 seed=5, extra_blocks=4)
+    got, ref, _ = _run(b, fill=float("nan"))
+    assert np.isfinite(got).all()
+    check_close(got, ref, "bf16", "NaN-filled pool")
+
+
+def test_one_row_chunks_equal_decode():
+    """n = 1 per sequence: pa_prefill and pa_decode read the same cache and
+    must agree with the oracle (and hence with each other)."""
+    lens = [1, 16, 17, 300, 1025]
+    b = workloads.prefill_custom("bf16", lens, [1] * len(lens), 32, 8, 128, 16, seed=9)
+    got, ref, g = _run(b)
+    check_close(got, ref, "bf16", "one-row chunks")
+    ws = pa.alloc_workspace(len(lens), 32, 8, 128, max(lens), 0, "cuda")
+    dec = torch.empty_like(g.q)
+    pa.pa_decode(dec, g.q, g.kc, g.vc, g.tab, g.lens, max(lens), b.scale, workspace=ws,
+                 err_flag=g.err)
+    torch.cuda.synchronize()
+    check_close(out_f64(dec, "bf16"), ref, "bf16", "decode on the same cache")
+
+
+@pytest.mark.parametrize("name", ["prefill_gqa8b_bf16", "prefill_mha7b_f16"])
+def test_full_size_sampled_rows(name):
+    """The benchmark's batches at full size: every output row is finite, and
+    sampled rows (first, last and random rows of random chunks, all heads)
+    match the oracle computed row by row."""
+    b = workloads.PREFILL_BUILDERS[name]()
+    g = GpuPrefill(b)
+    out = g.step()
+    assert int(g.err.item()) == 0
+    got = out_f64(out, b.dtype)
+    assert np.isfinite(got).all()
+    rng = np.random.default_rng(17)
+    S = len(b.context_lens)
+    rows = {}
+    for s in rng.choice(S, size=min(S, 6), replace=False):
+        n = b.query_lens[s]
+        rows[int(s)] = sorted({0, n - 1, *rng.integers(0, n, size=3).tolist()})
+    ref = oracle.run_prefill(b, rows=rows)
+    assert np.array_equal(g.tab_h.numpy(), ref.block_tables)
+    cu = b.query_offsets
+    for s, rs in rows.items():
+        idx = [cu[s] + r for r in rs]
+        check_close(got[idx], ref.out[idx], b.dtype, f"{name} seq {s} rows {rs}")
+
+
+def test_bad_block_and_bad_len_are_reported():
+    b = workloads.prefill_custom("f16", [100, 50], [30, 50], 4, 2, 64, 16, seed=3)
+    g = GpuPrefill(b)
+    g.write_chunks()
+    tab = g.tab.clone()
+    tab[0, 2] = b.num_blocks + 7             # a block the chunk reads
+    pa.pa_prefill(g.out, g.q, g.kc, g.vc, tab, g.lens, g.cu, g.max_q, b.scale, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == pa.PA_DEV_BAD_BLOCK
+    g.err.zero_()
+    lens = g.lens.clone()
+    lens[1] = 20                              # shorter than its 50-row chunk
+    pa.pa_prefill(g.out, g.q, g.kc, g.vc, g.tab, lens, g.cu, g.max_q, b.scale, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == pa.PA_DEV_BAD_LEN
+    g.err.zero_()
+    g.attend()                                # the context is still usable
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == 0
+    check_close(out_f64(g.out, "f16"), oracle.run_prefill(b).out, "f16", "after bad calls")
+
+
+def test_rejected_shapes_and_empty_batch():
+    b = workloads.prefill_custom("bf16", [20], [20], 4, 2, 128, 16, seed=1)
+    g = GpuPrefill(b)
+    with pytest.raises(pa.PAError) as e:     # fp32 has no tensor-core path
+        pa.pa_prefill(g.out.float(), g.q.float(), g.kc.float(), g.vc.float(), g.tab, g.lens,
+                      g.cu, g.max_q, b.scale)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+    q3 = torch.zeros((20, 6, 128), dtype=torch.bfloat16, device="cuda")   # G = 3
+    with pytest.raises(pa.PAError) as e:
+        pa.pa_prefill(torch.empty_like(q3), q3, g.kc, g.vc, g.tab, g.lens, g.cu, g.max_q, b.scale)
+    assert e.value.status == pa.PA_ERR_UNSUPPORTED
+    empty = torch.zeros((0, 4, 128), dtype=torch.bfloat16, device="cuda")
+    cu0 = torch.zeros(2, dtype=torch.int32, device="cuda")
+    pa.pa_prefill(empty, empty, g.kc, g.vc, g.tab, g.lens, cu0, 1, b.scale)   # nothing to do
+
+
+def test_repeat_is_bit_identical():
+    b = workloads.prefill_custom("bf16", LENS, QLENS, 8, 2, 128, 16, seed=21)
+    g = GpuPrefill(b)
+    a = g.step().clone()
+    g.attend()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), g.out.view(torch.int16))
+    assert TOL["bf16"]["atol"] > 0

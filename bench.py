@@ -292,7 +292,7 @@ def run_prefill_bench(args):
     value = flop * args.steps / (span_ms * 1e-3) / 1e12
     achieved = flop / (pf_ms * 1e-3) / 1e12
     peak, kind = tensor_peak()
-    prof = profiled_fields(os.path.join(ROOT, "profiles", f"prefill_{b.name}.md"))
+    prof = profiled_fields(os.path.join(ROOT, "profiles", f"{b.name}.md"))
     traffic = int(prof["traffic_bytes_per_launch"]) if prof else None
     T = sum(b.query_lens)
     res = {

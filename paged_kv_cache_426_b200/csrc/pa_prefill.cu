@@ -131,6 +131,31 @@ __device__ __forceinline__ bool pf_wait(uint64_t* bar, uint32_t parity, volatile
     }
 }
 
+// 32 columns of this warp's tensor-memory lane quarter (32x32b shape: thread
+// t reads lane 32 * (warp % 4) + t), waiting for the copy in the same asm.
+__device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 2^x by the PTX ex2.approx instruction with subnormal results flushed to
+// zero: softmax weights below 2^-126 are zero after rounding to 16 bits
+// anyway (the sum they would add is far below the output's precision).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -347,22 +372,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             const uint32_t tSb = tS + (uint32_t)(PF_KT * b) + lq;
             // pass 1: the row maximum of the raw scores (the scale is positive)
             float mraw = -INFINITY;
-            if (whole) {                               // warp-uniform: no key is hidden
 #pragma unroll
-                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
-                    uint32_t v[16];
-                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+            for (int h = 0; h < PF_KT / 32; ++h) {
+                uint32_t v[32];
+                tm_ld32(tSb + (uint32_t)(32 * h), v);
+                if (whole) {                           // warp-uniform: no key is hidden
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
-                }
-            } else {
+                    for (int i = 0; i < 32; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
+                } else {
 #pragma unroll
-                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
-                    uint32_t v[16];
-                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int k = 16 * q4 + i;
+                    for (int i = 0; i < 32; ++i) {
+                        const int k = 32 * h + i;
                         if (k < lim && ((vmask >> (k >> prl)) & 1u)) mraw = fmaxf(mraw, __uint_as_float(v[i]));
                     }
                 }
@@ -398,45 +418,38 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
             uint8_t* prow = smem + ly.p(t, b) + r * 128;
             float lsum = 0.f;
-            auto put16 = [&](int q4, const uint32_t (&w)[8]) {
-                const int q8 = 2 * q4;
-                *reinterpret_cast<uint4*>(prow + ((q8 ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(prow + (((q8 + 1) ^ (r & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
-            };
-            if (whole) {
+            // packed fp32x2: z = s * scale * log2 e - m for two keys at once; the
+            // row sum adds the weights as rounded to T (what the PV MMA multiplies)
+            const uint64_t SL2 = f2_pack(sl, sl), NM2 = f2_pack(nmr, nmr), ONE2 = f2_pack(1.f, 1.f);
+            uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
-                    uint32_t v[16], w[8];
-                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
+            for (int h = 0; h < PF_KT / 32; ++h) {
+                uint32_t v[32], w[16];
+                tm_ld32(tSb + (uint32_t)(32 * h), v);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        w[i] = pack2<T>(exp2f(fmaf(__uint_as_float(v[2 * i]), sl, nmr)),
-                                        exp2f(fmaf(__uint_as_float(v[2 * i + 1]), sl, nmr)));
-                        float rr[2];
-                        Unpack<T>::run(w[i], rr);
-                        lsum += rr[0] + rr[1];
+                for (int i = 0; i < 16; ++i) {
+                    float z0, z1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
+                                     SL2, NM2), z0, z1);
+                    if (!whole) {
+                        const int k0 = 32 * h + 2 * i;
+                        if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
+                        if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                     }
-                    put16(q4, w);
+                    w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
+                    acc2 = f2_fma(Pairs<T>::from_word(w[i]), ONE2, acc2);
                 }
-            } else {
 #pragma unroll
-                for (int q4 = 0; q4 < PF_KT / 16; ++q4) {
-                    uint32_t v[16], w[8];
-                    tc::ld16(tSb + (uint32_t)(16 * q4), v);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int k0 = 16 * q4 + 2 * i;
-                        const bool vis0 = k0 < lim && ((vmask >> (k0 >> prl)) & 1u);
-                        const bool vis1 = k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u);
-                        const float p0 = vis0 ? exp2f(fmaf(__uint_as_float(v[2 * i]), sl, nmr)) : 0.f;
-                        const float p1 = vis1 ? exp2f(fmaf(__uint_as_float(v[2 * i + 1]), sl, nmr)) : 0.f;
-                        w[i] = pack2<T>(p0, p1);
-                        float rr[2];
-                        Unpack<T>::run(w[i], rr);
-                        lsum += rr[0] + rr[1];
-                    }
-                    put16(q4, w);
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int q8 = 4 * h + qq;
+                    *reinterpret_cast<uint4*>(prow + ((q8 ^ (r & 7)) << 4)) =
+                        make_uint4(w[4 * qq], w[4 * qq + 1], w[4 * qq + 2], w[4 * qq + 3]);
                 }
+            }
+            {
+                float a0, a1;
+                f2_unpack(acc2, a0, a1);
+                lsum = a0 + a1;
             }
             tc::fence_before();
             __syncwarp();

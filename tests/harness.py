@@ -52,7 +52,7 @@ def check_close(gpu: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     return float(err.max()), float(rel.max())
 
 
-class GpuRun:
+class CudaPathRun:
     """The CUDA path driven through a workload's script."""
 
     def __init__(self, w, rec: oracle.OracleRun, *, partition_size=None, device="cuda",

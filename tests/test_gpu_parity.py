@@ -19,7 +19,7 @@ import torch
 
 import oracle
 import workloads
-from tests.harness import (GpuRun, check_close, oracle_sampled, out_f64, sample_pairs,
+from tests.harness import (CudaPathRun, check_close, oracle_sampled, out_f64, sample_pairs,
                            to_torch_storage)
 
 pytestmark = pytest.mark.gpu
@@ -43,7 +43,7 @@ def run_full_compare(w, partition_size=None, steps=None):
     if _current[0] == "tensor" and w.dtype == "f32":
         pytest.skip("the tensor-core engine takes 16-bit types")
     rec = oracle.run(w, keep_prefill_cache=True, steps=steps)
-    g = GpuRun(w, rec, partition_size=partition_size)
+    g = CudaPathRun(w, rec, partition_size=partition_size)
     g.replay_prefill()
     errs = []
     for k in range(len(rec.steps)):
@@ -113,7 +113,7 @@ def _decode_outputs(w, P, engine_id=0):
     prev = pa.pa_set_decode_engine(engine_id)
     try:
         rec = oracle.run(w, keep_prefill_cache=True, decode=False)
-        g = GpuRun(w, rec, partition_size=P)
+        g = CudaPathRun(w, rec, partition_size=P)
         g.replay_prefill()
         return [g.step(k).cpu() for k in range(len(rec.steps))], rec
     finally:
@@ -244,7 +244,7 @@ def test_zero_and_one_token():
 def test_max_context_fills_table_exactly():
     w = workloads.custom("f16", [256, 255], 8, 8, 128, 16, seed=11, partition_size=64)
     rec = oracle.run(w, keep_prefill_cache=True)
-    g = GpuRun(w, rec, max_blocks=16)            # 256 tokens = 16 blocks exactly
+    g = CudaPathRun(w, rec, max_blocks=16)            # 256 tokens = 16 blocks exactly
     g.replay_prefill()
     out = g.step(0)
     check_close(out_f64(out, "f16"), rec.steps[0].out, "f16", "full table")
@@ -403,7 +403,7 @@ def test_full_size_sampled(name, kw):
     and the whole caches bit-exact after the last step."""
     w = workloads.make(name, **kw)
     rec = oracle.run(w, keep_prefill_cache=True, decode=False)
-    g = GpuRun(w, rec)
+    g = CudaPathRun(w, rec)
     g.replay_prefill()
     S, Hq = rec.steps[0].context_lens.shape[0], w.num_q_heads
     for k in range(len(rec.steps)):
@@ -487,7 +487,7 @@ def test_bounded_wait_reports_timeout(engine_id):
     import time
     w = workloads.gqa8b_bf16(num_seqs=6)
     rec = oracle.run(w, keep_prefill_cache=True)
-    g = GpuRun(w, rec, partition_size=512)
+    g = CudaPathRun(w, rec, partition_size=512)
     g.replay_prefill()
     st = rec.steps[0]
     slots, _ = g.mgr.append_step(st.seqs)

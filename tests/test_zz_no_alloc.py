@@ -20,7 +20,7 @@ import torch
 
 import oracle
 import workloads
-from tests.harness import GpuRun, check_close, out_f64
+from tests.harness import CudaPathRun, check_close, out_f64
 
 pytestmark = pytest.mark.gpu
 pa = pytest.importorskip("paged_kv_cache_426_b200")
@@ -45,7 +45,7 @@ def test_static_matches_workspace_two_calls(name, P):
     else:
         w = workloads.gqa8b_bf16(num_seqs=12, steps=2)
     rec = oracle.run(w, keep_prefill_cache=True)
-    g = GpuRun(w, rec, partition_size=P)
+    g = CudaPathRun(w, rec, partition_size=P)
     g.replay_prefill()
     for k in range(2):                       # two calls in a row, on successive steps
         ref_out = g.step(k)                  # pa_decode with a caller workspace

@@ -65,6 +65,36 @@ def test_bad_arguments_rejected_before_launch():
     assert L.pa_copy_blocks(None, None, None, 0, 2, 128, 16, 8, 1, None, None) == pa.PA_OK
 
 
+def test_prefill_bad_arguments_rejected_before_launch():
+    """pa_prefill validates everything on the host before touching the
+    device: arguments (args order: out, query, key_cache, value_cache,
+    block_tables, max_blocks_per_seq, context_lens, cu_seqlens_q, num_seqs,
+    total_q, max_query_len, Hq, Hkv, head_dim, block_size, num_blocks, scale,
+    dtype, err_flag, stream)."""
+    L = pa.lib
+    f = 1 << 20                          # aligned, never dereferenced: validation fails first
+    ok = dict(mbps=4, S=2, T=8, maxq=8, hq=8, hkv=2, d=128, bs=16, nb=8, scale=0.125, dt=2)
+
+    def call(ptr=f, **kw):
+        a = dict(ok, **kw)
+        return L.pa_prefill(ptr, f, f, f, f, a["mbps"], f, f, a["S"], a["T"], a["maxq"], a["hq"],
+                            a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["dt"], None, None)
+
+    assert call(S=0) == pa.PA_OK and call(T=0) == pa.PA_OK         # nothing to do
+    assert call(ptr=None) == pa.PA_ERR_INVALID
+    assert call(ptr=f + 8) == pa.PA_ERR_INVALID                    # not 16-byte aligned
+    assert call(dt=0) == pa.PA_ERR_UNSUPPORTED                     # fp32: no tensor-core path
+    assert call(dt=7) == pa.PA_ERR_INVALID
+    assert call(d=96) == pa.PA_ERR_UNSUPPORTED
+    assert call(hq=6) == pa.PA_ERR_UNSUPPORTED                     # G = 3
+    assert call(hq=7) == pa.PA_ERR_INVALID                         # not a multiple of Hkv
+    assert call(bs=24) == pa.PA_ERR_UNSUPPORTED
+    assert call(maxq=0) == pa.PA_ERR_INVALID
+    assert call(scale=0.0) == pa.PA_ERR_INVALID and call(scale=-1.0) == pa.PA_ERR_INVALID
+    assert call(scale=float("inf")) == pa.PA_ERR_INVALID
+    assert call(nb=0) == pa.PA_ERR_INVALID and call(mbps=0) == pa.PA_ERR_INVALID
+
+
 def test_workspace_size_formula():
     # the scheduler header only when nothing is split
     n0 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 0)

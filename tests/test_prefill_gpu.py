@@ -149,3 +149,63 @@ def test_repeat_is_bit_identical():
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), g.out.view(torch.int16))
     assert TOL["bf16"]["atol"] > 0
+
+
+def test_prefix_cache_prefills_only_the_suffix():
+    """Prefix caching + paged prefill: request B's prompt starts with request
+    A's first 64 tokens (four full blocks), so the manager serves those from
+    A's cached blocks and B's prefill chunk is only its own suffix, attending
+    over the shared blocks through its table.  Both managers (the library's
+    and the oracle's) give the same tables; B's and A's outputs match the
+    oracle's causal attention over the same tokens."""
+    hq, hkv, d, bs = 8, 2, 128, 16
+    LA, LB, shared = 100, 150, 64
+    b = workloads.prefill_custom("bf16", [LA, LB], [LA, LB - shared], hq, hkv, d, bs, seed=31,
+                                 extra_blocks=8)
+    rng = np.random.default_rng(31)
+    tok_a = rng.integers(1, 1000, LA).tolist()
+    tok_b = tok_a[:shared] + rng.integers(1000, 2000, LB - shared).tolist()
+    kB, vB = b.k[1].clone(), b.v[1].clone()
+    kB[:shared], vB[:shared] = b.k[0][:shared], b.v[0][:shared]   # same tokens, same K/V
+
+    # oracle: its own prefix-caching manager, cache writes and causal attention
+    om = oracle.BlockManager(oracle.BlockAllocator(b.num_blocks, b.free_order), bs)
+    om.enable_prefix_cache()
+    osa, ca = om.add_seq_prompt(0, tok_a)
+    osb, cb = om.add_seq_prompt(1, tok_b)
+    assert (ca, cb) == (0, shared)
+    okc = oracle.empty_cache(b.num_blocks, hkv, bs, d, "bf16")
+    ovc = oracle.empty_cache(b.num_blocks, hkv, bs, d, "bf16")
+    oracle.reshape_and_cache(okc, ovc, oracle.as_storage(b.k[0], "bf16"),
+                             oracle.as_storage(b.v[0], "bf16"), osa)
+    oracle.reshape_and_cache(okc, ovc, oracle.as_storage(kB, "bf16")[shared:],
+                             oracle.as_storage(vB, "bf16")[shared:], osb[shared:])
+    mb = -(-LB // bs)
+    otab, olens = om.table_rows([0, 1], mb)
+    otab = np.asarray(otab, dtype=np.int32)
+    cu = np.array([0, LA, LA + LB - shared], dtype=np.int32)
+    ref = oracle.paged_prefill(oracle.as_storage(b.q, "bf16"), okc, ovc, otab, olens, cu, b.scale,
+                               "bf16")
+
+    # CUDA path: the library's manager, cache writes of what is not cached, prefill
+    m = pa.BlockManager(pa.BlockAllocator(b.num_blocks, b.free_order), bs)
+    m.enable_prefix_cache()
+    sa, _ = m.add_seq_prompt(0, tok_a)
+    sb, cached = m.add_seq_prompt(1, tok_b)
+    assert cached == shared and sb[:shared].tolist() == [-1] * shared
+    kc = torch.zeros((b.num_blocks, hkv, bs, d), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    keys = torch.cat([b.k[0], kB[shared:]]).cuda()
+    vals = torch.cat([b.v[0], vB[shared:]]).cuda()
+    slots = torch.cat([sa, sb[shared:]]).cuda()
+    pa.pa_reshape_and_cache(keys, vals, kc, vc, slots, err_flag=err)
+    tab, lens = m.block_tables([0, 1], mb)
+    assert np.array_equal(tab.numpy(), otab) and lens.tolist() == [LA, LB]
+    q = b.q.cuda()
+    out = torch.full_like(q, float("nan"))
+    pa.pa_prefill(out, q, kc, vc, tab.cuda(), lens.cuda(), torch.from_numpy(cu).cuda(),
+                  max(LA, LB - shared), b.scale, err_flag=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    check_close(out_f64(out, "bf16"), ref, "bf16", "prefix-cached prompt, suffix prefill")

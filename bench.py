@@ -573,6 +573,8 @@ def run_e2e(sess, w, args, world):
                     lens=torch.empty(S, dtype=torch.int32).pin_memory(),
                     out=torch.empty((S, hq, d), dtype=w.torch_dtype).pin_memory())
     pins = [pinned_set(), pinned_set()]          # alternate steps use alternate sets
+    # the batch of each step (which sequences run) is a step input like q/K/V
+    seq_ids = [torch.tensor(w.step_seqs(k), dtype=torch.int64) for k in range(w.num_steps)]
     qs = [w.step_q[k].pin_memory() for k in range(w.num_steps)]
     kk = [w.step_k[k].pin_memory() for k in range(w.num_steps)]
     vv = [w.step_v[k].pin_memory() for k in range(w.num_steps)]
@@ -586,7 +588,7 @@ def run_e2e(sess, w, args, world):
     dout = torch.empty((S, hq, d), dtype=w.torch_dtype, device=dev)
 
     def host_part(k, pin):
-        seqs = w.step_seqs(k)
+        seqs = seq_ids[k]
         _, cow = mgr.append_step(seqs, slots_out=pin["slots"], cow_out=pin["cow"])
         _, lens = mgr.block_tables(seqs, mb, tables_out=pin["tab"], lens_out=pin["lens"])
         ncow = cow.shape[0]

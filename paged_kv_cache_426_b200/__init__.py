@@ -63,9 +63,9 @@ SIGNATURES = {
     "pa_manager_fork": ([_vp, _i64, _i64], _i),
     "pa_manager_free_seq": ([_vp, _i64], _i),
     "pa_manager_append": ([_vp, _i64, _i, _pi64, _pi64, C.POINTER(_i)], _i),
-    "pa_manager_append_step": ([_vp, _pi64, _i, _pi64, _pi64, C.POINTER(_i)], _i),
+    "pa_manager_append_step": ([_vp, _vp, _i, _vp, _vp, C.POINTER(_i)], _i),
     "pa_manager_seq_len": ([_vp, _i64, _pi32], _i),
-    "pa_manager_block_tables": ([_vp, _pi64, _i, _pi32, _i, _pi32], _i),
+    "pa_manager_block_tables": ([_vp, _vp, _i, _vp, _i, _vp], _i),
     "pa_manager_enable_prefix_cache": ([_vp], _i),
     "pa_manager_add_seq_prompt": ([_vp, _i64, _pi32, _i, _pi64, C.POINTER(_i)], _i),
     "pa_manager_prefix_cache_stats": ([_vp, _pi64], _i),
@@ -290,10 +290,10 @@ class BlockManager:
         slots = slots_out if slots_out is not None else torch.empty(n, dtype=torch.int64)
         cow = cow_out if cow_out is not None else torch.empty((max(n, 1), 2), dtype=torch.int64)
         k = C.c_int(0)
-        check(lib.pa_manager_append_step(self._h, C.cast(ids.data_ptr(), _pi64), n,
-                                         C.cast(slots.data_ptr(), _pi64),
-                                         C.cast(cow.data_ptr(), _pi64), C.byref(k)), "append_step")
-        return slots[:n], cow[:k.value]
+        # per-step call: raw addresses, no ctypes casts (the arrays are contiguous int64)
+        check(lib.pa_manager_append_step(self._h, ids.data_ptr(), n, slots.data_ptr(),
+                                         cow.data_ptr(), C.byref(k)), "append_step")
+        return (slots if slots.numel() == n else slots[:n]), cow[:k.value]
 
     def seq_len(self, seq: int) -> int:
         r = C.c_int32()
@@ -306,9 +306,8 @@ class BlockManager:
         n = ids.numel()
         tab = tables_out if tables_out is not None else torch.empty((n, max_blocks), dtype=torch.int32)
         lens = lens_out if lens_out is not None else torch.empty(n, dtype=torch.int32)
-        check(lib.pa_manager_block_tables(self._h, C.cast(ids.data_ptr(), _pi64), n,
-                                          C.cast(tab.data_ptr(), _pi32), max_blocks,
-                                          C.cast(lens.data_ptr(), _pi32)), "block_tables")
+        check(lib.pa_manager_block_tables(self._h, ids.data_ptr(), n, tab.data_ptr(), max_blocks,
+                                          lens.data_ptr()), "block_tables")
         return tab, lens
 
     # ---- prefix caching

@@ -1,5 +1,8 @@
 /*
- * pa.h - C ABI of the B200 paged KV-cache decode library (libpa_b200.so).
+ * pa.h - C ABI of the B200 paged KV-cache library (libpa_b200.so): cache
+ * writes (pa_reshape_and_cache), decode attention (pa_decode,
+ * pa_decode_static), prefill-chunk attention (pa_prefill), copy-on-write
+ * copies (pa_copy_blocks) and the host block allocator / manager.
  *
  * PagedAttention keeps each request's K/V cache in fixed-size physical blocks
  * that a per-request block table maps from logical order; attention reads the
@@ -29,7 +32,8 @@
  *    row-major, 16-byte aligned.  One (block, KV head) tile is
  *    block_size*head_dim contiguous elements; slot = block*block_size + offset.
  *  - Supported: head_dim 64 or 128; block_size 8, 16, 32, 64 or 128;
- *    dtype f32, f16, bf16; num_q_heads = G * num_kv_heads with G in 1,2,4,8.
+ *    dtype f32, f16, bf16 (pa_prefill: f16, bf16); num_q_heads =
+ *    G * num_kv_heads with G in 1,2,4,8.
  *  - Host objects (allocator, manager) are not thread-safe.
  */
 #ifndef PA_B200_H

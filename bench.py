@@ -2,25 +2,36 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl ours|reference] [--partition-size P] [--engine auto|core|tensor]
+                    [--only] [--extra-steps K2]
 
 A step is one decode step of the workload's batch: copy-on-write block
 copies (when the host manager reports any), the cache write of the step's new
-tokens, and decode attention over every sequence.  The host metadata of every
-step (slot mapping, copy pairs, block tables, lengths) is produced by the
-library's C++ manager before the timed region and sits in HBM with the
-queries and new K/V rows, so the timed region holds only the library's
-kernels.  Timing: CUDA events on the launching stream around K consecutive
-steps after W warm-up steps, synchronised on both sides; every step is a new
-token of the same sequences (the KV cache, 0.6-2.7 GB, is larger than the
-126 MB L2, so no flush is needed).
+tokens, and decode attention over every sequence (the decode kernel plus the
+split-K merge).  The host metadata of every step (slot mapping, copy pairs,
+block tables, lengths) is produced by the library's C++ manager before the
+timed region and sits in HBM with the queries and new K/V rows.  Each step is
+captured once as a CUDA graph from the public calls and replayed; CUDA events
+on the launching stream around each replay give per-step device times (and
+their percentiles), W warm-up steps run first, everything synchronised on
+both sides.  Every step is a new token of the same sequences; the KV cache of
+the headline batch (1.1 GB) is larger than the 126 MB L2, so no flush is
+needed there; batches whose cache is not several times L2 are flushed (a
+256 MB write) before each timed replay and are also reported warm.
 
 value = algorithmic bytes of the K steps / timed span, algorithmic bytes per
 step = sum_s L_s * Hkv * D * 2 * e (K and V) + 2 * S * Hq * D * e (q, out)
-+ sum_s ceil(L_s / bs) * 4 (block-table entries).
++ sum_s ceil(L_s / bs) * 4 (block-table entries).  roofline.achieved is the
+same bytes over the decode call alone (its own graph replays).  At one GPU the
+line also carries per_workload: the other decode batches (GQA at block 16 and
+32, long context, shared prefix with logical and unique-physical bytes, the
+tiny fp32 batch), each with decode and whole-step GB/s, fractions of the
+measured copy peak, of a read peak measured here and of 8 TB/s, p10/p50/p90
+step times and ncu traffic over algorithmic bytes.
 
 e2e = the same metric through the public API with host buffers: the C++
 manager appends the step's tokens live, pinned host buffers are copied to the
-device, the kernels run and the output comes back to the host, every step.
+device, the kernels run and the output comes back to the host, every step,
+pipelined one step ahead as a serving loop runs.
 
 Multi-GPU: independent replicas (the decode path has no exchange step); each
 rank runs its own copy of the batch; value = bytes of all ranks / max-over-
@@ -47,6 +58,9 @@ import workloads  # noqa: E402
 
 METRIC = "paged decode attention: KV-read GB/s (% of B200 HBM peak) and seqs/s per step"
 DEFAULT_WORKLOAD = "mha7b_f16"
+# the other decode batches, measured in the same run (one GPU) and reported under per_workload
+GATE_WORKLOADS = ("gqa8b_bf16_bs16", "gqa8b_bf16_bs32", "long_bf16", "prefix_f16", "tiny_f32")
+NOMINAL_HBM_GBS = 8000.0
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -372,11 +386,13 @@ def aggregate(rank_bytes, rank_span_ms, world):
 # ----------------------------------------------------------------------------- our path
 
 class Session:
-    """One replica: caches, the C++ manager, and per-step device inputs."""
+    """One replica of one workload: caches, the C++ manager, and per-step
+    device inputs."""
 
     def __init__(self, w, P, dev, engine="auto"):
         import paged_kv_cache_426_b200 as pa
         self.pa, self.w, self.P, self.dev = pa, w, P, dev
+        self.engine = None if engine == "auto" else engine     # per-call option
         dt = w.torch_dtype
         self.esize = torch.tensor([], dtype=dt).element_size()
         self.kc = torch.empty((w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim), dtype=dt,
@@ -440,12 +456,14 @@ class Session:
             plan.append(dict(
                 slots=slots.to(self.dev), cow=cow.to(self.dev) if cow.shape[0] else None,
                 tab=tab.to(self.dev), lens=lens.to(self.dev), lens_host=lens.tolist(),
-                q=w.step_q[k].to(self.dev), k=w.step_k[k].to(self.dev),
+                tab_host=tab, q=w.step_q[k].to(self.dev), k=w.step_k[k].to(self.dev),
                 v=w.step_v[k].to(self.dev)))
         return plan
 
-    def run_step(self, st, out):
-        pa, w = self.pa, self.w
+    def write(self, st):
+        """Copy-on-write copies (when the manager reported any) and the cache
+        write of one step.  Returns the launches."""
+        pa = self.pa
         n = 0
         if st["cow"] is not None:
             pa.pa_copy_blocks(self.kc, self.vc, st["cow"], err_flag=self.err)
@@ -458,230 +476,444 @@ class Session:
         when a sequence can span several partitions.  Returns the launches."""
         self.pa.pa_decode(out, st["q"], self.kc, self.vc, st["tab"], st["lens"], self.max_len,
                           self.w.scale, partition_size=self.P, workspace=self.ws,
-                          err_flag=self.err)
+                          err_flag=self.err, engine=self.engine)
         n_pmax = -(-self.max_len // self.P) if self.P > 0 else 1
         return 2 if n_pmax > 1 else 1
+
+    def step(self, st, out):
+        return self.write(st) + self.decode(st, out)
 
     def bytes_of(self, lens):
         w = self.w
         return algorithmic_bytes(lens, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
                                  self.esize)
 
+    def unique_bytes_of(self, st):
+        """Like bytes_of, but K/V counted once per physical block (the largest
+        number of its rows any sequence reads): blocks shared by reference
+        count are stored once and can be read from HBM once."""
+        w = self.w
+        bs = w.block_size
+        rows = {}
+        for row, L in zip(st["tab_host"].tolist(), st["lens_host"]):
+            for i in range(-(-L // bs)):
+                b = row[i]
+                rows[b] = max(rows.get(b, 0), min(bs, L - i * bs))
+        kv = sum(rows.values()) * w.num_kv_heads * w.head_dim * 2 * self.esize
+        S = len(st["lens_host"])
+        return (kv + 2 * S * w.num_q_heads * w.head_dim * self.esize
+                + sum(-(-L // bs) for L in st["lens_host"]) * 4)
+
+
+def capture(fn):
+    """A CUDA graph of whatever ``fn`` launches on the current stream."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def replay_timed(graphs, flush=None):
+    """Replay ``graphs`` in order on the current stream, a CUDA event pair
+    around each replay; with ``flush`` (a buffer larger than L2) the buffer
+    is overwritten before each replay, outside its event pair.  Returns the
+    per-replay device times (ms) and the span from the first start to the
+    last end (ms)."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in graphs]
+    for g, (a, b) in zip(graphs, ev):
+        if flush is not None:
+            flush.fill_(1)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev], ev[0][0].elapsed_time(ev[-1][1])
+
+
+def pct(xs, q):
+    """q-th percentile (0..100) of xs, linear interpolation."""
+    xs = sorted(xs)
+    if len(xs) == 1:
+        return xs[0]
+    r = (len(xs) - 1) * q / 100.0
+    lo = int(math.floor(r))
+    hi = min(lo + 1, len(xs) - 1)
+    return xs[lo] + (xs[hi] - xs[lo]) * (r - lo)
+
+
+def spread(ms):
+    return {"p10": round(pct(ms, 10), 4), "p50": round(pct(ms, 50), 4),
+            "p90": round(pct(ms, 90), 4)}
+
+
+def read_peak(dev, gib=4, reps=6):
+    """HBM read bandwidth of this GPU, measured here: a plain reduction over
+    ``gib`` GiB (torch's sum kernel reads every byte once and writes a
+    scalar), best of ``reps``; GB/s.  The buffer is freed afterwards."""
+    x = torch.ones((gib << 30) // 4, dtype=torch.float32, device=dev)
+    best = 0.0
+    for i in range(reps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum()
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            best = max(best, x.numel() * 4 / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del x
+    torch.cuda.empty_cache()
+    return round(best, 1)
+
+
+def workload_config(w, P, S, lens, step_bytes, world, engine, l2):
+    return {"workload": w.name, "num_seqs": S, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+            "block_size": w.block_size, "partition_size": P,
+            "mean_context_len": round(sum(lens) / S, 1), "kv_bytes_per_step": step_bytes,
+            "parallelism": f"replicas x{world}", "l2": l2, "engine": engine}
+
+
+L2_BYTES = 126 << 20
+
+
+def measure(name, args, dev, n_timed, world, engine="auto", flush_buf=None, warm_too=False,
+            sampler=None):
+    """Device-timed steps of one workload.  Every step (copy-on-write copies,
+    cache write, decode + merge) and, separately, its decode call alone are
+    captured as CUDA graphs and replayed in step order with CUDA events around
+    each replay.  Returns the numbers and the session (for the end-to-end
+    leg)."""
+    n_steps = args.warmup + n_timed
+    w = workloads.make(name, steps=n_steps)
+    P = w.partition_size if args.partition_size is None else args.partition_size
+    sess = Session(w, P, dev, engine)
+    _, mgr = sess.prefill()
+    plan = sess.plan_steps(mgr, n_steps)
+    out = torch.empty_like(plan[0]["q"])
+    # eager warm-up steps (kernel attributes are set on first use), then graphs
+    for k in range(args.warmup):
+        sess.step(plan[k], out)
+    torch.cuda.synchronize()
+    timed = plan[args.warmup:]
+    launches = 0
+    step_graphs, dec_graphs = [], []
+    for st in timed:
+        n = [0]
+
+        def whole(st=st, n=n):
+            n[0] = sess.step(st, out)
+        step_graphs.append(capture(whole))
+        dec_graphs.append(capture(lambda st=st: sess.decode(st, out)))
+        launches += n[0]
+    # clock soak (the first step again and again: idempotent writes); the
+    # sampler sees the soak and the timed replays only
+    if sampler is not None:
+        sampler.start()
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        for _ in range(10):
+            step_graphs[0].replay()
+        torch.cuda.synchronize()
+    step_graphs[0].replay()
+    dec_graphs[0].replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    need_flush = flush_buf is not None and sess.kc.numel() * sess.esize * 2 < 4 * L2_BYTES
+    step_ms, span_ms = replay_timed(step_graphs, flush_buf if need_flush else None)
+    dec_ms, _ = replay_timed(dec_graphs, flush_buf if need_flush else None)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
+    barrier(world)
+    assert int(sess.err.item()) == 0, f"{name}: device error flag {int(sess.err.item())}"
+    step_bytes = [sess.bytes_of(st["lens_host"]) for st in timed]
+    res = dict(w=w, sess=sess, P=P, plan=plan, step_bytes=step_bytes, step_ms=step_ms,
+               dec_ms=dec_ms, span_ms=span_ms if not need_flush else sum(step_ms),
+               launches=launches, flushed=need_flush, clocks=clocks)
+    if name.startswith("prefix"):
+        res["unique_bytes"] = [sess.unique_bytes_of(st) for st in timed]
+    if warm_too and need_flush:
+        res["warm_step_ms"], _ = replay_timed(step_graphs)
+        res["warm_dec_ms"], _ = replay_timed(dec_graphs)
+    del step_graphs, dec_graphs
+    return res
+
+
+def summarize(m, peak, rpeak):
+    """Per-workload summary: GB/s of the decode call and of the whole step,
+    their fractions of the measured copy peak, the read peak and 8 TB/s,
+    step-time percentiles, and ncu traffic over algorithmic bytes."""
+    w, sess = m["w"], m["sess"]
+    b = sum(m["step_bytes"]) / len(m["step_bytes"])
+    dec = sum(m["dec_ms"]) / len(m["dec_ms"])
+    stp = sum(m["step_ms"]) / len(m["step_ms"])
+    dec_gbs = b / (dec * 1e-3) / 1e9
+    stp_gbs = b / (stp * 1e-3) / 1e9
+    traffic = profiled_traffic(w.name, b)
+    r = {"decode_gbs": round(dec_gbs, 1), "step_gbs": round(stp_gbs, 1),
+         "decode_frac_measured_copy": round(dec_gbs / peak, 4),
+         "decode_frac_read_peak": round(dec_gbs / rpeak, 4) if rpeak else None,
+         "decode_frac_8tbs": round(dec_gbs / NOMINAL_HBM_GBS, 4),
+         "step_frac_measured_copy": round(stp_gbs / peak, 4),
+         "step_frac_8tbs": round(stp_gbs / NOMINAL_HBM_GBS, 4),
+         "decode_ms": spread(m["dec_ms"]), "step_ms": spread(m["step_ms"]),
+         "algorithmic_bytes_per_step": int(b),
+         "traffic_over_algorithmic": round(traffic / b, 4) if traffic else None,
+         "seqs_per_s": round(sess.S / (stp * 1e-3), 1),
+         "decode_seqs_per_s": round(sess.S / (dec * 1e-3), 1),
+         "steps": len(m["step_ms"]), "partition_size": m["P"], "dtype": w.dtype,
+         "l2": ("L2 flushed (256 MB write) before every timed replay" if m["flushed"]
+                else "KV cache larger than L2")}
+    if "unique_bytes" in m:
+        u = sum(m["unique_bytes"]) / len(m["unique_bytes"])
+        r["logical_bytes_per_step"] = int(b)
+        r["unique_physical_bytes_per_step"] = int(u)
+        r["decode_unique_gbs"] = round(u / (dec * 1e-3) / 1e9, 1)
+        r["step_unique_gbs"] = round(u / (stp * 1e-3) / 1e9, 1)
+    if "warm_step_ms" in m:
+        wd = sum(m["warm_dec_ms"]) / len(m["warm_dec_ms"])
+        ws = sum(m["warm_step_ms"]) / len(m["warm_step_ms"])
+        r["warm"] = {"decode_gbs": round(b / (wd * 1e-3) / 1e9, 1),
+                     "step_gbs": round(b / (ws * 1e-3) / 1e9, 1),
+                     "decode_ms": spread(m["warm_dec_ms"]), "step_ms": spread(m["warm_step_ms"])}
+    return r
+
 
 def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    n_steps = args.warmup + args.steps
-    w = workloads.make(args.workload, steps=n_steps)
-    P = w.partition_size if args.partition_size is None else args.partition_size
-    import paged_kv_cache_426_b200 as pa
-    pa.pa_set_decode_engine({"auto": 0, "core": 1, "tensor": 2}[args.engine])
-    sess = Session(w, P, dev, args.engine)
-    _, mgr = sess.prefill()
-    plan = sess.plan_steps(mgr, n_steps)
-    out = torch.empty_like(plan[0]["q"])
-    stream = torch.cuda.current_stream()
-
-    # clock soak: step 0 again and again (idempotent writes) while the sampler starts
-    sampler = ClockSampler(local)
-    sampler.start()
-    t_end = time.time() + args.soak
-    while time.time() < t_end:
-        for _ in range(10):
-            sess.run_step(plan[0], out)
-            sess.decode(plan[0], out)
-        torch.cuda.synchronize()
-
-    for k in range(args.warmup):
-        sess.run_step(plan[k], out)
-        sess.decode(plan[k], out)
-    torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    launches = 0
-    for i in range(args.steps):
-        st = plan[args.warmup + i]
-        ev[i][0].record(stream)
-        launches += sess.run_step(st, out)
-        ev[i][1].record(stream)
-        launches += sess.decode(st, out)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = sampler.stop()
-    assert int(sess.err.item()) == 0, f"device error flag {int(sess.err.item())}"
-    span_ms = ev[0][0].elapsed_time(ev[-1][2])
-    dec_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    step_bytes = [sess.bytes_of(plan[args.warmup + i]["lens_host"]) for i in range(args.steps)]
-    total_bytes, span_ms, value = aggregate(sum(step_bytes), span_ms, world)
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    dec_gbs = (sum(step_bytes) / len(step_bytes)) / (dec_avg_ms * 1e-3) / 1e9
     peak, peak_kind = measured_peaks()
+    rpeak = read_peak(dev) if world == 1 else None
+    m = measure(args.workload, args, dev, args.steps, world, args.engine,
+                sampler=ClockSampler(local))
+    w, sess, P, launches, clocks = m["w"], m["sess"], m["P"], m["launches"], m["clocks"]
+    step_bytes = m["step_bytes"]
+    total_bytes, span_ms, value = aggregate(sum(step_bytes), m["span_ms"], world)
+    dec_avg_ms = sum(m["dec_ms"]) / len(m["dec_ms"])
+    dec_gbs = (sum(step_bytes) / len(step_bytes)) / (dec_avg_ms * 1e-3) / 1e9
     S = sess.S
-
+    lens0 = m["plan"][args.warmup]["lens_host"]
     e2e = run_e2e(sess, w, args, world) if args.e2e else None
+    head = summarize(m, peak, rpeak)
+    del m
+
+    per = {}
+    if world == 1 and args.all_workloads:
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        for name in GATE_WORKLOADS:
+            if name == args.workload:
+                continue
+            mw = measure(name, args, dev, args.extra_steps, world, args.engine, flush_buf=flush,
+                         warm_too=True)
+            per[name] = summarize(mw, peak, rpeak)
+            del mw
+            torch.cuda.empty_cache()
+        del flush
+    per[args.workload] = head
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(span_ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded; see workloads/)",
-        "config": {"workload": w.name, "num_seqs": S, "num_q_heads": w.num_q_heads,
-                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
-                   "block_size": w.block_size, "partition_size": P,
-                   "mean_context_len": round(sum(plan[args.warmup]["lens_host"]) / S, 1),
-                   "kv_bytes_per_step": step_bytes[0],
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (KV cache >= 0.6 GB vs 126 MB)",
-                   "engine": args.engine},
+        "config": workload_config(w, P, S, lens0, step_bytes[0], world, args.engine,
+                                  "inputs larger than L2 (KV cache >= 0.6 GB vs 126 MB)"),
+        "timing": "each step a CUDA graph replay (captured from the public calls), CUDA events "
+                  "around each replay",
         "seqs_per_s": round(S * world / (span_ms * 1e-3 / args.steps), 1),
         "decode_only": {"gbs": round(dec_gbs, 1), "ms": round(dec_avg_ms, 4),
                         "seqs_per_s": round(S / (dec_avg_ms * 1e-3), 1)},
+        "step_ms": head["step_ms"], "decode_ms": head["decode_ms"],
+        "frac_of_8tbs": {"step": round(value / world / NOMINAL_HBM_GBS, 4),
+                         "decode": round(dec_gbs / NOMINAL_HBM_GBS, 4)},
+        "read_peak_gbs": rpeak,
         "roofline": {"bound": "hbm", "achieved": round(dec_gbs, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(dec_gbs / peak, 4),
                      "traffic": profiled_traffic(w.name, sum(step_bytes) / len(step_bytes)),
-                     "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "pa_decode"},
+                     "peak_kind": f"{peak_kind} copy bandwidth (burst, kernel timed alone)",
+                     "frac_of_read_peak": round(dec_gbs / rpeak, 4) if rpeak else None,
+                     "kernel": "pa_decode"},
         "gpu_launches": launches,
         "clocks": clocks,
     }
+    if per and len(per) > 1:
+        result["per_workload"] = per
     if e2e:
         result["e2e"] = e2e
     if rank == 0 and world == 1 and args.cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        result["cpu_baseline"]["one_core"] = cpu_baseline(w, args.cpu_seconds, threads=1)
     return result
 
 
 def run_e2e(sess, w, args, world):
     """Same metric through the public API with host buffers, every step: the
-    live C++ manager's appends and block tables (host), then the step's H2D
-    copies from pinned buffers, cache write, decode and the D2H of out.  The
-    device part of each timed step is one CUDA graph (captured beforehand from
-    the same public calls), so Python launch overhead does not pose as step
-    time; the host part runs every step inside the timed region."""
+    live C++ manager's appends and block tables (host), the step's H2D copies
+    from pinned buffers, copy-on-write copies, cache write, decode and the D2H
+    of out.  Steps are pipelined the way a serving loop runs them: while step
+    k's kernels run, the host prepares step k+1 (manager calls into the other
+    pinned set) and step k+1's inputs cross PCIe on a copy stream into the
+    other device set; out of step k returns on a third stream, and the host
+    waits for it one step later.  The device work of the copy and compute
+    stages is CUDA graphs captured beforehand from the same public calls, so
+    Python launch overhead does not pose as step time."""
     pa = sess.pa
     dev = sess.dev
     _, mgr = sess.prefill(write=False)       # same script -> same pool state
     S, mb = sess.S, sess.mb
     hq, hkv, d = w.num_q_heads, w.num_kv_heads, w.head_dim
+    dt = w.torch_dtype
+    n = w.num_steps
 
     def pinned_set():
         return dict(slots=torch.empty(S, dtype=torch.int64).pin_memory(),
                     cow=torch.empty((S, 2), dtype=torch.int64).pin_memory(),
                     tab=torch.empty((S, mb), dtype=torch.int32).pin_memory(),
                     lens=torch.empty(S, dtype=torch.int32).pin_memory(),
-                    out=torch.empty((S, hq, d), dtype=w.torch_dtype).pin_memory())
-    pins = [pinned_set(), pinned_set()]          # alternate steps use alternate sets
-    # the batch of each step (which sequences run) is a step input like q/K/V
-    seq_ids = [torch.tensor(w.step_seqs(k), dtype=torch.int64) for k in range(w.num_steps)]
-    qs = [w.step_q[k].pin_memory() for k in range(w.num_steps)]
-    kk = [w.step_k[k].pin_memory() for k in range(w.num_steps)]
-    vv = [w.step_v[k].pin_memory() for k in range(w.num_steps)]
-    dq = torch.empty((S, hq, d), dtype=w.torch_dtype, device=dev)
-    dk = torch.empty((S, hkv, d), dtype=w.torch_dtype, device=dev)
-    dvv = torch.empty_like(dk)
-    dslots = torch.empty(S, dtype=torch.int64, device=dev)
-    dcow = torch.empty((S, 2), dtype=torch.int64, device=dev)
-    dtab = torch.empty((S, mb), dtype=torch.int32, device=dev)
-    dlens = torch.empty(S, dtype=torch.int32, device=dev)
-    dout = torch.empty((S, hq, d), dtype=w.torch_dtype, device=dev)
+                    out=torch.empty((S, hq, d), dtype=dt).pin_memory())
 
-    def host_part(k, pin):
-        seqs = seq_ids[k]
-        _, cow = mgr.append_step(seqs, slots_out=pin["slots"], cow_out=pin["cow"])
-        _, lens = mgr.block_tables(seqs, mb, tables_out=pin["tab"], lens_out=pin["lens"])
+    def device_set():
+        return dict(q=torch.empty((S, hq, d), dtype=dt, device=dev),
+                    k=torch.empty((S, hkv, d), dtype=dt, device=dev),
+                    v=torch.empty((S, hkv, d), dtype=dt, device=dev),
+                    slots=torch.empty(S, dtype=torch.int64, device=dev),
+                    cow=torch.empty((S, 2), dtype=torch.int64, device=dev),
+                    tab=torch.empty((S, mb), dtype=torch.int32, device=dev),
+                    lens=torch.empty(S, dtype=torch.int32, device=dev),
+                    out=torch.empty((S, hq, d), dtype=dt, device=dev))
+    pins = [pinned_set(), pinned_set()]          # step k uses set k % 2
+    devs = [device_set(), device_set()]
+    # the batch of each step (which sequences run) is a step input like q/K/V
+    seq_ids = [torch.tensor(w.step_seqs(k), dtype=torch.int64) for k in range(n)]
+    qs = [w.step_q[k].pin_memory() for k in range(n)]
+    kk = [w.step_k[k].pin_memory() for k in range(n)]
+    vv = [w.step_v[k].pin_memory() for k in range(n)]
+    main = torch.cuda.current_stream()
+    copy_s, out_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def h2d(k, b):
+        D, pin = devs[b], pins[b]
+        D["q"].copy_(qs[k], non_blocking=True)
+        D["k"].copy_(kk[k], non_blocking=True)
+        D["v"].copy_(vv[k], non_blocking=True)
+        D["slots"].copy_(pin["slots"], non_blocking=True)
+        D["tab"].copy_(pin["tab"], non_blocking=True)
+        D["lens"].copy_(pin["lens"], non_blocking=True)
+
+    def compute(b):
+        D = devs[b]
+        pa.pa_reshape_and_cache(D["k"], D["v"], sess.kc, sess.vc, D["slots"], err_flag=sess.err)
+        pa.pa_decode(D["out"], D["q"], sess.kc, sess.vc, D["tab"], D["lens"], sess.max_len,
+                     w.scale, partition_size=sess.P, workspace=sess.ws, err_flag=sess.err,
+                     engine=sess.engine)
+
+    def host_part(k, b):
+        pin = pins[b]
+        _, cow = mgr.append_step(seq_ids[k], slots_out=pin["slots"], cow_out=pin["cow"])
+        _, lens = mgr.block_tables(seq_ids[k], mb, tables_out=pin["tab"], lens_out=pin["lens"])
         ncow = cow.shape[0]
         if ncow:                                 # copy-on-write pairs vary: never in a graph
-            dcow[:ncow].copy_(pin["cow"][:ncow], non_blocking=True)
-            pa.pa_copy_blocks(sess.kc, sess.vc, dcow[:ncow], err_flag=sess.err)
+            dcow = devs[b]["cow"][:ncow]
+            dcow.copy_(pin["cow"][:ncow], non_blocking=True)
+            pa.pa_copy_blocks(sess.kc, sess.vc, dcow, err_flag=sess.err)
         return ncow, lens
 
-    def device_part(k, pin):
-        dq.copy_(qs[k], non_blocking=True)
-        dk.copy_(kk[k], non_blocking=True)
-        dvv.copy_(vv[k], non_blocking=True)
-        dslots.copy_(pin["slots"], non_blocking=True)
-        dtab.copy_(pin["tab"], non_blocking=True)
-        dlens.copy_(pin["lens"], non_blocking=True)
-        pa.pa_reshape_and_cache(dk, dvv, sess.kc, sess.vc, dslots, err_flag=sess.err)
-        pa.pa_decode(dout, dq, sess.kc, sess.vc, dtab, dlens, sess.max_len, w.scale,
-                     partition_size=sess.P, workspace=sess.ws, err_flag=sess.err)
-        pin["out"].copy_(dout, non_blocking=True)
-
-    for k in range(args.warmup):                 # eager: first launches set kernel attributes
-        host_part(k, pins[k % 2])
-        device_part(k, pins[k % 2])
-        torch.cuda.synchronize()
-    graphs = {}
-    try:
-        for k in range(args.warmup, args.warmup + args.steps):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                device_part(k, pins[k % 2])
-            graphs[k] = g
-    except Exception:                            # capture unavailable: launch eagerly
-        graphs = {}
+    g_h2d, g_comp = [], []
+    for k in range(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=copy_s):
+            h2d(k, k % 2)
+        g_h2d.append(g)
+        g_comp.append(capture(lambda b=k % 2: compute(b)))
     torch.cuda.synchronize()
-    h2d = d2h = 0
-    total_bytes = 0
-    times = []
-    for k in range(args.warmup, args.warmup + args.steps):
-        pin = pins[k % 2]
-        torch.cuda.synchronize()
-        t0 = time.perf_counter()
-        ncow, lens = host_part(k, pin)
-        if graphs:
-            graphs[k].replay()
-        else:
-            device_part(k, pin)
-        torch.cuda.synchronize()                 # out is in host memory
-        times.append(time.perf_counter() - t0)
-        total_bytes += sess.bytes_of(lens.tolist())
-        h2d = sum(t.numel() * t.element_size() for t in (qs[k], kk[k], vv[k], pin["slots"],
-                                                          pin["tab"], pin["lens"]))
-        h2d += ncow * 16
-        d2h = pin["out"].numel() * pin["out"].element_size()
-    used_graphs = bool(graphs)
-    graphs.clear()
-    total_bytes, span_ms, gbs = aggregate(total_bytes, sum(times) * 1e3, world)
-    span = span_ms * 1e-3
+
+    ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
+    h2d_done, comp_done, out_done = ev(), ev(), ev()
+    stats = dict(bytes=0, h2d=0, d2h=0)
+
+    def run(ks, count):
+        pend = host_part(ks[0], ks[0] % 2)
+        for i, k in enumerate(ks):
+            b = k % 2
+            ncow, lens = pend
+            copy_s.wait_event(comp_done[b])      # compute k-2 has read device set b
+            with torch.cuda.stream(copy_s):
+                g_h2d[k].replay()
+                h2d_done[b].record(copy_s)
+            main.wait_event(h2d_done[b])
+            main.wait_event(out_done[b])         # D2H k-2 has read out of set b
+            g_comp[k].replay()
+            comp_done[b].record(main)
+            out_s.wait_event(comp_done[b])
+            with torch.cuda.stream(out_s):
+                pins[b]["out"].copy_(devs[b]["out"], non_blocking=True)
+                out_done[b].record(out_s)
+            if count:
+                stats["bytes"] += sess.bytes_of(lens.tolist())
+                stats["h2d"] = (sum(t.numel() * t.element_size() for t in
+                                    (qs[k], kk[k], vv[k], pins[b]["slots"], pins[b]["tab"],
+                                     pins[b]["lens"])) + ncow * 16)
+                stats["d2h"] = pins[b]["out"].numel() * pins[b]["out"].element_size()
+            if i + 1 < len(ks):
+                nb = ks[i + 1] % 2
+                h2d_done[nb].synchronize()       # step k-1's copies have read pinned set nb
+                pend = host_part(ks[i + 1], nb)
+            if i >= 1:
+                out_done[(k - 1) % 2].synchronize()   # step k-1's out is in host memory
+        out_done[ks[-1] % 2].synchronize()
+
+    run(list(range(args.warmup)), False)
+    torch.cuda.synchronize()
+    barrier(world)
+    t0 = time.perf_counter()
+    run(list(range(args.warmup, n)), True)
+    t1 = time.perf_counter()
+    assert int(sess.err.item()) == 0, f"e2e: device error flag {int(sess.err.item())}"
+    del g_h2d, g_comp
+    total_bytes, span_ms, gbs = aggregate(stats["bytes"], (t1 - t0) * 1e3, world)
+    K = n - args.warmup
     return {"value": round(gbs, 1), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(span / args.steps * 1e3, 4),
-            "device_part": "cuda graph" if used_graphs else "eager"}
+            "h2d_bytes_per_step": stats["h2d"], "d2h_bytes_per_step": stats["d2h"],
+            "ms_per_step": round(span_ms / K, 4),
+            "device_part": "cuda graphs (copy and compute stages), pipelined one step ahead"}
 
 
 # ----------------------------------------------------------------------------- the oracle on the host
 
-def cpu_baseline(w, seconds):
+def cpu_baseline(w, seconds, threads=None):
     """The oracle, as it stands, on the host cores: float64 decode of as many
-    whole sequences of the first step's batch as fit in about ``seconds``."""
-    import numpy as np
+    whole sequences of the first step's batch as fit in about ``seconds``.
+    ``threads``: cap on the BLAS threads (None = all the process may use)."""
+    import contextlib
     import oracle
-    from threadpoolctl import threadpool_info
+    from threadpoolctl import threadpool_info, threadpool_limits
     rec = oracle.run(w, decode=False, steps=1)
     st = rec.steps[0]
     q = oracle.as_storage(w.step_q[0], w.dtype)
     esize = torch.tensor([], dtype=w.torch_dtype).element_size()
-    done, nbytes, t0 = 0, 0, time.perf_counter()
     S = len(st.seqs)
-    while True:                 # whole sequences, cycling over the batch, ~`seconds` of work
-        s = done % S
-        oracle.paged_decode(q[s:s + 1], rec.key_cache, rec.value_cache, st.block_tables[s:s + 1],
-                            st.context_lens[s:s + 1], w.scale, w.dtype)
-        nbytes += algorithmic_bytes([int(st.context_lens[s])], w.num_q_heads, w.num_kv_heads,
-                                    w.head_dim, w.block_size, esize)
-        done += 1
-        if time.perf_counter() - t0 > seconds:
-            break
-    dt = time.perf_counter() - t0
-    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": threads,
+    limit = threadpool_limits(limits=threads) if threads else contextlib.nullcontext()
+    with limit:
+        done, nbytes, t0 = 0, 0, time.perf_counter()
+        while True:             # whole sequences, cycling over the batch, ~`seconds` of work
+            s = done % S
+            oracle.paged_decode(q[s:s + 1], rec.key_cache, rec.value_cache,
+                                st.block_tables[s:s + 1], st.context_lens[s:s + 1], w.scale,
+                                w.dtype)
+            nbytes += algorithmic_bytes([int(st.context_lens[s])], w.num_q_heads,
+                                        w.num_kv_heads, w.head_dim, w.block_size, esize)
+            done += 1
+            if time.perf_counter() - t0 > seconds:
+                break
+        dt = time.perf_counter() - t0
+        used = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": used,
             "kind": "oracle",
             "sample": f"{done} sequence decodes ({done / S:.2f} passes over the {S} sequences of "
                       f"step 0 of {w.name}), float64 numpy (gather through the block table + "
-                      f"softmax attention), {dt:.1f} s",
+                      f"softmax attention), {dt:.1f} s, {used} BLAS thread(s)",
             "seqs_per_s": round(done / dt, 3), "host_cpus": len(os.sched_getaffinity(0))}
 
 
@@ -702,12 +934,21 @@ def run_reference(args, rank, world):
     span = time.perf_counter() - t0
     value = sum(vals) / len(vals)
     base["value"] = round(value, 4)
+    P = w.partition_size if getattr(args, "partition_size", None) is None else args.partition_size
+    S = len(w.step_seqs(0))
+    lens = w.meta["lens"][:S] if len(w.meta["lens"]) >= S else w.meta["lens"]
+    esize = torch.tensor([], dtype=w.torch_dtype).element_size()
+    cfg = workload_config(w, P, S, lens,
+                          algorithmic_bytes(lens, w.num_q_heads, w.num_kv_heads, w.head_dim,
+                                            w.block_size, esize),
+                          world, getattr(args, "engine", "auto"), "host memory (oracle on CPU)")
+    cfg["parallelism"] = "host cores"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(span / args.steps * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded; see workloads/)",
-            "config": {"workload": w.name, "parallelism": "host cores"},
+            "config": cfg,
             "cpu_baseline": base,
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -792,8 +1033,6 @@ def run_sweep(args):
     ``args.steps`` steps; one JSON line per point."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    import paged_kv_cache_426_b200 as pa
-    pa.pa_set_decode_engine({"auto": 0, "core": 1, "tensor": 2}[args.engine])
     n = args.warmup + args.steps
     gqa_lens = workloads.make("gqa8b_bf16_bs16", steps=1).meta["lens"]
     points = [("block_size", bs, layout, gqa_lens) for bs in (8, 16, 32, 64, 128)
@@ -808,12 +1047,12 @@ def run_sweep(args):
         plan = sess.plan_steps(mgr, n)
         out = torch.empty_like(plan[0]["q"])
         for k in range(args.warmup):
-            sess.run_step(plan[k], out)
+            sess.write(plan[k])
             sess.decode(plan[k], out)
         torch.cuda.synchronize()
         total_ms, total_bytes = 0.0, 0
         for k in range(args.warmup, n):
-            sess.run_step(plan[k], out)
+            sess.write(plan[k])
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             sess.decode(plan[k], out)
@@ -843,6 +1082,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--only", dest="all_workloads", action="store_false",
+                    help="measure only --workload (no per_workload section)")
+    ap.add_argument("--extra-steps", type=int, default=10,
+                    help="timed steps of each other decode batch in per_workload")
     ap.add_argument("--sweep", action="store_true",
                     help="block-size / indirection study instead of the benchmark line")
     ap.add_argument("--waste", action="store_true",

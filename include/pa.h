@@ -140,11 +140,14 @@ int pa_decode(void* out, const void* query, const void* key_cache,
  * library keeps in device memory on every GPU that loads it, until exit.
  * Arguments and results are those of pa_decode.  A call whose workspace
  * (pa_decode_workspace_size) exceeds the array returns PA_ERR_INVALID and
- * launches nothing.  The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Each call clears the scheduler words on
- * `stream` and then runs pa_decode.  All calls on a device share the one
- * array: calls that overlap on the GPU race and must be serialised by the
+ * launches nothing, and so does a call that fails any other of pa_decode's
+ * host checks.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current, and looks it up
+ * again when the current context changes (e.g. after cudaDeviceReset); make
+ * that first call before any stream capture.  Each call clears the scheduler
+ * words on `stream` and then runs the decode with pa_decode's defaults.  All
+ * calls on a device share the one array and it keeps the last call's
+ * contents: calls that overlap on the GPU race and must be serialised by the
  * caller (e.g. one stream).  Allocates nothing. */
 #define PA_DECODE_STATIC_WORKSPACE_BYTES (16u << 20)
 int pa_decode_static(void* out, const void* query, const void* key_cache,
@@ -155,24 +158,39 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
                      float scale, int partition_size, pa_dtype dtype,
                      int32_t* err_flag, void* stream);
 
-/* Decode engine selection (for measurement).  PA_ENGINE_CUDA_CORE: fp32
- * dot products on CUDA cores (any dtype).  PA_ENGINE_TENSOR: tcgen05
- * tensor-core MMAs with accumulators in tensor memory, f16/bf16 only (f32
- * returns PA_ERR_UNSUPPORTED).  PA_ENGINE_AUTO (the default): the tensor
- * engine for f16/bf16 (falling back to CUDA cores for batches too large for
- * its shared-memory ring), CUDA cores for f32.  Process-wide; returns the
- * previous value. */
+/* pa_decode_ex - pa_decode with per-call options; options = NULL is exactly
+ * pa_decode.  The options apply to this call only (no process-wide state).
+ *   struct_size  sizeof(pa_decode_options) as the caller was compiled (a
+ *                smaller value returns PA_ERR_INVALID)
+ *   engine       PA_ENGINE_AUTO (pa_decode's choice): tcgen05 tensor-core
+ *                MMAs with accumulators in tensor memory for f16/bf16 (the
+ *                CUDA-core engine when its shared-memory ring does not fit,
+ *                i.e. several thousand sequences), CUDA cores for f32.
+ *                PA_ENGINE_CUDA_CORE: fp32 dot products on CUDA cores, any
+ *                dtype.  PA_ENGINE_TENSOR: the tensor-core engine, f16/bf16
+ *                only (f32 returns PA_ERR_UNSUPPORTED).
+ *   test_withhold_stage  failure-detection test aid, -1 = off.  With s >= 0
+ *                the producer that takes the first work unit of this call
+ *                withholds that unit's stage s (no copies, no arrival on the
+ *                stage's barrier), so the warps that need it give up after
+ *                the 2 s wait limit, set PA_DEV_TIMEOUT in err_flag and
+ *                return; the context and the workspace stay usable.  No GPU
+ *                fault is involved.  The pages have no counterpart.
+ * Out-of-range option values return PA_ERR_INVALID before any launch. */
 enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_TENSOR = 2 };
-int pa_set_decode_engine(int engine);
-
-/* Test hook for the bounded-wait path (failure detection without a fault):
- * with stage >= 0, in every later pa_decode call the producer that takes the
- * first work unit withholds that unit's stage number `stage` (no copies, no
- * arrival on the stage's barrier), so the warps that need it give up after
- * the 2 s wait limit, set PA_DEV_TIMEOUT in err_flag and return; the context
- * and the workspace stay usable.  -1 (the default) switches it off.
- * Process-wide; returns the previous value.  The pages have no counterpart. */
-int pa_test_withhold_stage(int stage);
+typedef struct pa_decode_options {
+    int struct_size;
+    int engine;
+    int test_withhold_stage;
+} pa_decode_options;
+int pa_decode_ex(void* out, const void* query, const void* key_cache,
+                 const void* value_cache, const int32_t* block_tables,
+                 int max_blocks_per_seq, const int32_t* context_lens,
+                 int max_context_len, int num_seqs, int num_q_heads,
+                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                 float scale, int partition_size, void* workspace,
+                 size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
+                 void* stream, const pa_decode_options* options);
 
 /* --------------------------------------------------------------------------
  * pa_prefill - causal multi-query attention of prefill chunks over the paged

@@ -48,9 +48,11 @@ def max_blocks_needed(w) -> int:
 
 
 def run(w, *, decode=True, steps=None, max_blocks=None, canary=0,
-        keep_prefill_cache=False) -> OracleRun:
+        keep_prefill_cache=False, decode_steps=None) -> OracleRun:
     """Execute the script.  ``steps``: how many decode steps to run (default all);
-    ``decode``: compute the float64 outputs of each step."""
+    ``decode``: compute the float64 outputs of each step; ``decode_steps``
+    (optional set of step indices): compute them for those steps only, each
+    from the cache as it stands at that step."""
     alloc = BlockAllocator(w.num_blocks, w.free_order)
     mgr = BlockManager(alloc, w.block_size)
     kc = empty_cache(w.num_blocks, w.num_kv_heads, w.block_size, w.head_dim, w.dtype, canary)
@@ -96,7 +98,7 @@ def run(w, *, decode=True, steps=None, max_blocks=None, canary=0,
             rows, lens = mgr.table_rows(seqs, mb)
             st = StepRecord(list(seqs), slots, cows, np.asarray(rows, np.int32),
                             np.asarray(lens, np.int32))
-            if decode:
+            if decode and (decode_steps is None or k in decode_steps):
                 st.out = paged_decode(as_storage(w.step_q[k], w.dtype), kc, vc,
                                       st.block_tables, st.context_lens, w.scale, w.dtype)
             rec.steps.append(st)

@@ -45,8 +45,8 @@ SIGNATURES = {
                    _sz, _i, _vp, _vp], _i),
     "pa_decode_static": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i,
                           _i, _vp, _vp], _i),
-    "pa_set_decode_engine": ([_i], _i),
-    "pa_test_withhold_stage": ([_i], _i),
+    "pa_decode_ex": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
+                      _sz, _i, _vp, _vp, _vp], _i),
     "pa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                     _i, _vp, _vp], _i),
     "pa_copy_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
@@ -157,21 +157,38 @@ def alloc_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_l
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
+class pa_decode_options(C.Structure):
+    """Per-call options of pa_decode_ex (include/pa.h)."""
+    _fields_ = [("struct_size", C.c_int), ("engine", C.c_int), ("test_withhold_stage", C.c_int)]
+
+
+ENGINES = {"auto": PA_ENGINE_AUTO, "core": PA_ENGINE_CUDA_CORE, "tensor": PA_ENGINE_TENSOR}
+
+
 def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len,
-              scale, *, partition_size=0, workspace=None, err_flag=None, stream=None):
+              scale, *, partition_size=0, workspace=None, err_flag=None, stream=None,
+              engine=None, test_withhold_stage=-1):
     """out/query [S, Hq, D]; caches [NB, Hkv, bs, D]; block_tables int32 [S, max_blocks];
-    context_lens int32 [S]."""
+    context_lens int32 [S].  ``engine`` ("auto", "core", "tensor" or a PA_ENGINE_*
+    value) and ``test_withhold_stage`` are per-call options (pa_decode_ex);
+    with neither given this is the plain pa_decode call."""
     _cuda(out, query, key_cache, value_cache, block_tables, context_lens, workspace, err_flag)
     S, hq, d = query.shape
     NB, hkv, bs, _ = key_cache.shape
     if workspace is None:
         raise PAError(PA_ERR_INVALID, "pa_decode needs a workspace (alloc_workspace)")
-    check(lib.pa_decode(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
-                        _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
-                        int(max_context_len), S, hq, hkv, d, bs, NB, float(scale),
-                        int(partition_size), _ptr(workspace),
-                        workspace.numel() * workspace.element_size(), pa_dtype(query),
-                        _ptr(err_flag), _stream(stream)), "pa_decode")
+    args = (_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, hq, hkv, d, bs,
+            NB, float(scale), int(partition_size), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), pa_dtype(query), _ptr(err_flag),
+            _stream(stream))
+    if engine is None and test_withhold_stage == -1:
+        check(lib.pa_decode(*args), "pa_decode")
+        return
+    eng = ENGINES[engine] if isinstance(engine, str) else (PA_ENGINE_AUTO if engine is None
+                                                            else int(engine))
+    opts = pa_decode_options(C.sizeof(pa_decode_options), eng, int(test_withhold_stage))
+    check(lib.pa_decode_ex(*args, C.byref(opts)), "pa_decode_ex")
 
 
 PA_DECODE_STATIC_WORKSPACE_BYTES = 16 << 20
@@ -208,13 +225,6 @@ def pa_prefill(out, query, key_cache, value_cache, block_tables, context_lens, c
                          _ptr(cu_seqlens_q), S, T, int(max_query_len), hq, hkv, d, bs, NB,
                          float(scale), pa_dtype(query), _ptr(err_flag), _stream(stream)),
           "pa_prefill")
-
-
-def pa_set_decode_engine(engine: int) -> int:
-    prev = lib.pa_set_decode_engine(engine)
-    if prev < 0:
-        raise PAError(prev, "pa_set_decode_engine")
-    return prev
 
 
 # ------------------------------------------------------------------ host objects

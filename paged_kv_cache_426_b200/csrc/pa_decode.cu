@@ -1670,8 +1670,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 // ------------------------------------------------------------ host side
 namespace {
 
-int g_engine = PA_ENGINE_AUTO;
-int g_hold_stage = -1;
 std::mutex g_mu;
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1707,6 +1705,37 @@ int make_map(CUtensorMap* map, const void* base, pa_dtype dt, int D, int64_t row
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
 }
+
+// Tensor maps of recent calls, per host thread.  A map holds nothing but the
+// base address, the element type and the shape, so an entry with the same key
+// is the same map, whatever memory now sits at that address; the cache only
+// saves the encoding on the host (a decode step needs three maps).
+struct MapCache {
+    struct Entry {
+        const void* base = nullptr;
+        int dt = -1, D = 0, box_rows = 0;
+        int64_t rows = 0;
+        CUtensorMap map;
+    };
+    static constexpr int N = 8;
+    Entry e[N];
+    int next = 0;
+    int get(CUtensorMap* out, const void* base, pa_dtype dt, int D, int64_t rows, int box_rows) {
+        for (int k = 0; k < N; ++k)
+            if (e[k].base == base && e[k].dt == (int)dt && e[k].D == D && e[k].rows == rows &&
+                e[k].box_rows == box_rows) {
+                *out = e[k].map;
+                return PA_OK;
+            }
+        const int st = make_map(out, base, dt, D, rows, box_rows);
+        if (st != PA_OK) return st;
+        Entry& n = e[next];
+        next = (next + 1) % N;
+        n.base = base; n.dt = (int)dt; n.D = D; n.rows = rows; n.box_rows = box_rows;
+        n.map = *out;
+        return PA_OK;
+    }
+};
 
 struct DevInfo {
     int sms = 0;
@@ -1899,51 +1928,16 @@ int launch_merge(const Launch& L, pa_dtype dt, int D, int G, int n_pmax) {
 
 using namespace pa;
 
-extern "C" {
+namespace {
 
-int pa_test_withhold_stage(int stage) {
-    if (stage < -1) return PA_ERR_INVALID;
-    std::lock_guard<std::mutex> lk(g_mu);
-    const int prev = g_hold_stage;
-    g_hold_stage = stage;
-    return prev;
-}
-
-int pa_set_decode_engine(int engine) {
-    if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_TENSOR) return PA_ERR_INVALID;
-    std::lock_guard<std::mutex> lk(g_mu);
-    const int prev = g_engine;
-    g_engine = engine;
-    return prev;
-}
-
-int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                             int max_context_len, int partition_size, size_t* bytes) {
-    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-        max_context_len < 0 || partition_size < 0 || (partition_size % TOK) != 0 ||
-        num_q_heads % num_kv_heads != 0)
-        return PA_ERR_INVALID;
-    const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
-    const int n_pmax = std::max(1, (max_context_len + P - 1) / P);
-    *bytes = ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, n_pmax);
-    return PA_OK;
-}
-
-int pa_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
-    if (!workspace || workspace_bytes < sizeof(WsHeader)) return PA_ERR_INVALID;
-    return cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) == cudaSuccess
-               ? PA_OK
-               : PA_ERR_CUDA;
-}
-
-int pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
-              const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
-              int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-              int block_size, int num_blocks, float scale, int partition_size, void* workspace,
-              size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag, void* stream) {
-    if (num_seqs == 0) return PA_OK;
-    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens ||
-        !workspace)
+// Host-side argument checks of pa_decode other than the workspace (everything
+// that can be checked without touching the GPU); PA_OK or the status to return.
+int validate_args(const void* out, const void* query, const void* key_cache,
+                  const void* value_cache, const int32_t* block_tables, int max_blocks_per_seq,
+                  const int32_t* context_lens, int max_context_len, int num_seqs, int num_q_heads,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                  int partition_size, pa_dtype dtype) {
+    if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens)
         return PA_ERR_INVALID;
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0 ||
@@ -1954,26 +1948,45 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     if (block_size != 8 && block_size != 16 && block_size != 32 && block_size != 64 &&
         block_size != 128)
         return PA_ERR_UNSUPPORTED;
-    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out) ||
-        (reinterpret_cast<uintptr_t>(workspace) & 255))
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
         return PA_ERR_INVALID;
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
     if (rows >= (int64_t(1) << 31)) return PA_ERR_UNSUPPORTED;
+    // the per-CTA prefix array must leave room for the pipeline
+    if (num_seqs > 16384) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+// The workspace checks: present, 256-byte aligned, at least `need` bytes.
+int validate_workspace(const void* workspace, size_t workspace_bytes, int num_seqs,
+                       int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                       int partition_size) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return PA_ERR_INVALID;
     size_t need = 0;
     pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
                              partition_size, &need);
-    if (workspace_bytes < need) return PA_ERR_INVALID;
-    const int G = num_q_heads / num_kv_heads;
+    return workspace_bytes < need ? PA_ERR_INVALID : PA_OK;
+}
 
+// The launches of one decode call; the arguments have passed validate().
+int decode_launch(void* out, const void* query, const void* key_cache, const void* value_cache,
+                  const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                  int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads,
+                  int head_dim, int block_size, int num_blocks, float scale, int partition_size,
+                  void* workspace, pa_dtype dtype, int32_t* err_flag, void* stream, int engine,
+                  int hold_stage) {
+    const int G = num_q_heads / num_kv_heads;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
     DevInfo di;
     if (dev_info(&di) != PA_OK) return PA_ERR_CUDA;
-    // the per-CTA prefix array must leave room for the pipeline
-    if (num_seqs > 16384) return PA_ERR_UNSUPPORTED;
 
     static thread_local Launch L;
+    static thread_local MapCache maps;
     const int box_rows = block_size >= TOK ? TOK : block_size;
-    int st = make_map(&L.kmap, key_cache, dtype, head_dim, rows, box_rows);
-    if (st == PA_OK) st = make_map(&L.vmap, value_cache, dtype, head_dim, rows, box_rows);
+    int st = maps.get(&L.kmap, key_cache, dtype, head_dim, rows, box_rows);
+    if (st == PA_OK) st = maps.get(&L.vmap, value_cache, dtype, head_dim, rows, box_rows);
     if (st != PA_OK) return st;
 
     const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
@@ -1999,21 +2012,13 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader));
     p.part_o = p.part_ml + ((((size_t)num_seqs * num_q_heads * n_pmax * 2 * 4 + 255) / 256) * 256) / 4;
     p.err = err_flag;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        p.hold_stage = g_hold_stage;
-    }
+    p.hold_stage = hold_stage;
 
     const int64_t units_ub = (int64_t)num_seqs * num_kv_heads * n_pmax;
     L.units_ub = units_ub;
     L.grid = dim3((unsigned)std::max<int64_t>(1, std::min<int64_t>(units_ub, di.sms)));
     L.stream = (cudaStream_t)stream;
 
-    int engine;
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        engine = g_engine;
-    }
     // tcgen05 engine: 16-bit types only (the default for them); fp32 runs on
     // CUDA cores
     const bool sixteen = dtype != PA_F32;
@@ -2028,7 +2033,7 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
         return (int)PA_ERR_INVALID;
     };
     if (tensor) {
-        st = make_map(&L.qmap, query, dtype, head_dim, (int64_t)num_seqs * num_q_heads, G);
+        st = maps.get(&L.qmap, query, dtype, head_dim, (int64_t)num_seqs * num_q_heads, G);
         if (st != PA_OK) return st;
         st = run(true);
         // by default, shapes whose stage ring does not fit (very many
@@ -2040,6 +2045,67 @@ int pa_decode(void* out, const void* query, const void* key_cache, const void* v
     // sequences split into several partitions are merged by a second launch
     if (st == PA_OK && n_pmax > 1) st = launch_merge(L, dtype, head_dim, G, n_pmax);
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                             int max_context_len, int partition_size, size_t* bytes) {
+    if (!bytes || num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_context_len < 0 || partition_size < 0 || (partition_size % TOK) != 0 ||
+        num_q_heads % num_kv_heads != 0)
+        return PA_ERR_INVALID;
+    const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
+    const int n_pmax = std::max(1, (max_context_len + P - 1) / P);
+    *bytes = ws_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, n_pmax);
+    return PA_OK;
+}
+
+int pa_decode_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+    if (!workspace || workspace_bytes < sizeof(WsHeader)) return PA_ERR_INVALID;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, (cudaStream_t)stream) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
+
+int pa_decode_ex(void* out, const void* query, const void* key_cache, const void* value_cache,
+                 const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                 int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads,
+                 int head_dim, int block_size, int num_blocks, float scale, int partition_size,
+                 void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
+                 void* stream, const pa_decode_options* options) {
+    int engine = PA_ENGINE_AUTO, hold = -1;
+    if (options) {
+        if (options->struct_size < (int)sizeof(pa_decode_options)) return PA_ERR_INVALID;
+        engine = options->engine;
+        hold = options->test_withhold_stage;
+        if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_TENSOR || hold < -1) return PA_ERR_INVALID;
+    }
+    if (num_seqs == 0) return PA_OK;
+    int st = validate_args(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                           context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                           head_dim, block_size, num_blocks, partition_size, dtype);
+    if (st == PA_OK)
+        st = validate_workspace(workspace, workspace_bytes, num_seqs, num_q_heads, num_kv_heads,
+                                head_dim, max_context_len, partition_size);
+    if (st != PA_OK) return st;
+    return decode_launch(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                         context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                         head_dim, block_size, num_blocks, scale, partition_size, workspace, dtype,
+                         err_flag, stream, engine, hold);
+}
+
+int pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+              const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+              int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+              int block_size, int num_blocks, float scale, int partition_size, void* workspace,
+              size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag, void* stream) {
+    return pa_decode_ex(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                        context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, scale, partition_size, workspace,
+                        workspace_bytes, dtype, err_flag, stream, nullptr);
 }
 
 }  // extern "C"
@@ -2056,8 +2122,56 @@ namespace {
 constexpr size_t kStaticWsBytes = (size_t)PA_DECODE_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) uint8_t g_static_ws[kStaticWsBytes];
 
+// Device address of g_static_ws per device, with the context it was looked up
+// in: after a device reset the module is loaded again (into a new context) and
+// the array may sit elsewhere, so a different current context means a new
+// lookup rather than a stale address.
+struct StaticWs {
+    void* ctx = nullptr;
+    void* ptr = nullptr;
+};
 std::mutex g_static_mu;
-void* g_static_ptr[64] = {};   // device address of g_static_ws, per device
+StaticWs g_static[64];
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+    });
+    return fn;
+}
+
+// The array's device address on the current device (looked up with that
+// device current, once per device and context); nullptr on a CUDA error.
+void* static_ws_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    auto get_ctx = ctx_get_current_fn();
+    CUcontext ctx = nullptr;
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
+    if (!ctx) {
+        // no context current on this thread yet: cudaSetDevice makes the
+        // device's primary context current (and allocates nothing)
+        if (cudaSetDevice(dev) != cudaSuccess || get_ctx(&ctx) != CUDA_SUCCESS || !ctx)
+            return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    StaticWs& e = g_static[dev];
+    if (!e.ptr || e.ctx != (void*)ctx) {
+        // host code cannot use g_static_ws's name as a device address
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) return nullptr;
+        e.ptr = ptr;
+        e.ctx = (void*)ctx;
+    }
+    return e.ptr;
+}
 
 }  // namespace
 
@@ -2074,25 +2188,18 @@ extern "C" int pa_decode_static(void* out, const void* query, const void* key_ca
                                       max_context_len, partition_size, &need);
     if (st != PA_OK) return st;
     if (need > kStaticWsBytes) return PA_ERR_INVALID;   // larger than the fixed array
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PA_ERR_CUDA;
-    void* ws = nullptr;
-    {
-        // first call on this device (with it current): look up the array's
-        // device address; host code cannot use g_static_ws's name directly
-        std::lock_guard<std::mutex> lk(g_static_mu);
-        if (!g_static_ptr[dev]) {
-            void* ptr = nullptr;
-            if (cudaGetSymbolAddress(&ptr, g_static_ws) != cudaSuccess || !ptr) return PA_ERR_CUDA;
-            g_static_ptr[dev] = ptr;
-        }
-        ws = g_static_ptr[dev];
-    }
+    // every host check before the array is touched: a rejected call launches nothing
+    st = validate_args(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                       context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                       head_dim, block_size, num_blocks, partition_size, dtype);
+    if (st != PA_OK) return st;
+    void* ws = static_ws_ptr();
+    if (!ws) return PA_ERR_CUDA;
     // the scheduler words must start at zero; a call that stopped early
     // (PA_DEV_TIMEOUT) may have left them dirty
     if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
-    return pa_decode(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
-                     context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
-                     head_dim, block_size, num_blocks, scale, partition_size, ws,
-                     kStaticWsBytes, dtype, err_flag, stream);
+    return decode_launch(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                         context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
+                         head_dim, block_size, num_blocks, scale, partition_size, ws, dtype,
+                         err_flag, stream, PA_ENGINE_AUTO, -1);
 }

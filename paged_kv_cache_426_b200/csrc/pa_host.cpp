@@ -205,7 +205,7 @@ const char* pa_status_string(int status) {
     }
 }
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 200; }
 
 int pa_allocator_create(int num_blocks, const int32_t* free_order, int num_free,
                         pa_allocator** out) {

@@ -56,8 +56,9 @@ class CudaPathRun:
     """The CUDA path driven through a workload's script."""
 
     def __init__(self, w, rec: oracle.OracleRun, *, partition_size=None, device="cuda",
-                 max_blocks=None):
+                 max_blocks=None, engine=None):
         self.w = w
+        self.engine = engine          # None: plain pa_decode; else a per-call engine option
         self.dev = device
         self.P = w.partition_size if partition_size is None else partition_size
         self.mb = max_blocks if max_blocks is not None else oracle.max_blocks_needed(w)
@@ -113,7 +114,8 @@ class CudaPathRun:
         q = w.step_q[k].to(dev)
         out = torch.empty_like(q)
         pa.pa_decode(out, q, self.kc, self.vc, tab.to(dev), lens.to(dev), self.max_len, w.scale,
-                     partition_size=self.P, workspace=self.ws, err_flag=self.err)
+                     partition_size=self.P, workspace=self.ws, err_flag=self.err,
+                     engine=self.engine)
         torch.cuda.synchronize()
         assert int(self.err.item()) == 0, f"err_flag {int(self.err.item())}"
         return out

@@ -35,7 +35,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_status_strings_and_version():
     assert pa.lib.pa_status_string(pa.PA_ERR_OOM) == b"PA_ERR_OOM"
-    assert pa.lib.pa_version() >= 100
+    assert pa.lib.pa_version() >= 200
 
 
 def test_bad_arguments_rejected_before_launch():
@@ -63,6 +63,55 @@ def test_bad_arguments_rejected_before_launch():
     # empty work is a no-op
     assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 2, 128, 16, 8, 1, None, None) == pa.PA_OK
     assert L.pa_copy_blocks(None, None, None, 0, 2, 128, 16, 8, 1, None, None) == pa.PA_OK
+
+
+def test_decode_options_are_per_call():
+    """Engine choice and the failure-detection aid are per-call options of
+    pa_decode_ex; the library keeps no process-wide switch for either."""
+    lib = C.CDLL(pa.LIB_PATH)
+    assert not hasattr(lib, "pa_set_decode_engine")
+    assert not hasattr(lib, "pa_test_withhold_stage")
+    L = pa.lib
+    f = 1 << 20                          # aligned, never dereferenced: validation fails first
+
+    def call(opts):
+        return L.pa_decode_ex(f, f, f, f, f, 4, f, 64, 2, 4, 2, 96, 16, 8, 1.0, 0, f, 1 << 20, 1,
+                              None, None, C.byref(opts) if opts is not None else None)
+
+    size = C.sizeof(pa.pa_decode_options)
+    # valid options: the call proceeds to the argument checks (head_dim 96 unsupported)
+    assert call(None) == pa.PA_ERR_UNSUPPORTED
+    assert call(pa.pa_decode_options(size, pa.PA_ENGINE_TENSOR, -1)) == pa.PA_ERR_UNSUPPORTED
+    assert call(pa.pa_decode_options(size, pa.PA_ENGINE_CUDA_CORE, 3)) == pa.PA_ERR_UNSUPPORTED
+    # bad options are rejected first
+    assert call(pa.pa_decode_options(size - 4, 0, -1)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 3, -1)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, -1, -1)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 0, -2)) == pa.PA_ERR_INVALID
+
+
+def test_static_decode_checks_arguments_before_the_device():
+    """pa_decode_static runs every host check of pa_decode before it looks up
+    or clears its fixed array, so a rejected call touches no device state."""
+    L = pa.lib
+    f = 1 << 20
+
+    def call(hq=4, hkv=2, d=128, bs=16, P=0, dt=1, ptr=f, max_len=64, S=2):
+        return L.pa_decode_static(ptr, f, f, f, f, 4, f, max_len, S, hq, hkv, d, bs, 8, 1.0, P,
+                                  dt, None, None)
+
+    assert call(S=0) == pa.PA_OK
+    assert call(d=96) == pa.PA_ERR_UNSUPPORTED
+    assert call(bs=24) == pa.PA_ERR_UNSUPPORTED
+    assert call(hq=6, hkv=2) == pa.PA_ERR_UNSUPPORTED          # G = 3
+    assert call(hq=7, hkv=2) == pa.PA_ERR_INVALID
+    assert call(P=24) == pa.PA_ERR_INVALID
+    assert call(dt=7) == pa.PA_ERR_INVALID
+    assert call(ptr=None) == pa.PA_ERR_INVALID
+    assert call(ptr=f + 8) == pa.PA_ERR_INVALID
+    # larger than the fixed array
+    assert L.pa_decode_static(f, f, f, f, f, 8192, f, 131072, 256, 32, 8, 128, 16, 8, 1.0, 512,
+                              2, None, None) == pa.PA_ERR_INVALID
 
 
 def test_prefill_bad_arguments_rejected_before_launch():

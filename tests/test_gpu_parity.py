@@ -25,25 +25,21 @@ from tests.harness import (CudaPathRun, check_close, oracle_sampled, out_f64, sa
 pytestmark = pytest.mark.gpu
 pa = pytest.importorskip("paged_kv_cache_426_b200")
 
-# auto: tensor cores for 16-bit types with query groups, CUDA cores otherwise
+# auto: tensor cores for 16-bit types, CUDA cores for fp32; each call passes
+# the engine as a per-call option (pa_decode_ex)
 ENGINES = {"auto": 0, "core": 1, "tensor": 2}
-_current = ["auto"]
 
 
 @pytest.fixture(params=list(ENGINES))
 def engine(request):
-    prev = pa.pa_set_decode_engine(ENGINES[request.param])
-    _current[0] = request.param
-    yield request.param
-    _current[0] = "auto"
-    pa.pa_set_decode_engine(prev)
+    return request.param
 
 
-def run_full_compare(w, partition_size=None, steps=None):
-    if _current[0] == "tensor" and w.dtype == "f32":
+def run_full_compare(w, partition_size=None, steps=None, engine="auto"):
+    if engine == "tensor" and w.dtype == "f32":
         pytest.skip("the tensor-core engine takes 16-bit types")
     rec = oracle.run(w, keep_prefill_cache=True, steps=steps)
-    g = CudaPathRun(w, rec, partition_size=partition_size)
+    g = CudaPathRun(w, rec, partition_size=partition_size, engine=engine)
     g.replay_prefill()
     errs = []
     for k in range(len(rec.steps)):
@@ -58,28 +54,28 @@ def run_full_compare(w, partition_size=None, steps=None):
 
 @pytest.mark.parametrize("P", [0, 16, 32])
 def test_tiny_f32(engine, P):
-    run_full_compare(workloads.tiny_f32(), partition_size=P)
+    run_full_compare(workloads.tiny_f32(), partition_size=P, engine=engine)
 
 
 @pytest.mark.parametrize("P", [0, 64, 512])
 def test_mha_f16_small(engine, P):
-    run_full_compare(workloads.mha7b_f16(steps=3, num_seqs=5), partition_size=P)
+    run_full_compare(workloads.mha7b_f16(steps=3, num_seqs=5), partition_size=P, engine=engine)
 
 
 @pytest.mark.parametrize("bs", [16, 32])
 def test_gqa_bf16_small(engine, bs):
-    run_full_compare(workloads.gqa8b_bf16(block_size=bs, num_seqs=10), partition_size=512)
+    run_full_compare(workloads.gqa8b_bf16(block_size=bs, num_seqs=10), partition_size=512, engine=engine)
 
 
 def test_prefix_f16_small(engine):
     w = workloads.prefix_f16(n_req=6, plen=64, suffix_max=40, n_fork=2, heads=4)
-    run_full_compare(w, partition_size=32)
+    run_full_compare(w, partition_size=32, engine=engine)
 
 
 def test_long_bf16_small(engine):
     w = workloads.custom("bf16", [3001, 4096, 1500], 32, 8, 128, 64, seed=77,
                          partition_size=512)
-    run_full_compare(w)
+    run_full_compare(w, engine=engine)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
@@ -89,7 +85,7 @@ def test_shapes_and_groups(engine, dtype, d, G):
     hkv = 2
     w = workloads.custom(dtype, [1, 15, 16, 17, 100, 257], hkv * G, hkv, d, 16, seed=G * d,
                          partition_size=64)
-    run_full_compare(w)
+    run_full_compare(w, engine=engine)
 
 
 @pytest.mark.parametrize("L", [511, 512, 513, 1000])
@@ -98,26 +94,22 @@ def test_split_merge_boundary(engine, L):
     head), from 33 one CTA per (sequence, query head) with sliced partitions:
     both sides of the boundary, with a short sequence in the same batch."""
     w = workloads.custom("bf16", [L, 40], 16, 4, 128, 16, seed=L, partition_size=16)
-    run_full_compare(w)
+    run_full_compare(w, engine=engine)
 
 
 @pytest.mark.parametrize("bs", [8, 16, 32, 64, 128])
 def test_block_sizes(engine, bs):
     w = workloads.custom("f16", [3, 8, 9, 129, 300], 8, 2, 128, bs, seed=bs, partition_size=128)
-    run_full_compare(w)
+    run_full_compare(w, engine=engine)
 
 
 # ---------------------------------------------------------------- invariances
 
 def _decode_outputs(w, P, engine_id=0):
-    prev = pa.pa_set_decode_engine(engine_id)
-    try:
-        rec = oracle.run(w, keep_prefill_cache=True, decode=False)
-        g = CudaPathRun(w, rec, partition_size=P)
-        g.replay_prefill()
-        return [g.step(k).cpu() for k in range(len(rec.steps))], rec
-    finally:
-        pa.pa_set_decode_engine(prev)
+    rec = oracle.run(w, keep_prefill_cache=True, decode=False)
+    g = CudaPathRun(w, rec, partition_size=P, engine=engine_id)
+    g.replay_prefill()
+    return [g.step(k).cpu() for k in range(len(rec.steps))], rec
 
 
 def test_block_size_invariance_bit_identical():
@@ -198,19 +190,15 @@ def test_growing_logits(engine_id, dtype):
     name = "f16" if dtype == torch.float16 else "bf16"
     ref = oracle.paged_decode(oracle.as_storage(q, name), oracle.as_storage(kc, name),
                               oracle.as_storage(vc, name), tab.numpy(), lens.numpy(), 1.0, name)
-    prev = pa.pa_set_decode_engine(engine_id)
-    try:
-        for P in (0, 256):
-            ws = pa.alloc_workspace(1, hkv * G, hkv, d, L, P)
-            out = torch.full_like(q, float("nan")).cuda()
-            err = torch.zeros(1, dtype=torch.int32, device="cuda")
-            pa.pa_decode(out, q.cuda(), kc.cuda(), vc.cuda(), tab.cuda(), lens.cuda(), L, 1.0,
-                         partition_size=P, workspace=ws, err_flag=err)
-            torch.cuda.synchronize()
-            assert err.item() == 0
-            check_close(out_f64(out, name), ref, name, f"growing logits P={P}")
-    finally:
-        pa.pa_set_decode_engine(prev)
+    for P in (0, 256):
+        ws = pa.alloc_workspace(1, hkv * G, hkv, d, L, P)
+        out = torch.full_like(q, float("nan")).cuda()
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        pa.pa_decode(out, q.cuda(), kc.cuda(), vc.cuda(), tab.cuda(), lens.cuda(), L, 1.0,
+                     partition_size=P, workspace=ws, err_flag=err, engine=engine_id)
+        torch.cuda.synchronize()
+        assert err.item() == 0
+        check_close(out_f64(out, name), ref, name, f"growing logits P={P}")
 
 
 # ---------------------------------------------------------------- edge cases
@@ -285,26 +273,22 @@ def test_bad_block_id_tensor_engine():
     ws = pa.alloc_workspace(2, hkv * G, hkv, d, 32, 16)
     out = torch.zeros_like(q)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    prev = pa.pa_set_decode_engine(pa.PA_ENGINE_TENSOR)
-    try:
-        pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
-                     err_flag=err)
-        torch.cuda.synchronize()
-        assert err.item() == pa.PA_DEV_BAD_BLOCK
-        ref = oracle.paged_decode(oracle.as_storage(q.cpu()[1:], "bf16"),
-                                  oracle.as_storage(kc.cpu(), "bf16"),
-                                  oracle.as_storage(vc.cpu(), "bf16"), tab.cpu().numpy()[1:],
-                                  lens.cpu().numpy()[1:], 0.1, "bf16")
-        check_close(out_f64(out[1:], "bf16"), ref, "bf16", "the valid sequence is unaffected")
-        assert torch.isfinite(out[0].float()).all()
-        err.zero_()
-        tab[0, 1] = 3
-        pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
-                     err_flag=err)
-        torch.cuda.synchronize()
-        assert err.item() == 0
-    finally:
-        pa.pa_set_decode_engine(prev)
+    pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
+                 err_flag=err, engine="tensor")
+    torch.cuda.synchronize()
+    assert err.item() == pa.PA_DEV_BAD_BLOCK
+    ref = oracle.paged_decode(oracle.as_storage(q.cpu()[1:], "bf16"),
+                              oracle.as_storage(kc.cpu(), "bf16"),
+                              oracle.as_storage(vc.cpu(), "bf16"), tab.cpu().numpy()[1:],
+                              lens.cpu().numpy()[1:], 0.1, "bf16")
+    check_close(out_f64(out[1:], "bf16"), ref, "bf16", "the valid sequence is unaffected")
+    assert torch.isfinite(out[0].float()).all()
+    err.zero_()
+    tab[0, 1] = 3
+    pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.1, partition_size=16, workspace=ws,
+                 err_flag=err, engine="tensor")
+    torch.cuda.synchronize()
+    assert err.item() == 0
 
 
 def test_bad_length_is_clamped_and_flagged():
@@ -397,24 +381,46 @@ FULL = [
 
 @pytest.mark.slow
 @pytest.mark.parametrize("name,kw", FULL, ids=[f[0] for f in FULL])
-def test_full_size_sampled(name, kw):
-    """Full-size workload, the benchmark's launch configuration (its partition
-    size), every decode step; sampled outputs against the oracle one by one,
-    and the whole caches bit-exact after the last step."""
+def test_full_size(name, kw):
+    """Full-size workload in the benchmark's launch configuration (its
+    partition size), every decode step.  Step 0, every 8th step and the last
+    step are compared element by element (every sequence, query head and
+    column) with the oracle's output computed from the cache as it stands at
+    that step; the other steps on sampled (sequence, head) rows the oracle
+    computes one by one; the whole caches bit-exact after the last step."""
     w = workloads.make(name, **kw)
-    rec = oracle.run(w, keep_prefill_cache=True, decode=False)
+    n = w.num_steps
+    full = {0, n - 1} | set(range(0, n, 8))
+    rec = oracle.run(w, keep_prefill_cache=True, decode_steps=full)
     g = CudaPathRun(w, rec)
     g.replay_prefill()
     S, Hq = rec.steps[0].context_lens.shape[0], w.num_q_heads
     for k in range(len(rec.steps)):
         out = g.step(k)
-        if k in (0, len(rec.steps) - 1) or k % 8 == 0:
+        got = out_f64(out, w.dtype)
+        if k in full:
+            check_close(got, rec.steps[k].out, w.dtype, f"{name} step {k}, every row")
+        elif k % 4 == 0:
             pairs = sample_pairs(S, Hq, 48, seed=k)
-            ref = oracle_sampled(w, rec, k, pairs)
-            got = out_f64(out, w.dtype)
-            for (s, h), r in ref.items():
-                check_close(got[s, h][None, None], r[None, None], w.dtype, f"{name} step {k} ({s},{h})")
+            for (s, h), r in oracle_sampled(w, rec, k, pairs).items():
+                check_close(got[s, h][None, None], r[None, None], w.dtype,
+                            f"{name} step {k} ({s},{h})")
     assert g.caches_equal_oracle()
+
+
+@pytest.mark.parametrize("engine_id", ["auto", "core", "tensor"])
+@pytest.mark.parametrize("dtype,hq,hkv,P", [("bf16", 32, 8, 32), ("f16", 32, 32, 64)])
+def test_many_units_per_cta(engine_id, dtype, hq, hkv, P):
+    """More work units than three per resident CTA (2 x 148 for the tensor-core
+    engine, 148 x pipelines for the CUDA-core one), so every CTA takes several
+    units: the unit ring, the alternating output buffers and the ticket
+    prefetch run through many units.  Element by element against the oracle."""
+    rng = np.random.default_rng(hq + hkv)
+    lens = [int(x) for x in rng.integers(200, 420, size=40)]
+    w = workloads.custom(dtype, lens, hq, hkv, 128, 16, seed=41, partition_size=P, steps=2)
+    units = sum(-(-(L + 1) // P) for L in lens) * hkv
+    assert units > 3 * 296
+    run_full_compare(w, engine=engine_id)
 
 
 # ---------------------------------------------------------------- prefix caching
@@ -481,9 +487,10 @@ def test_prefix_cache_decode_bit_identical():
 @pytest.mark.parametrize("engine_id", [1, 2])
 def test_bounded_wait_reports_timeout(engine_id):
     """Failure detection without a fault: a stage whose barrier nothing will
-    arrive on (test hook pa_test_withhold_stage) makes the waiting warps give
-    up after the 2 s limit; the call returns, err_flag says PA_DEV_TIMEOUT, and
-    the next call on the same workspace and context is correct."""
+    arrive on (per-call option test_withhold_stage of pa_decode_ex) makes the
+    waiting warps give up after the 2 s limit; the call returns, err_flag says
+    PA_DEV_TIMEOUT, and the next call on the same workspace and context is
+    correct."""
     import time
     w = workloads.gqa8b_bf16(num_seqs=6)
     rec = oracle.run(w, keep_prefill_cache=True)
@@ -498,24 +505,17 @@ def test_bounded_wait_reports_timeout(engine_id):
     out = torch.empty_like(q)
     tab_d, lens_d = tab.cuda(), lens.cuda()
 
-    def decode():
+    def decode(hold):
         pa.pa_decode(out, q, g.kc, g.vc, tab_d, lens_d, g.max_len, w.scale, partition_size=512,
-                     workspace=g.ws, err_flag=g.err)
+                     workspace=g.ws, err_flag=g.err, engine=engine_id, test_withhold_stage=hold)
         torch.cuda.synchronize()
 
-    prev = pa.pa_set_decode_engine(engine_id)
-    try:
-        pa.lib.pa_test_withhold_stage(0)
-        t0 = time.time()
-        decode()
-        dt = time.time() - t0
-        assert int(g.err.item()) == pa.PA_DEV_TIMEOUT
-        assert 1.0 < dt < 30.0
-        pa.lib.pa_test_withhold_stage(-1)
-        g.err.zero_()
-        decode()
-        assert int(g.err.item()) == 0
-        check_close(out_f64(out, w.dtype), st.out, w.dtype, "the call after a timed-out one")
-    finally:
-        pa.lib.pa_test_withhold_stage(-1)
-        pa.pa_set_decode_engine(prev)
+    t0 = time.time()
+    decode(0)
+    dt = time.time() - t0
+    assert int(g.err.item()) == pa.PA_DEV_TIMEOUT
+    assert 1.0 < dt < 30.0
+    g.err.zero_()
+    decode(-1)
+    assert int(g.err.item()) == 0
+    check_close(out_f64(out, w.dtype), st.out, w.dtype, "the call after a timed-out one")

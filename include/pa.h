@@ -101,9 +101,11 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * fp32 accumulation; out is rounded to nearest even in dtype.  L = 0 gives 0.
  * Long contexts are split into partitions of `partition_size` tokens
  * (a positive multiple of 16; 0 = one partition per sequence) whose partial
- * results are merged with their log-sum-exp weights by a second kernel that
- * pa_decode launches on the same stream when ceil(max_context_len /
- * partition_size) > 1; otherwise one call is one launch.
+ * results are merged with their log-sum-exp weights.  With the tensor-core
+ * engine and ceil(max_context_len / partition_size) <= 16 the work unit that
+ * completes a split sequence merges it inside the decode kernel (one launch
+ * per call); otherwise, when ceil(max_context_len / partition_size) > 1, a
+ * second kernel on the same stream merges (two launches).
  *   out           device [num_seqs][num_q_heads][head_dim] dtype
  *   query         device [num_seqs][num_q_heads][head_dim] dtype, 16-B aligned
  *   block_tables  device int32 [num_seqs][max_blocks_per_seq]; entries past
@@ -113,7 +115,8 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  *   workspace     device, >= pa_decode_workspace_size() bytes, 256-B aligned;
  *                 must be zero-filled before its first use (see
  *                 pa_decode_workspace_init); every call leaves its scheduler
- *                 words zero again.  Calls sharing one workspace must not
+ *                 words and split counters zero again, also after a
+ *                 PA_DEV_TIMEOUT.  Calls sharing one workspace must not
  *                 overlap on the GPU.
  * The physical placement of blocks does not change the result: summation
  * order depends only on logical token positions.

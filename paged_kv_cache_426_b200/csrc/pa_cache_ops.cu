@@ -21,6 +21,10 @@ reshape_and_cache_kernel(const uint4* __restrict__ key, const uint4* __restrict_
                          uint4* __restrict__ key_cache, uint4* __restrict__ value_cache,
                          const int64_t* __restrict__ slots, int64_t total, int row_vecs, int Hkv,
                          int bs, int64_t num_slots, int32_t* err) {
+    // launched as a programmatic dependent of the kernel before it (e.g. the
+    // previous step's decode, which may still read the cache): its blocks may
+    // be resident early, but nothing is touched before that kernel completes
+    grid_dependency_wait();
     // a decode launched after this kernel may be scheduled now; it waits on
     // the device for this grid's writes before it reads the cache
     launch_dependents();
@@ -104,11 +108,25 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache, vo
     const int row_vecs = head_dim * (int)dtype_size(dtype) / 16;
     const int64_t total = (int64_t)num_tokens * num_kv_heads * row_vecs;
     const int64_t blocks = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
-    reshape_and_cache_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
-        static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), slot_mapping, total,
-        row_vecs, num_kv_heads, block_size, (int64_t)num_blocks * block_size, err_flag);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    // programmatic dependent launch: the grid's launch overlaps the tail of
+    // the kernel before it; the kernel waits (griddepcontrol.wait) for that
+    // kernel to complete before its first global access
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = (cudaStream_t)stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(
+        &cfg, reshape_and_cache_kernel, static_cast<const uint4*>(key),
+        static_cast<const uint4*>(value), static_cast<uint4*>(key_cache),
+        static_cast<uint4*>(value_cache), slot_mapping, total, row_vecs, num_kv_heads, block_size,
+        (int64_t)num_blocks * block_size, err_flag);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int num_pairs,

@@ -75,7 +75,8 @@ struct alignas(16) UnitDesc {
 struct alignas(16) WsHeader {
     int next_unit;   // dynamic scheduler ticket
     int done_ctas;   // CTAs finished; the last one re-zeroes both
-    int pad[62];
+    int dirty;       // a CTA gave up: the last CTA re-zeroes the split counters too
+    int pad[61];
 };
 
 struct DecodeParams {
@@ -89,6 +90,8 @@ struct DecodeParams {
     int hold_stage;    // test hook: stage of unit 0 that its producer withholds (-1: none)
     float* part_ml;    // [S*Hkv][n_pmax][G][2]
     float* part_o;     // [S*Hkv][n_pmax][G][D]
+    int* split_cnt;    // [S*Hkv] partitions of a split (sequence, KV head) finished so far
+    int fused_merge;   // the unit finishing a split last merges it (no merge kernel)
     int32_t* err;
 };
 
@@ -634,6 +637,33 @@ __device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
 // spread over thread slices, so no thread walks a long chain of loads.
 constexpr int MERGE_THREADS = 256;
 constexpr int kShortSplit = 32;     // partitions up to which the group shape is used
+constexpr int kFusedSplit = 16;     // partitions up to which the decode kernel merges itself
+
+// Column dd of the G heads' outputs of (sequence s, KV head j) from the n_p
+// partials, in partition order (the same arithmetic as the merge kernels).
+// Reads through L2 only: other CTAs wrote the partials.
+template <typename T, int D, int G>
+__device__ __forceinline__ void merge_column(const DecodeParams& p, int s, int j, int dd, int n_p) {
+    const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        float M = -INFINITY;
+#pragma unroll 4
+        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + h) * 2));
+        float acc = 0.f, Lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 4
+            for (int i = 0; i < n_p; ++i) {
+                const size_t pi = (base + i) * G + h;
+                const float w = exp2f(__ldcg(p.part_ml + pi * 2) - M);
+                Lsum += w * __ldcg(p.part_ml + pi * 2 + 1);
+                acc += w * __ldcg(p.part_o + pi * D + dd);
+            }
+        }
+        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h) * D + dd;
+        *outp = DT<T>::from_float(acc * (Lsum > 0.f ? 1.f / Lsum : 0.f));
+    }
+}
 
 template <typename T, int D>
 __device__ __forceinline__ void merge_store(const DecodeParams& p, int s, int h, int col, float4 o, float inv) {
@@ -1275,6 +1305,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     volatile int* abort_flag = misc + 0;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 60);   // outside the zeroed words
     int* wsum = misc + 32;
+    volatile int* last_flag = misc + 48;     // epilogue: this unit completes its split
 
     if (tid == 0) {
         const int n = 2 * nst + LY::NBAR;
@@ -1632,7 +1663,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         *outp = DT<T>::from_float(lh[h] > 0.f ? o[h] / lh[h] : 0.f);
                     }
             } else {
-                // partials for the merge kernel
+                // partials: for the merge kernel, or (fused_merge) for the unit
+                // that finishes this (sequence, KV head) last
                 if (dd >= 0)
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
@@ -1643,6 +1675,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                             p.part_ml[pi * 2 + 1] = lh[h];
                         }
                     }
+                if (p.fused_merge) {
+                    // release this unit's partials, then count it; the count
+                    // that completes the split makes this group the merger
+                    __threadfence();
+                    named_bar_sync(BAR_EPI, 128);
+                    if (et == 0) *last_flag = atomicAdd(p.split_cnt + sj, 1) == n_p - 1;
+                    named_bar_sync(BAR_EPI, 128);
+                    if (*last_flag) {
+                        __threadfence();                 // acquire the other units' partials
+                        if (dd >= 0) merge_column<T, D, G>(p, s, j, dd, n_p);
+                        if (et == 0) p.split_cnt[sj] = 0;   // the next call starts at zero
+                    }
+                }
             }
             ++ucount;
         }
@@ -1657,9 +1702,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         tc::dealloc(tmem, LY::TM_COLS);
     }
     if (tid == 0) {
+        if (*abort_flag) atomicExch(&p.hdr->dirty, 1);   // split counters may be left partial
         __threadfence();
         const int done = atomicAdd(&p.hdr->done_ctas, 1);
         if (done == (int)gridDim.x - 1) {
+            if (atomicAdd(&p.hdr->dirty, 0) && p.fused_merge) {
+                for (int k = 0; k < p.S * p.Hkv; ++k) p.split_cnt[k] = 0;
+                p.hdr->dirty = 0;
+            }
             p.hdr->next_unit = 0;
             p.hdr->done_ctas = 0;
             __threadfence();
@@ -1765,12 +1815,17 @@ int dev_info(DevInfo* out) {
 constexpr int kMaxStages = 8;     // stages per pipeline
 constexpr int kMinStages = 2;     // any count >= 1 is correct; fewer only slows the pipeline
 
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Workspace: the scheduler header; when sequences can be split, the split
+// counters [S*Hkv] int, the (m, l) pairs and the unnormalised outputs of every
+// partition of every query head.
+size_t ws_counters(int S, int Hkv) { return round256((size_t)S * Hkv * 4); }
+size_t ws_ml(int S, int Hq, int n_pmax) { return round256((size_t)S * Hq * n_pmax * 2 * 4); }
 size_t ws_bytes(int S, int Hq, int Hkv, int D, int n_pmax) {
     size_t b = sizeof(WsHeader);
-    if (n_pmax > 1) {
-        b += (((size_t)S * Hq * n_pmax * 2 * 4 + 255) / 256) * 256;
-        b += (size_t)S * Hq * n_pmax * D * 4;
-    }
+    if (n_pmax > 1)
+        b += ws_counters(S, Hkv) + ws_ml(S, Hq, n_pmax) + (size_t)S * Hq * n_pmax * D * 4;
     return b;
 }
 
@@ -1837,6 +1892,7 @@ template <typename T, int D, int G>
 int run_decode_core(Launch& L, const DevInfo& di) {
     using LY = Layout<T, D, G, cons_for<G>()>;
     auto kern = decode_kernel<T, D, G>;
+    L.p.fused_merge = 0;     // the CUDA-core engine leaves splits to the merge kernel
     const size_t per_stage = (size_t)LY::NPIPE * (LY::STAGE_BYTES + 2 * 8 + 4);
     int st = pick_stages<LY>(L, (size_t)di.smem_optin, per_stage, &L.p.nst, &L.smem);
     if (st != PA_OK) return st;
@@ -1853,6 +1909,8 @@ int run_decode_tc(Launch& L, const DevInfo& di) {
     } else {
         using LY = TcLayout<T, D, G>;
         auto kern = decode_tc_kernel<T, D, G>;
+        // short splits are merged by the unit that completes them
+        L.p.fused_merge = (L.p.n_pmax > 1 && L.p.n_pmax <= kFusedSplit) ? 1 : 0;
         // two CTAs per SM: each gets half of the SM's shared memory (less the
         // 1 KB the system reserves per CTA)
         const size_t budget = std::min<size_t>((size_t)di.smem_optin, (size_t)di.smem_sm / 2 - 1024);
@@ -2009,8 +2067,10 @@ int decode_launch(void* out, const void* query, const void* key_cache, const voi
     p.scale_log2e = scale * 1.4426950408889634f;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.hdr = reinterpret_cast<WsHeader*>(ws);
-    p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader));
-    p.part_o = p.part_ml + ((((size_t)num_seqs * num_q_heads * n_pmax * 2 * 4 + 255) / 256) * 256) / 4;
+    p.split_cnt = reinterpret_cast<int*>(ws + sizeof(WsHeader));
+    p.part_ml = reinterpret_cast<float*>(ws + sizeof(WsHeader) + ws_counters(num_seqs, num_kv_heads));
+    p.part_o = p.part_ml + ws_ml(num_seqs, num_q_heads, n_pmax) / 4;
+    p.fused_merge = 0;       // set by the engine that takes it
     p.err = err_flag;
     p.hold_stage = hold_stage;
 
@@ -2042,8 +2102,9 @@ int decode_launch(void* out, const void* query, const void* key_cache, const voi
     } else {
         st = run(false);
     }
-    // sequences split into several partitions are merged by a second launch
-    if (st == PA_OK && n_pmax > 1) st = launch_merge(L, dtype, head_dim, G, n_pmax);
+    // sequences split into several partitions are merged by a second launch,
+    // unless the decode kernel merged them itself
+    if (st == PA_OK && n_pmax > 1 && !L.p.fused_merge) st = launch_merge(L, dtype, head_dim, G, n_pmax);
     return st;
 }
 
@@ -2195,9 +2256,13 @@ extern "C" int pa_decode_static(void* out, const void* query, const void* key_ca
     if (st != PA_OK) return st;
     void* ws = static_ws_ptr();
     if (!ws) return PA_ERR_CUDA;
-    // the scheduler words must start at zero; a call that stopped early
-    // (PA_DEV_TIMEOUT) may have left them dirty
-    if (cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
+    // the scheduler words and split counters must start at zero; the array
+    // keeps whatever the last call left (a call that stopped early with
+    // PA_DEV_TIMEOUT, or one of other sizes, may have left them dirty)
+    const int P = partition_size > 0 ? partition_size : std::max(TOK, max_context_len);
+    const int n_pmax = std::max(1, (max_context_len + P - 1) / P);
+    const size_t clear = sizeof(WsHeader) + (n_pmax > 1 ? ws_counters(num_seqs, num_kv_heads) : 0);
+    if (cudaMemsetAsync(ws, 0, clear, (cudaStream_t)stream) != cudaSuccess) return PA_ERR_CUDA;
     return decode_launch(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                          context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
                          head_dim, block_size, num_blocks, scale, partition_size, ws, dtype,

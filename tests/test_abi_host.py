@@ -148,10 +148,14 @@ def test_workspace_size_formula():
     # the scheduler header only when nothing is split
     n0 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 0)
     assert n0 == 256
-    # + (m, l) and the unnormalised output of every partition of every head
+    # + a split counter per (sequence, KV head), (m, l) and the unnormalised
+    # output of every partition of every head, each part rounded up to 256 bytes
     n1 = pa.pa_decode_workspace_size(64, 32, 32, 128, 2080, 512)
     n_p = 5
-    assert n1 == 256 + 64 * 32 * n_p * 2 * 4 + 64 * 32 * n_p * 128 * 4
+    assert n1 == 256 + 64 * 32 * 4 + 64 * 32 * n_p * 2 * 4 + 64 * 32 * n_p * 128 * 4
+    n2 = pa.pa_decode_workspace_size(3, 8, 2, 64, 100, 16)
+    r = lambda b: -(-b // 256) * 256
+    assert n2 == 256 + r(3 * 2 * 4) + r(3 * 8 * 7 * 2 * 4) + 3 * 8 * 7 * 64 * 4
 
 
 def test_allocator_errors():

@@ -279,7 +279,9 @@ int pa_allocator_num_free(const pa_allocator* a, int32_t* num_free);
  * block is shared (count > 1) it is first replaced by a fresh block, the pair
  * (old, new) is reported for pa_copy_blocks and the old block loses one
  * reference.  slot = table[p / bs] * bs + p % bs.  Appends are all-or-nothing:
- * PA_ERR_OOM leaves every table and count unchanged.
+ * PA_ERR_OOM leaves every table and count unchanged, except that with the
+ * prefix cache on, cached blocks that the call evicted to find room stay
+ * evicted (they are back in the free pool; their cache entries are gone).
  *   pa_manager_append       num_tokens tokens to one sequence; slots[num_tokens];
  *                           cow_pairs int64 [>=1][2], *num_cow in {0,1}
  *   pa_manager_append_step  one token to each of seq_ids[0..n); slots[n];
@@ -317,7 +319,11 @@ int pa_manager_block_tables(const pa_manager* m, const int64_t* seq_ids,
  *                    token prefix up to its end matches: a 64-bit fingerprint
  *                    chained over the blocks, plus an exact comparison of the
  *                    block's own ids) until the first miss; hits are shared
- *                    (incref).  The remaining tokens are appended as usual and
+ *                    (incref).  The block holding the prompt's last token is
+ *                    never served from the cache (a prompt of whole blocks
+ *                    looks up all but its last), so *num_cached < num_tokens
+ *                    for any non-empty prompt and at least the last token is
+ *                    left to compute.  The remaining tokens are appended as usual and
  *                    every full block they fill is cached.  slots[n]: -1 for
  *                    the *num_cached leading tokens served from the cache
  *                    (pa_reshape_and_cache skips them), the slot otherwise; so

@@ -109,9 +109,10 @@ class BlockManager:
     # tuples of the whole prefix up to each block's end.  Reading of what the
     # pages leave open (the plainest one): the cache keeps one reference per
     # cached block; only full prompt blocks are cached, one block per prefix;
-    # lookup walks the leading full blocks until the first miss; when the free
-    # pool is empty the least recently used cached block that nothing else
-    # references is freed first.
+    # lookup walks the leading full blocks until the first miss and never
+    # serves the block holding the prompt's last token (that token must be
+    # computed); when the free pool is empty the least recently used cached
+    # block that nothing else references is freed first.
     def enable_prefix_cache(self) -> None:
         if self.tables:
             raise BlockStateError("enable the cache before adding sequences")
@@ -140,8 +141,12 @@ class BlockManager:
         bs, n = self.bs, len(tokens)
         self.add_seq(seq)
         table = self.tables[seq]
+        # the last prompt token is always computed (the first generated token
+        # needs its attention output), so a prompt of whole blocks looks up
+        # all but its last block
         hit, full = 0, n // bs
-        while hit < full:
+        lookable = (n - 1) // bs if n else 0
+        while hit < lookable:
             b = self.cache.get(tuple(tokens[:(hit + 1) * bs]))
             if b is None:
                 break

@@ -170,8 +170,11 @@ int append_one(pa_manager* m, pa_manager::Seq& s, int64_t* slot, Undo* u,
 
 // Reverse one append (applied newest first).  A block this append took is
 // still referenced only by this sequence, so it goes back to the front of the
-// pool; undoing newest first restores the pool's exact order.  A copy never
-// sends its source to the pool (its count was above 1), so nothing else moved.
+// pool; undoing newest first restores the pool's order as the appends found
+// it.  A copy never sends its source to the pool (its count was above 1).
+// With the prefix cache on, taking a block may first have evicted cached
+// blocks (have_free); those evictions are not reversed: the blocks stay in the
+// pool and their cache entries are gone.
 void undo_one(pa_manager* m, const Undo& u) {
     pa_allocator* a = m->alloc;
     pa_manager::Seq& s = *u.seq;
@@ -409,11 +412,15 @@ int pa_manager_add_seq_prompt(pa_manager* m, int64_t seq_id, const int32_t* toke
     pa_allocator* a = m->alloc;
     const int bs = m->block_size;
     pa_manager::Seq s;
-    // 1. the longest run of leading full blocks already cached
+    // 1. the longest run of leading full blocks already cached, leaving at
+    // least the prompt's last token to compute (its attention output is what
+    // the first generated token needs): a prompt that is a whole number of
+    // blocks looks up all but its last block
     uint64_t parent = 0;
     int hit = 0;
     const int full = num_tokens / bs;
-    for (; hit < full; ++hit) {
+    const int lookable = num_tokens > 0 ? (num_tokens - 1) / bs : 0;
+    for (; hit < lookable; ++hit) {
         const int32_t* t = tokens + static_cast<int64_t>(hit) * bs;
         const uint64_t key = block_key(parent, t, bs);
         const int32_t found = lookup(m, key, parent, t);

@@ -47,6 +47,33 @@ def test_golden_scenario_oracle():
     assert sorted(m.cache_of) == [0, 1, 2, 3, 4, 5, 6, 7]
 
 
+def test_whole_block_prompt_keeps_its_last_token_to_compute():
+    """A prompt that is a whole number of blocks, every one of them cached:
+    all but the last block are served from the cache; the last block is taken
+    fresh and written (its prefix is cached already, so it is not cached
+    again), so the prompt's last token is computed and the first generated
+    token has its attention input.  Worked by hand from the rules."""
+    alloc = oracle.BlockAllocator(6)
+    m = oracle.BlockManager(alloc, 4)
+    m.enable_prefix_cache()
+    assert m.add_seq_prompt(0, range(1, 9)) == (list(range(8)), 0)     # blocks 0, 1 cached
+    slots, cached = m.add_seq_prompt(1, range(1, 9))
+    assert cached == 4 and slots == [-1] * 4 + [8, 9, 10, 11]       # block 2, fresh
+    assert m.tables[1] == [0, 2] and alloc.refcount[:3] == [3, 2, 1]
+    assert m.cache_stats == dict(hits=1, misses=3, evictions=0)
+    assert sorted(m.cache_of) == [0, 1]
+    # a prompt of one whole block: nothing is served
+    assert m.add_seq_prompt(2, range(1, 5)) == ([12, 13, 14, 15], 0)
+    # the library's manager does the same
+    ca, cm = _cpp(6, 4)
+    cm.add_seq_prompt(0, range(1, 9))
+    slots, cached = cm.add_seq_prompt(1, range(1, 9))
+    assert cached == 4 and slots.tolist() == [-1] * 4 + [8, 9, 10, 11]
+    assert [ca.refcount(b) for b in range(3)] == [3, 2, 1]
+    slots, cached = cm.add_seq_prompt(2, range(1, 5))
+    assert cached == 0 and slots.tolist() == [12, 13, 14, 15]
+
+
 def _cpp(num_blocks, bs):
     a = pa.BlockAllocator(num_blocks)
     m = pa.BlockManager(a, bs)
@@ -134,7 +161,7 @@ def test_failed_prompt_leaves_cache_and_pool_unchanged():
     assert e.value.status == pa.PA_ERR_OOM
     assert (ca.num_free(), cm.prefix_cache_stats()) == before
     slots, cached = cm.add_seq_prompt(2, range(8))   # the survivors still hit
-    assert cached == 8 and slots.tolist() == [-1] * 8
+    assert cached == 4 and slots.tolist()[:4] == [-1] * 4   # (the last block is computed)
 
 
 def test_enable_after_sequences_is_a_state_error():

@@ -637,32 +637,60 @@ __device__ void producer_loop(const CUtensorMap* kmap, const CUtensorMap* vmap,
 // spread over thread slices, so no thread walks a long chain of loads.
 constexpr int MERGE_THREADS = 256;
 constexpr int kShortSplit = 32;     // partitions up to which the group shape is used
-constexpr int kFusedSplit = 16;     // partitions up to which the decode kernel merges itself
 
-// Column dd of the G heads' outputs of (sequence s, KV head j) from the n_p
-// partials, in partition order (the same arithmetic as the merge kernels).
-// Reads through L2 only: other CTAs wrote the partials.
+// Column dd of the G heads' outputs of (sequence s, KV head j) from its
+// n_p <= fused_parts<G>() partials, in partition order (the same arithmetic as
+// the merge kernels: exact zeros stand in for partitions past n_p).  All loads
+// of a batch of heads are issued before any is used, so a merge costs one or
+// two round trips to L2 rather than one per partition.  Reads through L2
+// only: other CTAs wrote the partials.
+template <int G> constexpr int fused_parts() { return G <= 2 ? 16 : 32 / G; }
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_column(const DecodeParams& p, int s, int j, int dd, int n_p) {
+    constexpr int NI = fused_parts<G>();
+    constexpr int HB = 16 / NI;                   // heads per batch: 16 (m, l, o) loads in flight
     const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-        float M = -INFINITY;
-#pragma unroll 4
-        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + h) * 2));
-        float acc = 0.f, Lsum = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll 4
-            for (int i = 0; i < n_p; ++i) {
-                const size_t pi = (base + i) * G + h;
-                const float w = exp2f(__ldcg(p.part_ml + pi * 2) - M);
-                Lsum += w * __ldcg(p.part_ml + pi * 2 + 1);
-                acc += w * __ldcg(p.part_o + pi * D + dd);
+    for (int h0 = 0; h0 < G; h0 += HB) {
+        float2 ml[HB][NI];
+        float o[HB][NI];
+#pragma unroll
+        for (int hh = 0; hh < HB; ++hh)
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                const size_t pi = (base + i) * G + h0 + hh;
+                ml[hh][i] = i < n_p ? __ldcg(reinterpret_cast<const float2*>(p.part_ml) + pi)
+                                    : make_float2(-INFINITY, 0.f);
+                o[hh][i] = i < n_p ? __ldcg(p.part_o + pi * D + dd) : 0.f;
             }
+#pragma unroll
+        for (int hh = 0; hh < HB; ++hh) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < NI; ++i) M = fmaxf(M, ml[hh][i].x);
+            float acc = 0.f, Lsum = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int i = 0; i < NI; ++i) {
+                    const float w = exp2f(ml[hh][i].x - M);
+                    Lsum += w * ml[hh][i].y;
+                    acc += w * o[hh][i];
+                }
+            }
+            T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h0 + hh) * D + dd;
+            *outp = DT<T>::from_float(acc * (Lsum > 0.f ? 1.f / Lsum : 0.f));
         }
-        T* outp = reinterpret_cast<T*>(p.out) + ((size_t)s * p.Hq + (size_t)j * G + h) * D + dd;
-        *outp = DT<T>::from_float(acc * (Lsum > 0.f ? 1.f / Lsum : 0.f));
     }
+}
+
+// atomicAdd with release and acquire semantics at GPU scope: the partials this
+// CTA wrote (ordered before by a barrier) are visible to whoever sees the new
+// count, and the partials of the units counted before are visible here.
+__device__ __forceinline__ int atomic_add_acq_rel(int* addr, int v) {
+    int old;
+    asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v)
+                 : "memory");
+    return old;
 }
 
 template <typename T, int D>
@@ -1676,14 +1704,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         }
                     }
                 if (p.fused_merge) {
-                    // release this unit's partials, then count it; the count
-                    // that completes the split makes this group the merger
-                    __threadfence();
+                    // count this unit once all 128 threads' partials are
+                    // written (barrier, then one release-acquire atomic); the
+                    // count that completes the split makes this group the
+                    // merger, and it sees every other unit's partials
                     named_bar_sync(BAR_EPI, 128);
-                    if (et == 0) *last_flag = atomicAdd(p.split_cnt + sj, 1) == n_p - 1;
+                    if (et == 0) *last_flag = atomic_add_acq_rel(p.split_cnt + sj, 1) == n_p - 1;
                     named_bar_sync(BAR_EPI, 128);
                     if (*last_flag) {
-                        __threadfence();                 // acquire the other units' partials
                         if (dd >= 0) merge_column<T, D, G>(p, s, j, dd, n_p);
                         if (et == 0) p.split_cnt[sj] = 0;   // the next call starts at zero
                     }
@@ -1910,7 +1938,7 @@ int run_decode_tc(Launch& L, const DevInfo& di) {
         using LY = TcLayout<T, D, G>;
         auto kern = decode_tc_kernel<T, D, G>;
         // short splits are merged by the unit that completes them
-        L.p.fused_merge = (L.p.n_pmax > 1 && L.p.n_pmax <= kFusedSplit) ? 1 : 0;
+        L.p.fused_merge = (L.p.n_pmax > 1 && L.p.n_pmax <= fused_parts<G>()) ? 1 : 0;
         // two CTAs per SM: each gets half of the SM's shared memory (less the
         // 1 KB the system reserves per CTA)
         const size_t budget = std::min<size_t>((size_t)di.smem_optin, (size_t)di.smem_sm / 2 - 1024);

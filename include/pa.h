@@ -82,7 +82,10 @@ int pa_version(void);
  * PA_DEV_BAD_SLOT and is skipped.
  *   key, value    device [num_tokens][num_kv_heads][head_dim] dtype, contiguous
  *   slot_mapping  device int64 [num_tokens]; distinct non-negative entries
- * Bit copy: the cache holds exactly the input bits.
+ * Bit copy: the cache holds exactly the input bits.  The kernel is a
+ * programmatic dependent of the kernel before it in the stream and touches
+ * memory only after that kernel has completed; it lets the kernel after it
+ * (pa_decode, pa_prefill) start early.
  */
 int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
                          void* value_cache, const int64_t* slot_mapping,
@@ -120,6 +123,13 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  *                 overlap on the GPU.
  * The physical placement of blocks does not change the result: summation
  * order depends only on logical token positions.
+ * Launch order: the decode kernel is a programmatic dependent of the kernel
+ * before it in the stream.  It may read context_lens before that kernel has
+ * completed if that kernel lets dependents start early
+ * (griddepcontrol.launch_dependents); everything else (queries, tables,
+ * cache, workspace, every write) waits for its completion.  Of this
+ * library's kernels only pa_reshape_and_cache starts dependents early, and
+ * it does not write context_lens.
  */
 int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                              int head_dim, int max_context_len,

@@ -1176,6 +1176,10 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
     // unit's plan, whose block-table loads are then in flight, is prepared as
     // soon as the current unit's first stage is issued.
     int gstage = 0, st = 0, round = 0, ucount = 0, t0 = 0, t1 = 0, t2 = 0;
+    // The kernel before this one has completed and its writes are visible:
+    // the cache may be read, and the scheduler ticket is free (a decode call
+    // just before on the same workspace has reset it).
+    grid_dependency_wait();
     if (lane == 0) {
         t0 = atomicAdd(&p.hdr->next_unit, 1);
         t1 = atomicAdd(&p.hdr->next_unit, 1);
@@ -1357,7 +1361,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
-    grid_dependency_wait();              // inputs written by the previous kernel are visible
+    // Launched as a programmatic dependent of the kernel before it (the cache
+    // write): the lengths may be read and the unit order computed while that
+    // kernel still runs (it writes only the cache); everything else - the
+    // scheduler ticket, tables, queries, the cache, and every write - waits
+    // for griddepcontrol.wait (the producer's first step, every other warp's
+    // before its loop).
     schedule_units<TC_THREADS>(p, lens_s, preF, order, reinterpret_cast<int*>(smem + ly.sched()), wsum, tid);
     tc::fence_before();
     __syncthreads();
@@ -1368,6 +1377,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     const int U = (preF[p.S] + p.S) * p.Hkv;
     const int PR = p.bs >= 16 ? 16 : p.bs;
 
+    if (warp != 8) grid_dependency_wait();
     if (warp == 8) {
         // ================================================= producer warp
         producer_tc<T, D, G>(&kmap, &vmap, &qmap, p, smem, ly, full, empty, ufull, uempty,

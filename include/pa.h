@@ -124,12 +124,12 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * The physical placement of blocks does not change the result: summation
  * order depends only on logical token positions.
  * Launch order: the decode kernel is a programmatic dependent of the kernel
- * before it in the stream.  It may read context_lens before that kernel has
- * completed if that kernel lets dependents start early
- * (griddepcontrol.launch_dependents); everything else (queries, tables,
- * cache, workspace, every write) waits for its completion.  Of this
- * library's kernels only pa_reshape_and_cache starts dependents early, and
- * it does not write context_lens.
+ * before it in the stream.  It may read context_lens and block_tables before
+ * that kernel has completed if that kernel lets dependents start early
+ * (griddepcontrol.launch_dependents); everything else (queries, cache,
+ * workspace, every write) waits for its completion.  Of this library's
+ * kernels only pa_reshape_and_cache starts dependents early, and it writes
+ * neither.
  */
 int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                              int head_dim, int max_context_len,

@@ -1174,18 +1174,20 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
     // Latency hiding at unit boundaries: lane 0 holds the tickets of the two
     // units after the current one (each fetched two units ahead), and the next
     // unit's plan, whose block-table loads are then in flight, is prepared as
-    // soon as the current unit's first stage is issued.
-    int gstage = 0, st = 0, round = 0, ucount = 0, t0 = 0, t1 = 0, t2 = 0;
+    // soon as the current unit's first stage is issued.  A CTA's first unit is
+    // its own index (the largest units, one per CTA), planned - block-table
+    // reads included - before the dependency wait; later units come from the
+    // ticket counter, which hands out gridDim.x onwards.
+    int gstage = 0, st = 0, round = 0, ucount = 0, t1 = 0, t2 = 0;
+    Plan cur = prepare((int)blockIdx.x);
     // The kernel before this one has completed and its writes are visible:
     // the cache may be read, and the scheduler ticket is free (a decode call
     // just before on the same workspace has reset it).
     grid_dependency_wait();
     if (lane == 0) {
-        t0 = atomicAdd(&p.hdr->next_unit, 1);
-        t1 = atomicAdd(&p.hdr->next_unit, 1);
-        t2 = atomicAdd(&p.hdr->next_unit, 1);
+        t1 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
+        t2 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
     }
-    Plan cur = prepare(__shfl_sync(FULL, t0, 0));
     bool ok = true;
     while (ok) {
         const int slot = ucount % NU;
@@ -1222,7 +1224,7 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
             have_next = true;
             if (lane == 0) {
                 t1 = t2;
-                t2 = atomicAdd(&p.hdr->next_unit, 1);
+                t2 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
             }
         };
         int win = 0;
@@ -1362,11 +1364,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&qmap);
     }
     // Launched as a programmatic dependent of the kernel before it (the cache
-    // write): the lengths may be read and the unit order computed while that
-    // kernel still runs (it writes only the cache); everything else - the
-    // scheduler ticket, tables, queries, the cache, and every write - waits
-    // for griddepcontrol.wait (the producer's first step, every other warp's
-    // before its loop).
+    // write): the lengths may be read, the unit order computed and the first
+    // unit's block-table entries read while that kernel still runs (it writes
+    // only the cache); the scheduler ticket, the queries, the cache and every
+    // write wait for griddepcontrol.wait (in the producer before its first
+    // ticket and copy, in every other warp before its loop).
     schedule_units<TC_THREADS>(p, lens_s, preF, order, reinterpret_cast<int*>(smem + ly.sched()), wsum, tid);
     tc::fence_before();
     __syncthreads();

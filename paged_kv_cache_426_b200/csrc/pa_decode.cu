@@ -641,10 +641,10 @@ constexpr int kShortSplit = 32;     // partitions up to which the group shape is
 // Column dd of the G heads' outputs of (sequence s, KV head j) from its
 // n_p <= fused_parts<G>() partials, in partition order (the same arithmetic as
 // the merge kernels: exact zeros stand in for partitions past n_p).  All loads
-// of a batch of heads are issued before any is used, so a merge costs one or
-// two round trips to L2 rather than one per partition.  Reads through L2
+// of a batch of heads (16 partials) are issued before any is used, so a merge
+// costs G * NI / 16 round trips to L2 rather than one per partition.  Reads through L2
 // only: other CTAs wrote the partials.
-template <int G> constexpr int fused_parts() { return G <= 2 ? 16 : 32 / G; }
+template <int G> constexpr int fused_parts() { return G <= 4 ? 16 : 4; }
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_column(const DecodeParams& p, int s, int j, int dd, int n_p) {
     constexpr int NI = fused_parts<G>();

@@ -642,9 +642,12 @@ constexpr int kShortSplit = 32;     // partitions up to which the group shape is
 // n_p <= fused_parts<G>() partials, in partition order (the same arithmetic as
 // the merge kernels: exact zeros stand in for partitions past n_p).  All loads
 // of a batch of heads (16 partials) are issued before any is used, so a merge
-// costs G * NI / 16 round trips to L2 rather than one per partition.  Reads through L2
+// costs G * NI / 16 round trips to L2 rather than one per partition.  Only
+// short splits are merged this way: the merging unit's epilogue holds its CTA
+// at the end of the schedule, where the last partitions of split sequences
+// sit, so splits of more partitions are left to the merge kernel.  Reads through L2
 // only: other CTAs wrote the partials.
-template <int G> constexpr int fused_parts() { return G <= 4 ? 16 : 4; }
+template <int G> constexpr int fused_parts() { return 4; }
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_column(const DecodeParams& p, int s, int j, int dd, int n_p) {
     constexpr int NI = fused_parts<G>();
@@ -703,12 +706,16 @@ __device__ __forceinline__ void merge_store(const DecodeParams& p, int s, int h,
 }
 
 // One CTA of G * D / 4 <= MERGE_THREADS threads per (sequence, KV head):
-// thread = (head g, 4 columns); every thread walks the few partitions itself
-// (independent loads).  Small CTAs keep the whole grid resident at once.
+// thread = (head g, 4 columns); every thread walks the few partitions itself.
+// The loads of each pass are issued in batches before any is used (16 maxima,
+// then 8 (m, l) pairs with their output columns), so a split of n_p partitions
+// costs about n_p / 16 + n_p / 8 round trips to L2.  Small CTAs keep the whole
+// grid resident at once.
 template <typename T, int D>
 __global__ void __launch_bounds__(MERGE_THREADS)
 merge_group_kernel(DecodeParams p) {
     constexpr int NV = D / 4;
+    constexpr int B1 = 16, B2 = 8;
     grid_dependency_wait();                          // the decode grid's partials are complete
     const int s = blockIdx.x / p.Hkv, j = blockIdx.x - s * p.Hkv;
     const int L = clamp_len(__ldg(p.lens + s), p);
@@ -719,17 +726,34 @@ merge_group_kernel(DecodeParams p) {
     for (int c = threadIdx.x; c < G * NV; c += blockDim.x) {
         const int g = c / NV, col = c - g * NV;
         float M = -INFINITY;
-        for (int i = 0; i < n_p; ++i) M = fmaxf(M, __ldcg(p.part_ml + ((base + i) * G + g) * 2));
+        for (int i0 = 0; i0 < n_p; i0 += B1) {
+            float m[B1];
+#pragma unroll
+            for (int k = 0; k < B1; ++k)
+                m[k] = i0 + k < n_p ? __ldcg(p.part_ml + ((base + i0 + k) * G + g) * 2) : -INFINITY;
+#pragma unroll
+            for (int k = 0; k < B1; ++k) M = fmaxf(M, m[k]);
+        }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float Lsum = 0.f;
         if (M != -INFINITY) {
-#pragma unroll 4
-            for (int i = 0; i < n_p; ++i) {
-                const size_t pi = (base + i) * G + g;
-                const float w = exp2f(__ldcg(p.part_ml + pi * 2) - M);
-                Lsum += w * __ldcg(p.part_ml + pi * 2 + 1);
-                const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + pi * D) + col);
-                acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
+            for (int i0 = 0; i0 < n_p; i0 += B2) {
+                float2 ml[B2];
+                float4 o[B2];
+#pragma unroll
+                for (int k = 0; k < B2; ++k) {
+                    const size_t pi = (base + i0 + k) * G + g;
+                    ml[k] = i0 + k < n_p ? __ldcg(reinterpret_cast<const float2*>(p.part_ml) + pi)
+                                         : make_float2(-INFINITY, 0.f);
+                    o[k] = i0 + k < n_p ? __ldcg(reinterpret_cast<const float4*>(p.part_o + pi * D) + col)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int k = 0; k < B2; ++k) {          // partition order
+                    const float w = exp2f(ml[k].x - M);
+                    Lsum += w * ml[k].y;
+                    acc.x += w * o[k].x; acc.y += w * o[k].y; acc.z += w * o[k].z; acc.w += w * o[k].w;
+                }
             }
         }
         merge_store<T, D>(p, s, j * G + g, col, acc, Lsum > 0.f ? 1.f / Lsum : 0.f);

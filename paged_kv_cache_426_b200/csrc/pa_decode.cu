@@ -651,7 +651,9 @@ template <int G> constexpr int fused_parts() { return 4; }
 template <typename T, int D, int G>
 __device__ __forceinline__ void merge_column(const DecodeParams& p, int s, int j, int dd, int n_p) {
     constexpr int NI = fused_parts<G>();
-    constexpr int HB = 16 / NI;                   // heads per batch: 16 (m, l, o) loads in flight
+    // heads per batch: up to 16 (m, l, o) loads in flight, never past the group
+    constexpr int HB = G < 16 / NI ? G : 16 / NI;
+    static_assert(HB >= 1 && G % HB == 0, "batches cover the group's heads exactly");
     const size_t base = ((size_t)s * p.Hkv + j) * p.n_pmax;
 #pragma unroll
     for (int h0 = 0; h0 < G; h0 += HB) {

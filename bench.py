@@ -727,6 +727,10 @@ def run_ours(args, rank, world, local):
             mw = measure(name, args, dev, args.extra_steps, world, args.engine, flush_buf=flush,
                          warm_too=True)
             per[name] = summarize(mw, peak, rpeak)
+            if args.e2e and name != "tiny_f32":
+                e = run_e2e(mw["sess"], mw["w"], args, world)
+                e["frac_of_step"] = round(e["value"] / per[name]["step_gbs"], 4)
+                per[name]["e2e"] = e
             del mw
             torch.cuda.empty_cache()
         del flush
@@ -761,6 +765,7 @@ def run_ours(args, rank, world, local):
     if per and len(per) > 1:
         result["per_workload"] = per
     if e2e:
+        e2e["frac_of_step"] = round(e2e["value"] / value, 4)
         result["e2e"] = e2e
     if rank == 0 and world == 1 and args.cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)

@@ -147,47 +147,6 @@ __device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
-// The same load without the wait: several can be in flight; tm_wait32 waits
-// for all of them and ties the registers of one load to the wait, so that no
-// use of them is scheduled before it.
-__device__ __forceinline__ void tm_ld32_async(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr)
-        : "memory");
-}
-__device__ __forceinline__ void tm_wait_pin(uint32_t (&r)[32], bool wait) {
-    if (wait) {
-        asm volatile(
-            "tcgen05.wait::ld.sync.aligned;"
-            : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-              "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
-              "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
-              "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
-              "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
-              "+r"(r[31])
-            :
-            : "memory");
-    } else {
-        asm volatile(
-            ""
-            : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-              "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
-              "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
-              "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
-              "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
-              "+r"(r[31])
-            :
-            : "memory");
-    }
-}
-
 // 2^x by the PTX ex2.approx instruction with subnormal results flushed to
 // zero: softmax weights below 2^-126 are zero after rounding to 16 bits
 // anyway (the sum they would add is far below the output's precision).
@@ -329,89 +288,54 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         __syncwarp();
     } else if (warp == 9) {
         // ================================================= MMA issuer (one thread)
-        // Event driven: every poll issues whatever is ready, so one tile's
-        // MMAs never wait behind the other tile's softmax or a late copy:
-        //   PV_t(m)  once tile t's softmax has written P(m)   (in order of m)
-        //   S_t(c)   once stage c has landed and tile t's softmax has read
-        //            its S buffer from stage c - 2           (in order of c)
-        // A ring slot is released once every PV that reads its stage is issued.
+        // Per stage c: S of both tiles, then PV of both tiles for stage c - 1,
+        // so the tensor core computes while the softmax groups work.
         if (lane == 0) {
             constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, PF_M, PF_KT);
             constexpr uint32_t ID_O = tc::idesc_f16<T>(false, true, PF_M, D);
             bool ok = pf_wait(q_full, 0, abort_flag, p.err);
-            int cs[PF_TILES], cp[PF_TILES], nk[PF_TILES];
+            for (int c = 0; ok && c <= nkt_all; ++c) {
+                if (c < nkt_all) {
+                    const int st = c % nst, b = c & 1;
+                    ok = pf_wait(full + st, (c / nst) & 1, abort_flag, p.err);
+                    const uint64_t kd = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
 #pragma unroll
-            for (int t = 0; t < PF_TILES; ++t) {
-                cs[t] = 0;
-                cp[t] = 0;
-                nk[t] = t < ntile ? nkt[t] : 0;
-            }
-            int rel = 0;                               // next stage whose slot is released
-            uint32_t idle = 0;
-            uint64_t t_idle = 0;
-            while (ok) {
-                bool prog = false, left = false;
-#pragma unroll
-                for (int t = 0; t < PF_TILES; ++t) {
-                    // ---- O += P V for tile t's oldest stage with P written
-                    const int m = cp[t];
-                    if (m < nk[t] && m < cs[t] && mbar_test(tbar(t, 2, m & 1), (m >> 1) & 1)) {
+                    for (int t = 0; t < PF_TILES; ++t) {
+                        if (!ok || t >= ntile || c >= nkt[t]) continue;
+                        if (c >= 2) ok = pf_wait(tbar(t, 1, b), ((c - 2) >> 1) & 1, abort_flag, p.err);
+                        if (!ok) break;
                         tc::fence_after();
-                        const uint64_t vd = tc::sdesc_sw128(
-                            smem_u32(smem + ly.ring(m % nst) + LY::KV_BYTES), LY::KBOX, 1024);
-                        const uint64_t pd = tc::sdesc_sw128(smem_u32(smem + ly.p(t, m & 1)), 16, 1024);
-                        const uint32_t od = tmem + (uint32_t)(t * LY::TM_TILE + 2 * PF_KT);
-#pragma unroll
-                        for (int kk = 0; kk < PF_KT / 16; ++kk)
-                            tc::mma_ss(od, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), ID_O,
-                                       (m > 0 || kk > 0) ? 1u : 0u);
-                        tc::commit(tbar(t, 3, m & 1));
-                        cp[t] = m + 1;
-                        prog = true;
-                    }
-                    // ---- S = Q K^T for tile t's next stage
-                    const int c = cs[t];
-                    if (c < nk[t] && mbar_test(full + c % nst, (c / nst) & 1) &&
-                        (c < 2 || mbar_test(tbar(t, 1, c & 1), ((c - 2) >> 1) & 1))) {
-                        tc::fence_after();
-                        const uint64_t kd = tc::sdesc_sw128(smem_u32(smem + ly.ring(c % nst)), 16, 1024);
                         const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
-                        const uint32_t sd = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * (c & 1));
+                        const uint32_t sd = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * b);
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
                             tc::mma_ss(sd, qd + (uint64_t)((k >> 2) * (LY::QBOX >> 4) + (k & 3) * 2),
                                        kd + (uint64_t)((k >> 2) * (LY::KBOX >> 4) + (k & 3) * 2), ID_S,
                                        k > 0 ? 1u : 0u);
-                        tc::commit(tbar(t, 0, c & 1));
-                        cs[t] = c + 1;
-                        prog = true;
+                        tc::commit(tbar(t, 0, b));
                     }
-                    left |= cp[t] < nk[t];
+                    if (!ok) break;
                 }
-                // release every stage whose PVs are all issued
-                while (rel < nkt_all) {
-                    bool done = true;
+                if (c >= 1) {
+                    const int m = c - 1, bm = m & 1, stm = m % nst;
+                    const uint64_t vd =
+                        tc::sdesc_sw128(smem_u32(smem + ly.ring(stm) + LY::KV_BYTES), LY::KBOX, 1024);
 #pragma unroll
-                    for (int t = 0; t < PF_TILES; ++t) done &= (cp[t] > rel || rel >= nk[t]);
-                    if (!done) break;
-                    tc::commit(empty + rel % nst);
-                    ++rel;
-                }
-                if (!left) break;
-                if (prog) {
-                    idle = 0;
-                } else if ((++idle & 255) == 0) {
-                    // bounded: give up after kWaitLimitNs without progress, or
-                    // when another warp has given up
-                    if (*abort_flag) break;
-                    const uint64_t now = global_ns();
-                    if (idle == 256) {
-                        t_idle = now;
-                    } else if (now - t_idle > kWaitLimitNs) {
-                        set_err(p.err, PA_DEV_TIMEOUT);
-                        *abort_flag = 1;
-                        break;
+                    for (int t = 0; t < PF_TILES; ++t) {
+                        if (!ok || t >= ntile || m >= nkt[t]) continue;
+                        ok = pf_wait(tbar(t, 2, bm), (m >> 1) & 1, abort_flag, p.err);
+                        if (!ok) break;
+                        tc::fence_after();
+                        const uint64_t pd = tc::sdesc_sw128(smem_u32(smem + ly.p(t, bm)), 16, 1024);
+                        const uint32_t od = tmem + (uint32_t)(t * LY::TM_TILE + 2 * PF_KT);
+#pragma unroll
+                        for (int kk = 0; kk < PF_KT / 16; ++kk)
+                            tc::mma_ss(od, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), ID_O,
+                                       (m > 0 || kk > 0) ? 1u : 0u);
+                        tc::commit(tbar(t, 3, bm));
                     }
+                    if (!ok) break;
+                    tc::commit(empty + stm);           // the stage slot may be refilled
                 }
             }
             // every MMA of this CTA completes before tensor memory is freed
@@ -446,12 +370,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             const int lim = pos - c * PF_KT + 1;
             const bool whole = __all_sync(PF_FULL, lim >= PF_KT && vmask == (1u << (PF_KT / PR)) - 1u);
             const uint32_t tSb = tS + (uint32_t)(PF_KT * b) + lq;
+            // pass 1: the row maximum of the raw scores (the scale is positive)
             float mraw = -INFINITY;
 #pragma unroll
             for (int h = 0; h < PF_KT / 32; ++h) {
                 uint32_t v[32];
                 tm_ld32(tSb + (uint32_t)(32 * h), v);
-                if (whole) {
+                if (whole) {                           // warp-uniform: no key is hidden
 #pragma unroll
                     for (int i = 0; i < 32; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
                 } else {

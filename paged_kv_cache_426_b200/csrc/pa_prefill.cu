@@ -12,13 +12,17 @@
 // takes two adjacent query tiles of one (sequence, KV head) and streams the
 // K/V stages once for both.  Per 64-key stage and tile:
 //   S  = Q K^T      M = 128, N = 64, K = head_dim        (tcgen05, fp32 in TMEM)
-//   P  = exp2(S * scale * log2 e - m), rounded to the input type, in smem
-//   O += P V        M = 128, N = head_dim, K = 64 keys    (tcgen05, fp32 in TMEM)
+//   P  = exp2(S * scale * log2 e - m), rounded to the input type, written
+//        back into tensor memory over the S columns it came from
+//   O += P V        M = 128, N = head_dim, K = 64 keys    (tcgen05, A = P from
+//                   TMEM, B = V from smem, fp32 in TMEM)
 // Warps: 0-3 softmax + epilogue of tile 0, 4-7 of tile 1 (thread = one row =
 // one tensor-memory lane), 8 TMA producer, 9 MMA issuer (one thread).  The
 // two softmax groups run side by side (two warps per SM sub-partition) while
-// the tensor core works on the other tile; S is double-buffered in tensor
-// memory and P in shared memory per tile.  The row maximum m is moved lazily:
+// the tensor core works on the other tile; S (and the P written over it) is
+// double-buffered in tensor memory per tile.  With no P in shared memory the
+// K/V ring holds five 64-key stages: a stage stays in its slot for the copy's
+// latency plus the S -> softmax -> PV chain, so the ring depth sets the pace.  The row maximum m is moved lazily:
 // only when a stage exceeds it by 2^8 is O rescaled in tensor memory.  Keys
 // past the row's position get weight 0; keys past the CTA's key range or in a
 // block whose table entry is bad also get their V rows zeroed in shared
@@ -42,7 +46,7 @@ constexpr int PF_KT = 64;          // keys per stage (N of S, K of PV)
 constexpr int PF_M = 128;          // query rows per tile
 constexpr int PF_TILES = 2;        // query tiles per CTA
 constexpr int PF_THREADS = 320;    // 8 softmax warps, producer, MMA issuer
-constexpr int PF_MAX_STAGES = 4;
+constexpr int PF_MAX_STAGES = 6;
 constexpr float kPfRescaleLog2 = 8.f;
 constexpr uint32_t PF_FULL = 0xffffffffu;
 
@@ -60,9 +64,10 @@ struct PrefillParams {
 // Shared memory (1024-byte aligned; every operand tile starts on a 1024-byte
 // boundary, as the 128-byte swizzle wants):
 //   Q        per tile NBOX boxes of [128 rows][128 B]
-//   P        per tile two buffers of [128 rows][128 B] (64 keys of a row per line)
 //   ring     nst stages of K then V, each NBOX boxes of [64 keys][128 B]
 //   barriers, per-stage valid-piece masks, misc
+// P never goes to shared memory: the softmax writes it into tensor memory
+// over the S columns it came from, and the PV MMA reads it from there.
 template <int D>
 struct PfLayout {
     static constexpr int NBOX = D * 2 / 128;           // 128-byte column boxes of a row
@@ -71,20 +76,17 @@ struct PfLayout {
     static constexpr int KBOX = PF_KT * 128;
     static constexpr int KV_BYTES = NBOX * KBOX;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int P_BYTES = PF_M * 128;
-    // per tile: S x2 (64 columns each) then O (head_dim columns), 256 columns
+    // per tile: S x2 (64 columns each; P, 16-bit pairs, overwrites the first 32
+    // columns of its S buffer) then O (head_dim columns), 256 columns
     static constexpr uint32_t TM_TILE = 256;
     static constexpr uint32_t TM_COLS = PF_TILES * TM_TILE;
-    // q_full, fin, then per tile s_full x2, s_free x2, p_full x2, pv_done x2
+    // q_full, fin, then per tile s_full x2, (spare) x2, p_full x2, pv_done x2
     static constexpr int NBAR_FIXED = 2 + 8 * PF_TILES;
     int nst;
     __host__ __device__ explicit PfLayout(int n) : nst(n) {}
     __host__ __device__ size_t q(int t) const { return (size_t)t * Q_BYTES; }
-    __host__ __device__ size_t p(int t, int b) const {
-        return (size_t)PF_TILES * Q_BYTES + (size_t)(2 * t + b) * P_BYTES;
-    }
     __host__ __device__ size_t ring(int st) const {
-        return (size_t)PF_TILES * (Q_BYTES + 2 * P_BYTES) + (size_t)st * STAGE_BYTES;
+        return (size_t)PF_TILES * Q_BYTES + (size_t)st * STAGE_BYTES;
     }
     __host__ __device__ size_t bars() const { return ring(nst); }
     __host__ __device__ size_t masks() const { return bars() + (size_t)(2 * nst + NBAR_FIXED) * 8; }
@@ -156,6 +158,46 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     return y;
 }
 
+// Packed fp32x2 add / subtract (one instruction for two lanes).
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^z for two lanes on the FMA pipe, to share the softmax's exponentials
+// between this path and the MUFU's ex2.approx (whose throughput bounds the
+// softmax).  Range reduction by rounding: adding 1.5 * 2^23 rounds z to the
+// nearest integer j (exactly, for |z| < 2^22), f = z - j lies in [-1/2, 1/2],
+// 2^f is a cubic fitted to it by reweighted least squares in relative error
+// (coefficients below; max relative error 7.5e-5, far below the 2^-9 / 2^-11
+// rounding of P to bf16 / fp16), and 2^j is added into the exponent field
+// (the low bits of z + 1.5 * 2^23 hold j).  z is clamped at -126 so the
+// exponent never wraps: results below 2^-126 come out as tiny non-negative
+// numbers, which is all a softmax weight of that size can be after rounding.
+// Valid for z <= 127 (here z <= 8: the reference max lags by at most 2^8).
+constexpr float kExpC0 = 0.9999280571937561f, kExpC1 = 0.6932601928710938f,
+                kExpC2 = 0.24261149764060974f, kExpC3 = 0.05517605319619179f;
+__device__ __forceinline__ void exp2_fma2(float z0, float z1, float& e0, float& e1) {
+    const uint64_t SH2 = f2_pack(12582912.f, 12582912.f);          // 1.5 * 2^23
+    const uint64_t z2 = f2_pack(fmaxf(z0, -126.f), fmaxf(z1, -126.f));
+    const uint64_t t2 = f2_add(z2, SH2);
+    const uint64_t f2 = f2_sub(z2, f2_sub(t2, SH2));
+    uint64_t p2 = f2_fma(f2_pack(kExpC3, kExpC3), f2, f2_pack(kExpC2, kExpC2));
+    p2 = f2_fma(p2, f2, f2_pack(kExpC1, kExpC1));
+    p2 = f2_fma(p2, f2, f2_pack(kExpC0, kExpC0));
+    float p0, p1, t0, t1;
+    f2_unpack(p2, p0, p1);
+    f2_unpack(t2, t0, t1);
+    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(PF_THREADS, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -203,8 +245,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     uint64_t* empty = full + nst;
     uint64_t* q_full = empty + nst;
     uint64_t* fin = q_full + 1;                    // issuer's final drain
-    // per tile t: s_full[2] (S in tensor memory), s_free[2] (S read by the 4
-    // softmax warps), p_full[2] (P written by them), pv_done[2] (PV complete)
+    // per tile t: s_full[2] (S in tensor memory), kind 1 unused, p_full[2] (P
+    // written by the 4 softmax warps), pv_done[2] (PV complete)
     auto tbar = [&](int t, int kind, int b) { return fin + 1 + t * 8 + kind * 2 + b; };
     int* masks = reinterpret_cast<int*>(smem + ly.masks());
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
@@ -214,10 +256,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (tid == 0) {
         for (int k = 0; k < 2 * nst + LY::NBAR_FIXED; ++k) mbar_init(full + k, 1);
         for (int t = 0; t < PF_TILES; ++t)
-            for (int b = 0; b < 2; ++b) {
-                mbar_init(tbar(t, 1, b), 4);       // s_free
-                mbar_init(tbar(t, 2, b), 4);       // p_full
-            }
+            for (int b = 0; b < 2; ++b) mbar_init(tbar(t, 2, b), 4);   // p_full
         misc[0] = 0;
         fence_barrier_init();
     }
@@ -302,8 +341,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 #pragma unroll
                     for (int t = 0; t < PF_TILES; ++t) {
                         if (!ok || t >= ntile || c >= nkt[t]) continue;
-                        if (c >= 2) ok = pf_wait(tbar(t, 1, b), ((c - 2) >> 1) & 1, abort_flag, p.err);
-                        if (!ok) break;
+                        // S buffer b last held S(c - 2), whose P the PV of
+                        // stage c - 2 reads from it: that PV was issued in
+                        // the previous round, and this thread's MMAs run in
+                        // the order issued
                         tc::fence_after();
                         const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
                         const uint32_t sd = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * b);
@@ -326,11 +367,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         ok = pf_wait(tbar(t, 2, bm), (m >> 1) & 1, abort_flag, p.err);
                         if (!ok) break;
                         tc::fence_after();
-                        const uint64_t pd = tc::sdesc_sw128(smem_u32(smem + ly.p(t, bm)), 16, 1024);
+                        // A = P in tensor memory (lane = row, column = two keys),
+                        // B = the V stage (MN-major)
+                        const uint32_t pt = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * bm);
                         const uint32_t od = tmem + (uint32_t)(t * LY::TM_TILE + 2 * PF_KT);
 #pragma unroll
                         for (int kk = 0; kk < PF_KT / 16; ++kk)
-                            tc::mma_ss(od, pd + (uint64_t)(kk * 2), vd + (uint64_t)(kk * 128), ID_O,
+                            tc::mma_ts(od, pt + (uint32_t)(kk * 8), vd + (uint64_t)(kk * 128), ID_O,
                                        (m > 0 || kk > 0) ? 1u : 0u);
                         tc::commit(tbar(t, 3, bm));
                     }
@@ -409,14 +452,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
                 if (need) m_ref = mt;
             }
-            if (c >= 2) {
-                // P buffer b was read by the PV two stages back
-                ok = __all_sync(PF_FULL, pf_wait(tbar(t, 3, b), ((c - 2) >> 1) & 1, abort_flag, p.err));
-                if (!ok) break;
-            }
-            // pass 2: P = exp2(s * scale * log2 e - m), rounded, into the swizzled P rows
+            // pass 2: P = exp2(s * scale * log2 e - m), rounded, written as
+            // 16-bit pairs over columns [0, 32) of S buffer b (each pass reads
+            // 32 score columns before it overwrites 16 already-read ones)
             const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
-            uint8_t* prow = smem + ly.p(t, b) + r * 128;
             float lsum = 0.f;
             // packed fp32x2: z = s * scale * log2 e - m for two keys at once; the
             // row sum adds the weights as rounded to T (what the PV MMA multiplies)
@@ -436,28 +475,28 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
                         if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                     }
-                    w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
+                    if (whole && (i & 1)) {
+                        // every other pair of an unmasked stage on the FMA pipe
+                        float e0, e1;
+                        exp2_fma2(z0, z1, e0, e1);
+                        w[i] = pack2<T>(e0, e1);
+                    } else {
+                        w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
+                    }
                     acc2 = f2_fma(Pairs<T>::from_word(w[i]), ONE2, acc2);
                 }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int q8 = 4 * h + qq;
-                    *reinterpret_cast<uint4*>(prow + ((q8 ^ (r & 7)) << 4)) =
-                        make_uint4(w[4 * qq], w[4 * qq + 1], w[4 * qq + 2], w[4 * qq + 3]);
-                }
+                tc::st16(tSb + (uint32_t)(16 * h), w);
             }
             {
                 float a0, a1;
                 f2_unpack(acc2, a0, a1);
                 lsum = a0 + a1;
             }
-            tc::fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(tbar(t, 1, b));    // S buffer b may be rewritten
             l += lsum;
             if (r < PF_KT) {
                 // rows past the CTA's key range or of a skipped block: zero V
-                // (both groups write the same zeros)
+                // (both groups write the same zeros), visible to the MMA's
+                // async-proxy reads
                 const int key = c * PF_KT + r;
                 if (key >= kend || !((vmask >> (r >> prl)) & 1u)) {
                     uint8_t* vrow = smem + ly.ring(st) + LY::KV_BYTES + r * 128;
@@ -466,9 +505,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 #pragma unroll
                         for (int q8 = 0; q8 < 8; ++q8)
                             *reinterpret_cast<uint4*>(vrow + bx * LY::KBOX + q8 * 16) = make_uint4(0, 0, 0, 0);
+                    fence_proxy_async_smem();
                 }
             }
-            fence_proxy_async_smem();
             tc::fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(tbar(t, 2, b));

@@ -149,6 +149,18 @@ __device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
+// 16 columns to tensor memory without waiting (tm_wait_st before the result
+// is handed to another thread).
+__device__ __forceinline__ void tm_st16_nowait(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+          "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tm_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // 2^x by the PTX ex2.approx instruction with subnormal results flushed to
 // zero: softmax weights below 2^-126 are zero after rounding to 16 bits
 // anyway (the sum they would add is far below the output's precision).
@@ -156,46 +168,6 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// Packed fp32x2 add / subtract (one instruction for two lanes).
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// 2^z for two lanes on the FMA pipe, to share the softmax's exponentials
-// between this path and the MUFU's ex2.approx (whose throughput bounds the
-// softmax).  Range reduction by rounding: adding 1.5 * 2^23 rounds z to the
-// nearest integer j (exactly, for |z| < 2^22), f = z - j lies in [-1/2, 1/2],
-// 2^f is a cubic fitted to it by reweighted least squares in relative error
-// (coefficients below; max relative error 7.5e-5, far below the 2^-9 / 2^-11
-// rounding of P to bf16 / fp16), and 2^j is added into the exponent field
-// (the low bits of z + 1.5 * 2^23 hold j).  z is clamped at -126 so the
-// exponent never wraps: results below 2^-126 come out as tiny non-negative
-// numbers, which is all a softmax weight of that size can be after rounding.
-// Valid for z <= 127 (here z <= 8: the reference max lags by at most 2^8).
-constexpr float kExpC0 = 0.9999280571937561f, kExpC1 = 0.6932601928710938f,
-                kExpC2 = 0.24261149764060974f, kExpC3 = 0.05517605319619179f;
-__device__ __forceinline__ void exp2_fma2(float z0, float z1, float& e0, float& e1) {
-    const uint64_t SH2 = f2_pack(12582912.f, 12582912.f);          // 1.5 * 2^23
-    const uint64_t z2 = f2_pack(fmaxf(z0, -126.f), fmaxf(z1, -126.f));
-    const uint64_t t2 = f2_add(z2, SH2);
-    const uint64_t f2 = f2_sub(z2, f2_sub(t2, SH2));
-    uint64_t p2 = f2_fma(f2_pack(kExpC3, kExpC3), f2, f2_pack(kExpC2, kExpC2));
-    p2 = f2_fma(p2, f2, f2_pack(kExpC1, kExpC1));
-    p2 = f2_fma(p2, f2, f2_pack(kExpC0, kExpC0));
-    float p0, p1, t0, t1;
-    f2_unpack(p2, p0, p1);
-    f2_unpack(t2, t0, t1);
-    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
 }
 
 template <typename T, int D, int G>
@@ -453,8 +425,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 if (need) m_ref = mt;
             }
             // pass 2: P = exp2(s * scale * log2 e - m), rounded, written as
-            // 16-bit pairs over columns [0, 32) of S buffer b (each pass reads
-            // 32 score columns before it overwrites 16 already-read ones)
+            // 16-bit pairs over columns [0, 32) of S buffer b (each half reads
+            // 32 score columns before it overwrites 16 already-read ones); the
+            // two stores complete before P is handed to the MMA issuer
             const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
             float lsum = 0.f;
             // packed fp32x2: z = s * scale * log2 e - m for two keys at once; the
@@ -463,7 +436,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < PF_KT / 32; ++h) {
-                uint32_t v[32], w[16];
+                uint32_t w[16], v[32];
                 tm_ld32(tSb + (uint32_t)(32 * h), v);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -475,18 +448,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
                         if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                     }
-                    if (whole && (i & 1)) {
-                        // every other pair of an unmasked stage on the FMA pipe
-                        float e0, e1;
-                        exp2_fma2(z0, z1, e0, e1);
-                        w[i] = pack2<T>(e0, e1);
-                    } else {
-                        w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
-                    }
+                    w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
                     acc2 = f2_fma(Pairs<T>::from_word(w[i]), ONE2, acc2);
                 }
-                tc::st16(tSb + (uint32_t)(16 * h), w);
+                tm_st16_nowait(tSb + (uint32_t)(16 * h), w);
             }
+            tm_wait_st();
             {
                 float a0, a1;
                 f2_unpack(acc2, a0, a1);

@@ -40,6 +40,7 @@ struct pa_manager {
     struct Seq {
         std::vector<int32_t> table;    // logical block -> physical block
         int32_t len = 0;               // tokens held
+        uint64_t stamp = 0;            // last append_step call that named it
     };
     // One cached block: the key of its whole prefix, the key of the prefix
     // before it (0 for a first block) and its own tokens (checked on a hit).
@@ -56,6 +57,7 @@ struct pa_manager {
     std::unordered_map<int32_t, Cached> cached;          // block -> entry
     std::list<int32_t> lru;                              // least recently used first
     int64_t hits = 0, misses = 0, evictions = 0;
+    uint64_t step_calls = 0;                             // append_step calls so far
 };
 
 namespace {
@@ -341,14 +343,14 @@ int pa_manager_append_step(pa_manager* m, const int64_t* seq_ids, int num_seqs,
     if (!m || num_seqs < 0 || !num_cow || (num_seqs > 0 && (!seq_ids || !slots || !cow_pairs)))
         return PA_ERR_INVALID;
     std::vector<pa_manager::Seq*> ss(num_seqs);
+    const uint64_t stamp = ++m->step_calls;   // a sequence may append once per step
     for (int i = 0; i < num_seqs; ++i) {
         auto it = m->seqs.find(seq_ids[i]);
         if (it == m->seqs.end()) return PA_ERR_STATE;
+        if (it->second.stamp == stamp) return PA_ERR_INVALID;
+        it->second.stamp = stamp;
         ss[i] = &it->second;
     }
-    for (int i = 0; i < num_seqs; ++i)        // a sequence may append once per step
-        for (int k = 0; k < i; ++k)
-            if (ss[k] == ss[i]) return PA_ERR_INVALID;
     std::vector<Undo> log(num_seqs);
     int n = 0;
     for (int i = 0; i < num_seqs; ++i) {
@@ -388,9 +390,8 @@ int pa_manager_block_tables(const pa_manager* m, const int64_t* seq_ids, int num
         const auto& t = it->second.table;
         if (static_cast<int>(t.size()) > max_blocks) return PA_ERR_INVALID;
         int32_t* row = block_tables + static_cast<int64_t>(i) * max_blocks;
-        int k = 0;
-        for (; k < static_cast<int>(t.size()); ++k) row[k] = t[k];
-        for (; k < max_blocks; ++k) row[k] = -1;
+        std::copy(t.begin(), t.end(), row);
+        std::fill(row + t.size(), row + max_blocks, int32_t(-1));
         context_lens[i] = it->second.len;
     }
     return PA_OK;

@@ -191,6 +191,23 @@ def test_append_is_all_or_nothing():
     assert [a.refcount(b) for b in range(3)] == [2, 2, 2]
 
 
+def test_append_step_rejects_a_sequence_named_twice():
+    """One token per sequence per step: a batch naming a sequence twice is
+    rejected before anything is appended, and the next step still works."""
+    a = pa.BlockAllocator(16)
+    m = pa.BlockManager(a, 4)
+    for s in range(3):
+        m.add_seq(s)
+    m.append_step([0, 1, 2])
+    with pytest.raises(pa.PAError) as e:
+        m.append_step([2, 0, 1, 0])
+    assert e.value.status == pa.PA_ERR_INVALID
+    assert [m.seq_len(s) for s in range(3)] == [1, 1, 1] and a.num_free() == 13
+    slots, cow = m.append_step([1, 0, 2])
+    assert [m.seq_len(s) for s in range(3)] == [2, 2, 2] and cow.shape[0] == 0
+    assert slots.tolist() == [5, 1, 9]
+
+
 def test_beam_sharing_example_matches_page():
     """velog 메모리 공유 example, through the C++ manager."""
     from tests.conftest import golden

@@ -9,9 +9,11 @@
   / 1e-2 (bf16).
 
 Small variants of the five workloads are compared element by element (they
-span several stages, partitions and a ragged tail); the full-size workloads,
-in the launch configuration the benchmark times, are compared on sampled
-(sequence, head) outputs that the oracle computes one by one.
+span several stages, partitions and a ragged tail; one set has more work units
+than three per resident CTA).  The full-size workloads, in the launch
+configuration the benchmark times, are compared element by element at step 0,
+every 8th step and the last step, and on sampled (sequence, head) outputs
+that the oracle computes one by one at the steps between.
 """
 import numpy as np
 import pytest
@@ -484,17 +486,19 @@ def test_prefix_cache_decode_bit_identical():
 
 # ---------------------------------------------------------------- failure detection
 
-@pytest.mark.parametrize("engine_id", [1, 2])
-def test_bounded_wait_reports_timeout(engine_id):
+@pytest.mark.parametrize("engine_id,P", [(1, 512), (2, 512), (2, 2048)])
+def test_bounded_wait_reports_timeout(engine_id, P):
     """Failure detection without a fault: a stage whose barrier nothing will
     arrive on (per-call option test_withhold_stage of pa_decode_ex) makes the
     waiting warps give up after the 2 s limit; the call returns, err_flag says
     PA_DEV_TIMEOUT, and the next call on the same workspace and context is
-    correct."""
+    correct.  With P = 2048 the tensor-core engine merges the sequences' 3
+    partitions itself: the timed-out call leaves split counters partly
+    counted, and the kernel's last CTA must zero them again."""
     import time
     w = workloads.gqa8b_bf16(num_seqs=6)
     rec = oracle.run(w, keep_prefill_cache=True)
-    g = CudaPathRun(w, rec, partition_size=512)
+    g = CudaPathRun(w, rec, partition_size=P)
     g.replay_prefill()
     st = rec.steps[0]
     slots, _ = g.mgr.append_step(st.seqs)
@@ -504,18 +508,30 @@ def test_bounded_wait_reports_timeout(engine_id):
     q = w.step_q[0].cuda()
     out = torch.empty_like(q)
     tab_d, lens_d = tab.cuda(), lens.cuda()
+    S = q.shape[0]
 
     def decode(hold):
-        pa.pa_decode(out, q, g.kc, g.vc, tab_d, lens_d, g.max_len, w.scale, partition_size=512,
+        pa.pa_decode(out, q, g.kc, g.vc, tab_d, lens_d, g.max_len, w.scale, partition_size=P,
                      workspace=g.ws, err_flag=g.err, engine=engine_id, test_withhold_stage=hold)
         torch.cuda.synchronize()
+
+    def scheduler_words_clear():
+        # header (ticket, CTA count, dirty flag), then one split counter per
+        # (sequence, KV head)
+        hdr = g.ws[:256].view(torch.int32)
+        cnt = g.ws[256:256 + 4 * S * w.num_kv_heads].view(torch.int32)
+        return int(hdr[:3].abs().sum()) == 0 and int(cnt.abs().sum()) == 0
 
     t0 = time.time()
     decode(0)
     dt = time.time() - t0
     assert int(g.err.item()) == pa.PA_DEV_TIMEOUT
     assert 1.0 < dt < 30.0
-    g.err.zero_()
-    decode(-1)
-    assert int(g.err.item()) == 0
-    check_close(out_f64(out, w.dtype), st.out, w.dtype, "the call after a timed-out one")
+    assert scheduler_words_clear()
+    for _ in range(2):
+        g.err.zero_()
+        out.fill_(float("nan"))
+        decode(-1)
+        assert int(g.err.item()) == 0
+        check_close(out_f64(out, w.dtype), st.out, w.dtype, "the call after a timed-out one")
+        assert scheduler_words_clear()

@@ -1772,8 +1772,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         __threadfence();
         const int done = atomicAdd(&p.hdr->done_ctas, 1);
         if (done == (int)gridDim.x - 1) {
-            if (atomicAdd(&p.hdr->dirty, 0) && p.fused_merge) {
-                for (int k = 0; k < p.S * p.Hkv; ++k) p.split_cnt[k] = 0;
+            if (atomicAdd(&p.hdr->dirty, 0)) {
+                // only the in-kernel merge counts splits; either way the
+                // header goes back to zero
+                if (p.fused_merge)
+                    for (int k = 0; k < p.S * p.Hkv; ++k) p.split_cnt[k] = 0;
                 p.hdr->dirty = 0;
             }
             p.hdr->next_unit = 0;

@@ -998,13 +998,9 @@ decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ 
 // is what keeps HBM busy (a ring slot stays held for the copy's latency plus
 // the S -> softmax -> PV chain).
 // Warps: 0-3 softmax (thread = one token of the stage: with M = 64, rows
-// 16w..16w+15 sit in lanes 0-15 of warp w's lane quarter; thread 0 also
-// issues each stage's PV MMAs once P^T is written), 4-7 epilogue (thread =
-// head_dim row of O^T), 8 producer, 9 S issuer (one thread).  An MMA
-// instruction takes ~70-100 cycles to issue, and two issuing threads overlap
-// that cost, so S and PV come from different threads: a PV never waits behind
-// the next stage's S issues.  Tensor memory: two S^T buffers and two O^T
-// buffers (alternating per unit, so a unit's epilogue overlaps the next unit).  The softmax keeps a
+// 16w..16w+15 sit in lanes 0-15 of warp w's lane quarter), 4-7 epilogue
+// (thread = head_dim row of O^T), 8 producer, 9 MMA issuer (one thread).  Tensor memory: two S^T buffers and two O^T buffers (alternating
+// per unit, so a unit's epilogue overlaps the next unit).  The softmax keeps a
 // per-head reference max m that lags the true running max by at most 2^8
 // (exp2 units): only when a stage exceeds it is m moved (a barrier-OR vote
 // over the 128 threads), O^T rescaled in tensor memory and l rescaled.
@@ -1033,7 +1029,7 @@ struct TcLayout {
     static constexpr int QT = NBOX * (NQ / 8) * 1024;  // Q tile: NQ rows x head_dim, 128B swizzle
     static constexpr int PTB = TTOK * NHP * 2;         // one P^T tile (2 KB)
     static constexpr uint32_t TM_COLS = 64;            // S^T x2 then O^T x2, 16 columns each
-    static constexpr int NBAR = 2 * NU + 14;           // + 2 per stage slot
+    static constexpr int NBAR = 2 * NU + 13;           // + 2 per stage slot
     // epilogue slot: ints s, j, i, n_p, n_stages, O buffer, 2 pad; m[16]; l[4][16]
     static constexpr int ES = 32 + NHP * 4 + 4 * NHP * 4;
     static_assert(4 * kSchedScratch <= 2 * ES, "schedule scratch fits the epilogue slots");
@@ -1354,13 +1350,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
     uint64_t* ufull = empty + nst;
     uint64_t* uempty = ufull + NU;        // 5 arrivals: MMA issuer + the 4 softmax warps
     uint64_t* s_full = uempty + NU;       // [2] S^T_g complete
-    uint64_t* p_full = s_full + 2;        // [2] S^T_g read and P^T_g written (softmax thread 0)
+    uint64_t* p_full = s_full + 2;        // [2] P^T_g written (4 softmax warps)
     uint64_t* o_done = p_full + 2;        // [2] last PV of a unit complete (per O buffer)
     uint64_t* o_free = o_done + 2;        // [2] O buffer read by the epilogue (4 warps)
     uint64_t* epi_full = o_free + 2;      // [2] epilogue slot filled (4 softmax warps)
     uint64_t* epi_empty = epi_full + 2;   // [2] epilogue slot read (4 epilogue warps)
-    uint64_t* fin = epi_empty + 2;        // S issuer's final drain
-    uint64_t* fin_pv = fin + 1;           // PV issuer's (softmax thread 0) final drain
+    uint64_t* fin = epi_empty + 2;        // issuer's final drain
     int* stage_ok = reinterpret_cast<int*>(smem + ly.stage_ok());
     float* red = reinterpret_cast<float*>(smem + ly.red());      // [4][16]
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
@@ -1377,7 +1372,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         for (int k = 0; k < n; ++k) mbar_init(full + k, 1);
         for (int k = 0; k < NU; ++k) mbar_init(uempty + k, 5);
         for (int k = 0; k < 2; ++k) {
-            mbar_init(p_full + k, 1);
+            mbar_init(p_full + k, 4);
             mbar_init(o_free + k, 4);
             mbar_init(epi_full + k, 4);
             mbar_init(epi_empty + k, 4);
@@ -1416,22 +1411,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         producer_tc<T, D, G>(&kmap, &vmap, &qmap, p, smem, ly, full, empty, ufull, uempty,
                              stage_ok, preF, order, lens_s, U, abort_flag, lane);
     } else if (warp == 9) {
-        // ================================================= S issuer (one thread)
-        // Issues S^T = K Q^T for each stage once its data has landed and the
-        // softmax has finished with the S^T buffer it reuses (stage g - 2:
-        // p_full).  The PV MMAs are issued by softmax thread 0 right after the
-        // softmax writes P^T, so a PV never waits behind this thread's S
-        // issues (each MMA instruction takes ~70-100 cycles to issue).
+        // ================================================= MMA issuer (one thread)
+        // Event driven: the thread polls the next stage's data (-> S MMAs) and
+        // the oldest pending stage's P (-> PV MMAs) and issues whichever is
+        // ready, so a PV never waits for the next stage's copy.  S_g is issued
+        // only once PV_{g-2} has been (its S^T and P^T buffers are reused).
         if (lane == 0) {
             constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, SM_M, LY::NQ);
-            int ucount = 0, c = 0, slot = 0;
+            constexpr uint32_t ID_O = tc::idesc_f16<T>(true, true, D, NHP);
+            struct Pending {
+                int g, nv, oseq;
+                bool first, last;
+            };
+            Pending pend0{}, pend1{};            // S issued, PV not yet (pend0 oldest)
+            int npend = 0;
+            int ucount = 0, ocount = 0, c = 0, oseq = 0, slot = 0;
             bool have = false, s_done = false, ok = true;
             UnitDesc d{};
             uint32_t idle = 0;
             uint64_t t_idle = 0;
             while (true) {
                 bool prog = false;
-                // ---- the next unit
+                // ---- the next unit, for the S side
                 if (!have && !s_done) {
                     slot = ucount % NU;
                     if (mbar_test(ufull + slot, (ucount / NU) & 1)) {
@@ -1446,15 +1447,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                             } else {
                                 have = true;
                                 c = 0;
+                                oseq = ocount++;
                             }
                         }
                     }
                 }
+                // ---- O^T += V^T P^T of the oldest pending stage
+                if (npend > 0) {
+                    const Pending r = pend0;
+                    const int ob = r.oseq & 1;
+                    bool ready = mbar_test(p_full + (r.g & 1), (r.g >> 1) & 1);
+                    if (ready && r.first && r.oseq >= 2)   // the epilogue has read this O^T buffer
+                        ready = mbar_test(o_free + ob, ((r.oseq >> 1) - 1) & 1);
+                    if (ready) {
+                        tc::fence_after();
+                        const int st = r.g % nst;
+                        const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st) + LY::KV_BYTES), LY::BOXT, 1024);
+                        const uint64_t b0 = tc::sdesc_none(smem_u32(smem + ly.pt(r.g & 1)), 256, 128);
+                        const uint32_t od = tO + (uint32_t)(NHP * ob);
+                        const int nk = (r.nv + 15) / 16;             // 16-token slices holding tokens
+                        for (int kk = 0; kk < nk; ++kk)
+                            tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
+                                       (r.first && kk == 0) ? 0u : 1u);
+                        tc::commit(empty + st);          // the stage slot may be refilled
+                        if (r.last) tc::commit(o_done + ob);
+                        pend0 = pend1;
+                        --npend;
+                        prog = true;
+                    }
+                }
                 // ---- S^T of the unit's next stage
-                if (have) {
+                if (have && npend < 2) {
                     const int g = d.stage_base + c, st = g % nst;
-                    if (mbar_test(full + st, (g / nst) & 1) &&
-                        (g < 2 || mbar_test(p_full + (g & 1), ((g - 2) >> 1) & 1))) {
+                    if (mbar_test(full + st, (g / nst) & 1)) {
                         tc::fence_after();
                         const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
                         const uint64_t b0 = tc::sdesc_sw128(smem_u32(smem + ly.q(slot)), 16, 1024);
@@ -1466,11 +1491,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                                        k > 0 ? 1u : 0u);
                         tc::commit(s_full + (g & 1));
                         if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
+                        const Pending nw{g, min(TTOK, d.t1 - (d.t0 + c * TTOK)), oseq, c == 0,
+                                         c == d.n_stages - 1};
+                        if (npend == 0) pend0 = nw; else pend1 = nw;
+                        ++npend;
                         if (++c == d.n_stages) have = false;
                         prog = true;
                     }
                 }
-                if (s_done && !have) break;
+                if (s_done && !have && npend == 0) break;
                 if (prog) {
                     idle = 0;
                 } else if ((++idle & 255) == 0) {
@@ -1496,9 +1525,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         __syncwarp();
     } else if (warp < 4) {
         // ================================================= softmax warps (thread = token)
-        // Thread 0 also issues each stage's O^T += V^T P^T once all four warps
-        // have written P^T (the MMAs come from this thread, in stage order).
-        constexpr uint32_t ID_O = tc::idesc_f16<T>(true, true, D, NHP);
         const int t = (lane < 16 && 16 * warp + lane < TTOK) ? 16 * warp + lane : -1;   // stage token (M = 64 layout)
         const int piece = t >= 0 ? t / PR : 0;
         int ucount = 0, ocount = 0;
@@ -1596,10 +1622,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         tc::st16(tO + (uint32_t)(NHP * ob) + lq, o);
                     }
                 }
-                // P^T buffer b was last read by the PV of stage g - 2 (issued
-                // by thread 0 two stages back): it must have completed
-                bool okp = true;
-                if (g >= 2) okp = wait_or_abort(empty + (g - 2) % nst, ((g - 2) / nst) & 1, abort_flag, p.err);
                 // P^T row t (16 heads, 16-bit), l sums the rounded weights the MMA uses
                 uint32_t pk[NHP / 2];
 #pragma unroll
@@ -1630,32 +1652,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                 }
                 fence_proxy_async_smem();
                 tc::fence_before();
-                // every P^T row and zeroed V row is written (or some wait gave up)
-                if (named_bar_or(BAR_SOFTMAX, 128, !okp)) {
-                    ok = false;
-                    break;
-                }
-                if (tid == 0) {
-                    mbar_arrive(p_full + b);              // S^T buffer b is free for S_{g+2}
-                    tc::fence_after();
-                    // the first PV of a unit overwrites its O^T buffer: the
-                    // epilogue must have read what the unit two back left there
-                    const bool okf = !(c == 0 && ocount >= 2) ||
-                                     wait_or_abort(o_free + ob, ((ocount >> 1) - 1) & 1, abort_flag, p.err);
-                    if (okf) {
-                        const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st) + LY::KV_BYTES), LY::BOXT, 1024);
-                        const uint64_t b0 = tc::sdesc_none(smem_u32(smem + ly.pt(b)), 256, 128);
-                        const uint32_t od = tO + (uint32_t)(NHP * ob);
-                        const int nv = min(TTOK, d.t1 - (d.t0 + c * TTOK));
-                        const int nk = (nv + 15) / 16;             // 16-token slices holding tokens
-                        for (int kk = 0; kk < nk; ++kk)
-                            tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
-                                       (c == 0 && kk == 0) ? 0u : 1u);
-                        tc::commit(empty + st);          // the stage slot may be refilled
-                        if (c == d.n_stages - 1) tc::commit(o_done + ob);
-                    }
-                }
                 __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + b);
             }
             if (!ok) break;
             // ---- hand (m, l partial sums, unit) to the epilogue warps
@@ -1676,11 +1674,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
             if (lane == 0) mbar_arrive(epi_full + e);
             if (d.n_stages > 0) ++ocount;
             ++ucount;
-        }
-        // every PV MMA thread 0 issued has completed before tensor memory is freed
-        if (tid == 0) {
-            tc::commit(fin_pv);
-            mbar_wait(fin_pv, 0);
         }
         __syncwarp();
     } else {

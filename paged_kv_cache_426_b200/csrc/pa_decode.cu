@@ -1430,35 +1430,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
             UnitDesc d{};
             uint32_t idle = 0;
             uint64_t t_idle = 0;
-            // Issue the oldest pending stage's PV if its P is written (and, for
-            // a unit's first stage, its O^T buffer has been read out).  Also
-            // called between the K slices of an S, so that a PV whose P turns
-            // up meanwhile does not wait for the whole S to be issued: the two
-            // write different accumulators, and every commit covers all MMAs
-            // issued before it.
-            auto try_pv = [&]() -> bool {
-                if (npend == 0) return false;
-                const Pending r = pend0;
-                const int ob = r.oseq & 1;
-                bool ready = mbar_test(p_full + (r.g & 1), (r.g >> 1) & 1);
-                if (ready && r.first && r.oseq >= 2)   // the epilogue has read this O^T buffer
-                    ready = mbar_test(o_free + ob, ((r.oseq >> 1) - 1) & 1);
-                if (!ready) return false;
-                tc::fence_after();
-                const int st = r.g % nst;
-                const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st) + LY::KV_BYTES), LY::BOXT, 1024);
-                const uint64_t b0 = tc::sdesc_none(smem_u32(smem + ly.pt(r.g & 1)), 256, 128);
-                const uint32_t od = tO + (uint32_t)(NHP * ob);
-                const int nk = (r.nv + 15) / 16;             // 16-token slices holding tokens
-                for (int kk = 0; kk < nk; ++kk)
-                    tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
-                               (r.first && kk == 0) ? 0u : 1u);
-                tc::commit(empty + st);          // the stage slot may be refilled
-                if (r.last) tc::commit(o_done + ob);
-                pend0 = pend1;
-                --npend;
-                return true;
-            };
             while (true) {
                 bool prog = false;
                 // ---- the next unit, for the S side
@@ -1482,7 +1453,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                     }
                 }
                 // ---- O^T += V^T P^T of the oldest pending stage
-                if (try_pv()) prog = true;
+                if (npend > 0) {
+                    const Pending r = pend0;
+                    const int ob = r.oseq & 1;
+                    bool ready = mbar_test(p_full + (r.g & 1), (r.g >> 1) & 1);
+                    if (ready && r.first && r.oseq >= 2)   // the epilogue has read this O^T buffer
+                        ready = mbar_test(o_free + ob, ((r.oseq >> 1) - 1) & 1);
+                    if (ready) {
+                        tc::fence_after();
+                        const int st = r.g % nst;
+                        const uint64_t a0 = tc::sdesc_sw128(smem_u32(smem + ly.ring(st) + LY::KV_BYTES), LY::BOXT, 1024);
+                        const uint64_t b0 = tc::sdesc_none(smem_u32(smem + ly.pt(r.g & 1)), 256, 128);
+                        const uint32_t od = tO + (uint32_t)(NHP * ob);
+                        const int nk = (r.nv + 15) / 16;             // 16-token slices holding tokens
+                        for (int kk = 0; kk < nk; ++kk)
+                            tc::mma_ss(od, a0 + (uint64_t)(kk * 128), b0 + (uint64_t)(kk * 32), ID_O,
+                                       (r.first && kk == 0) ? 0u : 1u);
+                        tc::commit(empty + st);          // the stage slot may be refilled
+                        if (r.last) tc::commit(o_done + ob);
+                        pend0 = pend1;
+                        --npend;
+                        prog = true;
+                    }
+                }
                 // ---- S^T of the unit's next stage
                 if (have && npend < 2) {
                     const int g = d.stage_base + c, st = g % nst;
@@ -1492,12 +1485,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
                         const uint64_t b0 = tc::sdesc_sw128(smem_u32(smem + ly.q(slot)), 16, 1024);
                         const uint32_t sd = tS + (uint32_t)(NHP * (g & 1));
 #pragma unroll
-                        for (int k = 0; k < D / 16; ++k) {   // descriptor start fields in 16-byte units
+                        for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
                             tc::mma_ss(sd, a0 + (uint64_t)((k >> 2) * (LY::BOXT >> 4) + (k & 3) * 2),
                                        b0 + (uint64_t)((k >> 2) * (LY::QT / LY::NBOX >> 4) + (k & 3) * 2), ID_S,
                                        k > 0 ? 1u : 0u);
-                            if ((k & 1) && k + 1 < D / 16) try_pv();
-                        }
                         tc::commit(s_full + (g & 1));
                         if (c == d.n_stages - 1) tc::commit(uempty + slot);   // Q tile no longer read
                         const Pending nw{g, min(TTOK, d.t1 - (d.t0 + c * TTOK)), oseq, c == 0,

@@ -17,9 +17,9 @@
 //   O += P V        M = 128, N = head_dim, K = 64 keys    (tcgen05, A = P from
 //                   TMEM, B = V from smem, fp32 in TMEM)
 // Warps: 0-3 softmax + epilogue of tile 0, 4-7 of tile 1 (thread = one row =
-// one tensor-memory lane), 8 TMA producer, 9 MMA issuer (one thread).  The
-// two softmax groups run side by side (two warps per SM sub-partition) while
-// the tensor core works on the other tile; S (and the P written over it) is
+// one tensor-memory lane), 8 TMA producer, 9 and 10 the MMA issuers of tiles
+// 0 and 1 (one thread each).  The two softmax groups run side by side (two
+// warps per SM sub-partition) while the tensor core works on the other tile; S (and the P written over it) is
 // double-buffered in tensor memory per tile.  With no P in shared memory the
 // K/V ring holds five 64-key stages: a stage stays in its slot for the copy's
 // latency plus the S -> softmax -> PV chain, so the ring depth sets the pace.  The row maximum m is moved lazily:
@@ -45,7 +45,7 @@ namespace {
 constexpr int PF_KT = 64;          // keys per stage (N of S, K of PV)
 constexpr int PF_M = 128;          // query rows per tile
 constexpr int PF_TILES = 2;        // query tiles per CTA
-constexpr int PF_THREADS = 320;    // 8 softmax warps, producer, MMA issuer
+constexpr int PF_THREADS = 352;    // 8 softmax warps, producer, 2 MMA issuers
 constexpr int PF_MAX_STAGES = 6;
 constexpr float kPfRescaleLog2 = 8.f;
 constexpr uint32_t PF_FULL = 0xffffffffu;
@@ -65,7 +65,7 @@ struct PrefillParams {
 // boundary, as the 128-byte swizzle wants):
 //   Q        per tile NBOX boxes of [128 rows][128 B]
 //   ring     nst stages of K then V, each NBOX boxes of [64 keys][128 B]
-//   barriers, per-stage valid-piece masks, misc
+//   barriers, misc
 // P never goes to shared memory: the softmax writes it into tensor memory
 // over the S columns it came from, and the PV MMA reads it from there.
 template <int D>
@@ -89,8 +89,7 @@ struct PfLayout {
         return (size_t)PF_TILES * Q_BYTES + (size_t)st * STAGE_BYTES;
     }
     __host__ __device__ size_t bars() const { return ring(nst); }
-    __host__ __device__ size_t masks() const { return bars() + (size_t)(2 * nst + NBAR_FIXED) * 8; }
-    __host__ __device__ size_t misc() const { return ((masks() + 4 * (size_t)nst + 15) / 16) * 16; }
+    __host__ __device__ size_t misc() const { return ((bars() + (size_t)(2 * nst + NBAR_FIXED) * 8 + 15) / 16) * 16; }
     __host__ __device__ size_t total() const { return misc() + 64; }
 };
 
@@ -145,6 +144,29 @@ __device__ __forceinline__ void tm_ld32(uint32_t taddr, uint32_t (&r)[32]) {
           "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
           "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// 64 columns of this warp's lane quarter in one load, waiting for it.
+__device__ __forceinline__ void tm_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,"
+        "%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,"
+        "%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+          "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+          "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+          "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+          "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+          "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+          "=r"(r[62]), "=r"(r[63])
         : "r"(taddr)
         : "memory");
 }
@@ -216,17 +238,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + ly.bars());
     uint64_t* empty = full + nst;
     uint64_t* q_full = empty + nst;
-    uint64_t* fin = q_full + 1;                    // issuer's final drain
-    // per tile t: s_full[2] (S in tensor memory), kind 1 unused, p_full[2] (P
-    // written by the 4 softmax warps), pv_done[2] (PV complete)
-    auto tbar = [&](int t, int kind, int b) { return fin + 1 + t * 8 + kind * 2 + b; };
-    int* masks = reinterpret_cast<int*>(smem + ly.masks());
+    uint64_t* tb = q_full + 2;
+    // per tile t: s_full[2] (S in tensor memory), fin (its issuer's final
+    // drain) and one spare, p_full[2] (P written by the 4 softmax warps),
+    // pv_done[2] (PV complete)
+    auto tbar = [&](int t, int kind, int b) { return tb + t * 8 + kind * 2 + b; };
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
     volatile int* abort_flag = misc;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 8);
 
     if (tid == 0) {
-        for (int k = 0; k < 2 * nst + LY::NBAR_FIXED; ++k) mbar_init(full + k, 1);
+        // empty: one arrival per tile's issuer
+        for (int k = 0; k < 2 * nst + LY::NBAR_FIXED; ++k) mbar_init(full + k, k >= nst && k < 2 * nst ? ntile : 1);
         for (int t = 0; t < PF_TILES; ++t)
             for (int b = 0; b < 2; ++b) mbar_init(tbar(t, 2, b), 4);   // p_full
         misc[0] = 0;
@@ -275,7 +298,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             const uint32_t want = __reduce_or_sync(PF_FULL, exists ? 1u << piece : 0u);
             const uint32_t got = __reduce_or_sync(PF_FULL, live ? 1u << piece : 0u);
             if (lane == 0) {
-                masks[st] = (int)got;
                 if (want & ~got) set_err(p.err, PA_DEV_BAD_BLOCK);
                 if (got)
                     mbar_arrive_expect_tx(full + st, (uint32_t)__popc(got) * 2u * PR * (D * 2));
@@ -297,65 +319,65 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             mbar_wait(q_full, 0);
         }
         __syncwarp();
-    } else if (warp == 9) {
-        // ================================================= MMA issuer (one thread)
-        // Per stage c: S of both tiles, then PV of both tiles for stage c - 1,
-        // so the tensor core computes while the softmax groups work.
-        if (lane == 0) {
+    } else if (warp == 9 || warp == 10) {
+        // ================================================= MMA issuers (one thread each)
+        // Warp 9 issues tile 0's MMAs and warp 10 tile 1's: one thread takes
+        // ~70 cycles to issue an MMA whatever its size, and two issuing warps
+        // get about 1.4x as many through the tensor core as one.  Per stage c:
+        // S(c), then PV(c - 1), so the tensor core computes while the softmax
+        // warps work.  Each issuer arrives on a stage's `empty` barrier once
+        // its MMAs reading that stage are complete (after waiting for the
+        // stage's data, so an arrival never counts toward an earlier round).
+        const int t = warp - 9;
+        if (lane == 0 && t < ntile) {
             constexpr uint32_t ID_S = tc::idesc_f16<T>(false, false, PF_M, PF_KT);
             constexpr uint32_t ID_O = tc::idesc_f16<T>(false, true, PF_M, D);
+            const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
+            const uint32_t tS = tmem + (uint32_t)(t * LY::TM_TILE);
             bool ok = pf_wait(q_full, 0, abort_flag, p.err);
             for (int c = 0; ok && c <= nkt_all; ++c) {
                 if (c < nkt_all) {
                     const int st = c % nst, b = c & 1;
                     ok = pf_wait(full + st, (c / nst) & 1, abort_flag, p.err);
-                    const uint64_t kd = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
-#pragma unroll
-                    for (int t = 0; t < PF_TILES; ++t) {
-                        if (!ok || t >= ntile || c >= nkt[t]) continue;
+                    if (!ok) break;
+                    if (c < nkt[t]) {
                         // S buffer b last held S(c - 2), whose P the PV of
                         // stage c - 2 reads from it: that PV was issued in
                         // the previous round, and this thread's MMAs run in
                         // the order issued
                         tc::fence_after();
-                        const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
-                        const uint32_t sd = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * b);
+                        const uint64_t kd = tc::sdesc_sw128(smem_u32(smem + ly.ring(st)), 16, 1024);
 #pragma unroll
                         for (int k = 0; k < D / 16; ++k)   // descriptor start fields in 16-byte units
-                            tc::mma_ss(sd, qd + (uint64_t)((k >> 2) * (LY::QBOX >> 4) + (k & 3) * 2),
+                            tc::mma_ss(tS + (uint32_t)(PF_KT * b),
+                                       qd + (uint64_t)((k >> 2) * (LY::QBOX >> 4) + (k & 3) * 2),
                                        kd + (uint64_t)((k >> 2) * (LY::KBOX >> 4) + (k & 3) * 2), ID_S,
                                        k > 0 ? 1u : 0u);
                         tc::commit(tbar(t, 0, b));
                     }
-                    if (!ok) break;
                 }
                 if (c >= 1) {
                     const int m = c - 1, bm = m & 1, stm = m % nst;
-                    const uint64_t vd =
-                        tc::sdesc_sw128(smem_u32(smem + ly.ring(stm) + LY::KV_BYTES), LY::KBOX, 1024);
-#pragma unroll
-                    for (int t = 0; t < PF_TILES; ++t) {
-                        if (!ok || t >= ntile || m >= nkt[t]) continue;
+                    if (m < nkt[t]) {
                         ok = pf_wait(tbar(t, 2, bm), (m >> 1) & 1, abort_flag, p.err);
                         if (!ok) break;
                         tc::fence_after();
                         // A = P in tensor memory (lane = row, column = two keys),
                         // B = the V stage (MN-major)
-                        const uint32_t pt = tmem + (uint32_t)(t * LY::TM_TILE + PF_KT * bm);
-                        const uint32_t od = tmem + (uint32_t)(t * LY::TM_TILE + 2 * PF_KT);
+                        const uint64_t vd =
+                            tc::sdesc_sw128(smem_u32(smem + ly.ring(stm) + LY::KV_BYTES), LY::KBOX, 1024);
 #pragma unroll
                         for (int kk = 0; kk < PF_KT / 16; ++kk)
-                            tc::mma_ts(od, pt + (uint32_t)(kk * 8), vd + (uint64_t)(kk * 128), ID_O,
-                                       (m > 0 || kk > 0) ? 1u : 0u);
+                            tc::mma_ts(tS + (uint32_t)(2 * PF_KT), tS + (uint32_t)(PF_KT * bm + kk * 8),
+                                       vd + (uint64_t)(kk * 128), ID_O, (m > 0 || kk > 0) ? 1u : 0u);
                         tc::commit(tbar(t, 3, bm));
                     }
-                    if (!ok) break;
-                    tc::commit(empty + stm);           // the stage slot may be refilled
+                    tc::commit(empty + stm);           // this tile is done with the stage slot
                 }
             }
-            // every MMA of this CTA completes before tensor memory is freed
-            tc::commit(fin);
-            mbar_wait(fin, 0);
+            // every MMA of this thread completes before tensor memory is freed
+            tc::commit(tbar(t, 1, 0));
+            mbar_wait(tbar(t, 1, 0), 0);
         }
         __syncwarp();
     } else {
@@ -373,34 +395,42 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const float sl = p.scale_log2e;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
+        // Which pieces of a stage hold loaded blocks: the producer's rule
+        // (piece inside the CTA's key range, table entry in range), read from
+        // the table here one stage ahead, so that only stages that need their
+        // V rows zeroed wait for the copy themselves (the S MMA already did).
+        const int32_t* trow = p.tables + (size_t)s * p.mbps;
+        const int npc = PF_KT / PR;
+        const uint32_t all_pieces = (1u << npc) - 1u;
+        auto piece_blk = [&](int c) {
+            const int tok = c * PF_KT + lane * PR;
+            return lane < npc && tok < kend ? __ldg(trow + (tok >> p.bs_log2)) : -1;
+        };
+        int blk_next = my_nkt > 0 ? piece_blk(0) : -1;
         for (int c = 0; c < my_nkt; ++c) {
-            const int b = c & 1, st = c % nst;
-            ok = __all_sync(PF_FULL, pf_wait(tbar(t, 0, b), (c >> 1) & 1, abort_flag, p.err) &&
-                                         pf_wait(full + st, (c / nst) & 1, abort_flag, p.err));
+            const int b = c & 1;
+            const int blk = blk_next;
+            if (c + 1 < my_nkt) blk_next = piece_blk(c + 1);
+            const uint32_t vmask = __ballot_sync(PF_FULL, blk >= 0 && blk < p.NB);
+            ok = __all_sync(PF_FULL, pf_wait(tbar(t, 0, b), (c >> 1) & 1, abort_flag, p.err));
             if (!ok) break;
             tc::fence_after();
-            const uint32_t vmask = (uint32_t)masks[st];
             // keys of this stage the row may see: the first `lim` by position,
             // and only those of pieces whose block was loaded
             const int lim = pos - c * PF_KT + 1;
-            const bool whole = __all_sync(PF_FULL, lim >= PF_KT && vmask == (1u << (PF_KT / PR)) - 1u);
+            const bool whole = __all_sync(PF_FULL, lim >= PF_KT && vmask == all_pieces);
             const uint32_t tSb = tS + (uint32_t)(PF_KT * b) + lq;
-            // pass 1: the row maximum of the raw scores (the scale is positive)
+            // the 64 scores of the row, then their maximum (the scale is positive)
+            uint32_t v[PF_KT];
+            tm_ld64(tSb, v);
             float mraw = -INFINITY;
+            if (whole) {                               // warp-uniform: no key is hidden
 #pragma unroll
-            for (int h = 0; h < PF_KT / 32; ++h) {
-                uint32_t v[32];
-                tm_ld32(tSb + (uint32_t)(32 * h), v);
-                if (whole) {                           // warp-uniform: no key is hidden
+                for (int i = 0; i < PF_KT; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
+            } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int k = 32 * h + i;
-                        if (k < lim && ((vmask >> (k >> prl)) & 1u)) mraw = fmaxf(mraw, __uint_as_float(v[i]));
-                    }
-                }
+                for (int i = 0; i < PF_KT; ++i)
+                    if (i < lim && ((vmask >> (i >> prl)) & 1u)) mraw = fmaxf(mraw, __uint_as_float(v[i]));
             }
             const float mt = mraw * sl;
             const bool need = mt > m_ref + kPfRescaleLog2;
@@ -424,27 +454,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 }
                 if (need) m_ref = mt;
             }
-            // pass 2: P = exp2(s * scale * log2 e - m), rounded, written as
-            // 16-bit pairs over columns [0, 32) of S buffer b (each half reads
-            // 32 score columns before it overwrites 16 already-read ones); the
-            // two stores complete before P is handed to the MMA issuer
+            // P = exp2(s * scale * log2 e - m), rounded, written as 16-bit pairs
+            // over columns [0, 32) of S buffer b (all 64 scores are in
+            // registers); both stores complete before P is handed to the issuer
             const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
-            float lsum = 0.f;
             // packed fp32x2: z = s * scale * log2 e - m for two keys at once; the
             // row sum adds the weights as rounded to T (what the PV MMA multiplies)
             const uint64_t SL2 = f2_pack(sl, sl), NM2 = f2_pack(nmr, nmr), ONE2 = f2_pack(1.f, 1.f);
             uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < PF_KT / 32; ++h) {
-                uint32_t w[16], v[32];
-                tm_ld32(tSb + (uint32_t)(32 * h), v);
+                uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
+                    const int k0 = 32 * h + 2 * i;
                     float z0, z1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])),
-                                     SL2, NM2), z0, z1);
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[k0]), __uint_as_float(v[k0 + 1])), SL2, NM2),
+                              z0, z1);
                     if (!whole) {
-                        const int k0 = 32 * h + 2 * i;
                         if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
                         if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                     }
@@ -457,15 +484,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             {
                 float a0, a1;
                 f2_unpack(acc2, a0, a1);
-                lsum = a0 + a1;
+                l += a0 + a1;
             }
-            l += lsum;
-            if (r < PF_KT) {
+            if ((c + 1) * PF_KT > kend || vmask != all_pieces) {
                 // rows past the CTA's key range or of a skipped block: zero V
-                // (both groups write the same zeros), visible to the MMA's
-                // async-proxy reads
+                // (both tiles' warps write the same zeros) once the stage's copy
+                // has landed, visible to the MMA's async-proxy reads
+                const int st = c % nst;
+                ok = __all_sync(PF_FULL, pf_wait(full + st, (c / nst) & 1, abort_flag, p.err));
+                if (!ok) break;
                 const int key = c * PF_KT + r;
-                if (key >= kend || !((vmask >> (r >> prl)) & 1u)) {
+                if (r < PF_KT && (key >= kend || !((vmask >> (r >> prl)) & 1u))) {
                     uint8_t* vrow = smem + ly.ring(st) + LY::KV_BYTES + r * 128;
 #pragma unroll
                     for (int bx = 0; bx < LY::NBOX; ++bx)

@@ -397,21 +397,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         bool ok = true;
         // Which pieces of a stage hold loaded blocks: the producer's rule
         // (piece inside the CTA's key range, table entry in range), read from
-        // the table here one stage ahead, so that only stages that need their
-        // V rows zeroed wait for the copy themselves (the S MMA already did).
+        // the table here so that only stages that need their V rows zeroed
+        // wait for the copy themselves (the S MMA already did).  Lane i holds
+        // the mask of stage 32k + i for the current group k of 32 stages and
+        // the next one, whose table entries load while the current is used.
         const int32_t* trow = p.tables + (size_t)s * p.mbps;
         const int npc = PF_KT / PR;
         const uint32_t all_pieces = (1u << npc) - 1u;
-        auto piece_blk = [&](int c) {
-            const int tok = c * PF_KT + lane * PR;
-            return lane < npc && tok < kend ? __ldg(trow + (tok >> p.bs_log2)) : -1;
+        auto stage_mask = [&](int c) {
+            uint32_t mk = 0;
+            for (int q = 0; q < npc; ++q) {
+                const int tok = c * PF_KT + q * PR;
+                if (c < my_nkt && tok < kend) {
+                    const int blk = __ldg(trow + (tok >> p.bs_log2));
+                    if (blk >= 0 && blk < p.NB) mk |= 1u << q;
+                }
+            }
+            return mk;
         };
-        int blk_next = my_nkt > 0 ? piece_blk(0) : -1;
+        uint32_t mask_cur = stage_mask(lane), mask_next = stage_mask(32 + lane);
         for (int c = 0; c < my_nkt; ++c) {
             const int b = c & 1;
-            const int blk = blk_next;
-            if (c + 1 < my_nkt) blk_next = piece_blk(c + 1);
-            const uint32_t vmask = __ballot_sync(PF_FULL, blk >= 0 && blk < p.NB);
+            if (c > 0 && (c & 31) == 0) {
+                mask_cur = mask_next;
+                mask_next = stage_mask(c + 32 + lane);
+            }
+            const uint32_t vmask = __shfl_sync(PF_FULL, mask_cur, c & 31);
             ok = __all_sync(PF_FULL, pf_wait(tbar(t, 0, b), (c >> 1) & 1, abort_flag, p.err));
             if (!ok) break;
             tc::fence_after();
@@ -458,8 +469,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             // over columns [0, 32) of S buffer b (all 64 scores are in
             // registers); both stores complete before P is handed to the issuer
             const float nmr = m_ref == -INFINITY ? 0.f : -m_ref;
-            // packed fp32x2: z = s * scale * log2 e - m for two keys at once; the
-            // row sum adds the weights as rounded to T (what the PV MMA multiplies)
+            // packed fp32x2: z = s * scale * log2 e - m for two keys at once, and
+            // the row sum of the weights before their rounding to T
             const uint64_t SL2 = f2_pack(sl, sl), NM2 = f2_pack(nmr, nmr), ONE2 = f2_pack(1.f, 1.f);
             uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
@@ -475,8 +486,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
                         if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                     }
-                    w[i] = pack2<T>(ex2_ftz(z0), ex2_ftz(z1));
-                    acc2 = f2_fma(Pairs<T>::from_word(w[i]), ONE2, acc2);
+                    const float e0 = ex2_ftz(z0), e1 = ex2_ftz(z1);
+                    w[i] = pack2<T>(e0, e1);
+                    acc2 = f2_fma(f2_pack(e0, e1), ONE2, acc2);
                 }
                 tm_st16_nowait(tSb + (uint32_t)(16 * h), w);
             }

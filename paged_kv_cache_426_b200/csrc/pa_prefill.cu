@@ -335,10 +335,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             const uint64_t qd = tc::sdesc_sw128(smem_u32(smem + ly.q(t)), 16, 1024);
             const uint32_t tS = tmem + (uint32_t)(t * LY::TM_TILE);
             bool ok = pf_wait(q_full, 0, abort_flag, p.err);
+            // ring slot and phase of stage c, and the slot of stage c - 1
+            int st = 0, stm = nst - 1;
+            uint32_t ph = 0;
             for (int c = 0; ok && c <= nkt_all; ++c) {
                 if (c < nkt_all) {
-                    const int st = c % nst, b = c & 1;
-                    ok = pf_wait(full + st, (c / nst) & 1, abort_flag, p.err);
+                    const int b = c & 1;
+                    ok = pf_wait(full + st, ph, abort_flag, p.err);
                     if (!ok) break;
                     if (c < nkt[t]) {
                         // S buffer b last held S(c - 2), whose P the PV of
@@ -357,7 +360,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     }
                 }
                 if (c >= 1) {
-                    const int m = c - 1, bm = m & 1, stm = m % nst;
+                    const int m = c - 1, bm = m & 1;
                     if (m < nkt[t]) {
                         ok = pf_wait(tbar(t, 2, bm), (m >> 1) & 1, abort_flag, p.err);
                         if (!ok) break;
@@ -374,6 +377,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                     }
                     tc::commit(empty + stm);           // this tile is done with the stage slot
                 }
+                stm = st;
+                if (++st == nst) { st = 0; ph ^= 1u; }
             }
             // every MMA of this thread completes before tensor memory is freed
             tc::commit(tbar(t, 1, 0));
@@ -436,8 +441,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             tm_ld64(tSb, v);
             float mraw = -INFINITY;
             if (whole) {                               // warp-uniform: no key is hidden
+                // eight independent chains, then a tree
+                float mx[8];
 #pragma unroll
-                for (int i = 0; i < PF_KT; ++i) mraw = fmaxf(mraw, __uint_as_float(v[i]));
+                for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(v[k]);
+#pragma unroll
+                for (int i = 8; i < PF_KT; ++i) mx[i & 7] = fmaxf(mx[i & 7], __uint_as_float(v[i]));
+#pragma unroll
+                for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                    for (int k = 0; k < w; ++k) mx[k] = fmaxf(mx[k], mx[k + w]);
+                mraw = mx[0];
             } else {
 #pragma unroll
                 for (int i = 0; i < PF_KT; ++i)

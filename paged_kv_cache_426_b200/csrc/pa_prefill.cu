@@ -34,6 +34,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "pa.h"
 #include "pa_common.cuh"
@@ -487,25 +488,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             // the row sum of the weights before their rounding to T
             const uint64_t SL2 = f2_pack(sl, sl), NM2 = f2_pack(nmr, nmr), ONE2 = f2_pack(1.f, 1.f);
             uint64_t acc2 = f2_pack(0.f, 0.f);
+            // two copies of the loop, so that the common one carries no masking
+            // (a per-pair test would split the unrolled loop into blocks the
+            // compiler cannot interleave)
+            auto exps = [&](auto masked) {
 #pragma unroll
-            for (int h = 0; h < PF_KT / 32; ++h) {
-                uint32_t w[16];
+                for (int h = 0; h < PF_KT / 32; ++h) {
+                    uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int k0 = 32 * h + 2 * i;
-                    float z0, z1;
-                    f2_unpack(f2_fma(f2_pack(__uint_as_float(v[k0]), __uint_as_float(v[k0 + 1])), SL2, NM2),
-                              z0, z1);
-                    if (!whole) {
-                        if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
-                        if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
+                    for (int i = 0; i < 16; ++i) {
+                        const int k0 = 32 * h + 2 * i;
+                        float z0, z1;
+                        f2_unpack(f2_fma(f2_pack(__uint_as_float(v[k0]), __uint_as_float(v[k0 + 1])), SL2, NM2),
+                                  z0, z1);
+                        if (decltype(masked)::value) {
+                            if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
+                            if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
+                        }
+                        const float e0 = ex2_ftz(z0), e1 = ex2_ftz(z1);
+                        w[i] = pack2<T>(e0, e1);
+                        acc2 = f2_fma(f2_pack(e0, e1), ONE2, acc2);
                     }
-                    const float e0 = ex2_ftz(z0), e1 = ex2_ftz(z1);
-                    w[i] = pack2<T>(e0, e1);
-                    acc2 = f2_fma(f2_pack(e0, e1), ONE2, acc2);
+                    tm_st16_nowait(tSb + (uint32_t)(16 * h), w);
                 }
-                tm_st16_nowait(tSb + (uint32_t)(16 * h), w);
-            }
+            };
+            if (whole) exps(std::false_type{});
+            else exps(std::true_type{});
             tm_wait_st();
             {
                 float a0, a1;

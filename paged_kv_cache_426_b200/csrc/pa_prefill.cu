@@ -18,15 +18,17 @@
 //                   TMEM, B = V from smem, fp32 in TMEM)
 // Warps: 0-3 softmax + epilogue of tile 0, 4-7 of tile 1 (thread = one row =
 // one tensor-memory lane), 8 TMA producer, 9 and 10 the MMA issuers of tiles
-// 0 and 1 (one thread each).  The two softmax groups run side by side (two
-// warps per SM sub-partition) while the tensor core works on the other tile; S (and the P written over it) is
-// double-buffered in tensor memory per tile.  With no P in shared memory the
-// K/V ring holds five 64-key stages: a stage stays in its slot for the copy's
-// latency plus the S -> softmax -> PV chain, so the ring depth sets the pace.  The row maximum m is moved lazily:
-// only when a stage exceeds it by 2^8 is O rescaled in tensor memory.  Keys
-// past the row's position get weight 0; keys past the CTA's key range or in a
-// block whose table entry is bad also get their V rows zeroed in shared
-// memory (the product 0 * V must not meet stale or non-finite data).
+// 0 and 1 (one thread each), 11 idle (it completes the third warpgroup, which
+// hands registers to the softmax warps).  The two softmax groups run side by
+// side (two warps per SM sub-partition); S (and the P written over it) is
+// double-buffered in tensor memory per tile, so the tensor core computes the
+// next stage's S while the softmax works.  With no P in shared memory the K/V
+// ring holds five 64-key stages, more than the copy latency needs.  The row
+// maximum m is moved lazily: only when a stage exceeds it by 2^8 is O
+// rescaled in tensor memory.  Keys past the row's position get weight 0; keys
+// past the CTA's key range or in a block whose table entry is bad also get
+// their V rows zeroed in shared memory (the product 0 * V must not meet stale
+// or non-finite data).
 //
 // Every wait is bounded (2 s): a timeout sets PA_DEV_TIMEOUT, makes the other
 // warps give up at their next wait, and the kernel returns.
@@ -46,7 +48,13 @@ namespace {
 constexpr int PF_KT = 64;          // keys per stage (N of S, K of PV)
 constexpr int PF_M = 128;          // query rows per tile
 constexpr int PF_TILES = 2;        // query tiles per CTA
-constexpr int PF_THREADS = 352;    // 8 softmax warps, producer, 2 MMA issuers
+// 3 warpgroups: 8 softmax warps, then producer, 2 MMA issuers and an idle
+// warp.  The block is launched with 168 registers a thread; the third
+// warpgroup gives registers back (setmaxnreg) and the softmax warpgroups take
+// them: 256 * 208 + 128 * 80 = 63488 <= 384 * 168 = 64512.
+constexpr int PF_THREADS = 384;
+constexpr int PF_REGS_HIGH = 208, PF_REGS_LOW = 80;
+static_assert(256 * PF_REGS_HIGH + 128 * PF_REGS_LOW <= PF_THREADS * 168, "register split");
 constexpr int PF_MAX_STAGES = 6;
 constexpr float kPfRescaleLog2 = 8.f;
 constexpr uint32_t PF_FULL = 0xffffffffu;
@@ -267,6 +275,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const int PR = p.bs >= 16 ? 16 : p.bs;         // rows of one TMA box (block piece)
     const int prl = p.bs >= 16 ? 4 : p.bs_log2;
 
+    if (warp >= 8) {
+    // (the whole warpgroup executes this, the idle warp 11 included)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(PF_REGS_LOW));
     if (warp == 8) {
         // ================================================= TMA producer
         if (lane == 0) {
@@ -386,7 +397,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             mbar_wait(tbar(t, 1, 0), 0);
         }
         __syncwarp();
+    }
     } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(PF_REGS_HIGH));   // both warpgroups
         // ================================================= softmax + epilogue (row of tile t)
         const int t = warp >> 2;
         const int r = tid & 127;
@@ -637,6 +650,13 @@ int pf_run(PfLaunch& L) {
                 return PA_ERR_CUDA;
             attr_set[dev & 63] = true;
         }
+    }
+    {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return PA_ERR_CUDA;
+        // the register split must fit in what the block is launched with, or
+        // the softmax warpgroups would wait for registers for ever
+        if ((long)fa.numRegs * PF_THREADS < 256L * PF_REGS_HIGH + 128L * PF_REGS_LOW) return PA_ERR_UNSUPPORTED;
     }
     kern<<<L.grid, PF_THREADS, smem, L.stream>>>(L.kmap, L.vmap, L.qmap, L.p);
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;

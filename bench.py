@@ -275,8 +275,10 @@ def run_prefill_bench(args):
     def write():
         pa.pa_reshape_and_cache(ch_k, ch_v, kc, vc, ch_slots, err_flag=err)
 
+    ws = pa.prefill_workspace(dev)
+
     def attend():
-        pa.pa_prefill(out, q, kc, vc, tab, lens, cu, max_q, b.scale, err_flag=err)
+        pa.pa_prefill(out, q, kc, vc, tab, lens, cu, max_q, b.scale, workspace=ws, err_flag=err)
 
     sampler = ClockSampler(0)
     sampler.start()

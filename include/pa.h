@@ -228,6 +228,12 @@ int pa_decode_ex(void* out, const void* query, const void* key_cache,
  *   cu_seqlens_q [num_seqs + 1] int32 device, 0 = cu[0] <= ... <= cu[num_seqs]
  *                = total_q
  *   max_query_len  an upper bound of every n_s (it sizes the launch)
+ *   workspace    device, >= PA_PREFILL_WORKSPACE_BYTES, 16-byte aligned, owned
+ *                by the caller: the work-item counter of the persistent launch
+ *                (one CTA per SM takes pairs of query tiles until none is
+ *                left).  Zero-filled before its first use; every call leaves
+ *                it zeroed again (also after a timeout), so it is reused as is.
+ *                Calls that may run at the same time need distinct workspaces.
  *   dtype        PA_F16 or PA_BF16 (tensor cores); PA_F32 -> PA_ERR_UNSUPPORTED
  * head_dim 64 or 128; num_q_heads / num_kv_heads in {1, 2, 4, 8}; block_size
  * 8, 16, 32, 64 or 128; every pointer 16-byte aligned.  Nothing is allocated;
@@ -237,12 +243,15 @@ int pa_decode_ex(void* out, const void* query, const void* key_cache,
  * leaves [0, total_q] (rows of that sequence may then be left unwritten);
  * PA_DEV_BAD_BLOCK for a table entry outside [0, num_blocks) that a chunk
  * reads (those tokens are skipped); PA_DEV_TIMEOUT as pa_decode.
- * Returns PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED or PA_ERR_CUDA. */
+ * Returns PA_OK, PA_ERR_INVALID (a null or short workspace included),
+ * PA_ERR_UNSUPPORTED or PA_ERR_CUDA. */
+#define PA_PREFILL_WORKSPACE_BYTES 64u
 int pa_prefill(void* out, const void* query, const void* key_cache, const void* value_cache,
                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
                const int32_t* cu_seqlens_q, int num_seqs, int total_q, int max_query_len,
                int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-               float scale, pa_dtype dtype, int32_t* err_flag, void* stream);
+               float scale, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+               int32_t* err_flag, void* stream);
 
 /* --------------------------------------------------------------------------
  * pa_copy_blocks - copy-on-write block copies.

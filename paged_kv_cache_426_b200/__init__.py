@@ -48,7 +48,7 @@ SIGNATURES = {
     "pa_decode_ex": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _i, _i, _i, _i, _f, _i, _vp,
                       _sz, _i, _vp, _vp, _vp], _i),
     "pa_prefill": ([_vp, _vp, _vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
-                    _i, _vp, _vp], _i),
+                    _vp, _sz, _i, _vp, _vp], _i),
     "pa_copy_blocks": ([_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "pa_allocator_create": ([_i, _pi32, _i, C.POINTER(_vp)], _i),
     "pa_allocator_destroy": ([_vp], None),
@@ -208,13 +208,26 @@ def pa_decode_static(out, query, key_cache, value_cache, block_tables, context_l
                                _stream(stream)), "pa_decode_static")
 
 
+PREFILL_WORKSPACE_BYTES = 64
+
+
+def prefill_workspace(device):
+    """A zero-filled pa_prefill workspace (every call leaves it zeroed, so one
+    serves all calls ordered on a stream)."""
+    return torch.zeros(PREFILL_WORKSPACE_BYTES // 4, dtype=torch.int32, device=device)
+
+
 def pa_prefill(out, query, key_cache, value_cache, block_tables, context_lens, cu_seqlens_q,
-               max_query_len, scale, *, err_flag=None, stream=None):
+               max_query_len, scale, *, workspace=None, err_flag=None, stream=None):
     """Causal attention of packed prefill chunks: out/query [T, Hq, D]; caches
     [NB, Hkv, bs, D]; block_tables int32 [S, max_blocks]; context_lens int32
     [S] (counting the chunk); cu_seqlens_q int32 [S + 1] (row offsets of the
-    chunks in query)."""
-    _cuda(out, query, key_cache, value_cache, block_tables, context_lens, cu_seqlens_q, err_flag)
+    chunks in query).  ``workspace``: from prefill_workspace (a fresh one per
+    call when None)."""
+    if workspace is None:
+        workspace = prefill_workspace(query.device)
+    _cuda(out, query, key_cache, value_cache, block_tables, context_lens, cu_seqlens_q, workspace,
+          err_flag)
     T, hq, d = query.shape
     NB, hkv, bs, _ = key_cache.shape
     S = context_lens.shape[0]
@@ -223,7 +236,8 @@ def pa_prefill(out, query, key_cache, value_cache, block_tables, context_lens, c
     check(lib.pa_prefill(_ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
                          _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
                          _ptr(cu_seqlens_q), S, T, int(max_query_len), hq, hkv, d, bs, NB,
-                         float(scale), pa_dtype(query), _ptr(err_flag), _stream(stream)),
+                         float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                         pa_dtype(query), _ptr(err_flag), _stream(stream)),
           "pa_prefill")
 
 

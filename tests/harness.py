@@ -175,6 +175,7 @@ class GpuPrefill:
         self.kc = torch.full(shape, fill, dtype=td, device=device)
         self.vc = torch.full(shape, fill, dtype=td, device=device)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        self.ws = pa.prefill_workspace(device)
         S = len(b.context_lens)
         ctx_s, chunk_s, ctx_k, ctx_v, ch_k, ch_v = [], [], [], [], [], []
         for s, (L, n) in enumerate(zip(b.context_lens, b.query_lens)):
@@ -210,7 +211,7 @@ class GpuPrefill:
 
     def attend(self):
         pa.pa_prefill(self.out, self.q, self.kc, self.vc, self.tab, self.lens, self.cu, self.max_q,
-                      self.b.scale, err_flag=self.err)
+                      self.b.scale, workspace=self.ws, err_flag=self.err)
 
     def step(self):
         self.write_chunks()

@@ -119,15 +119,17 @@ def test_prefill_bad_arguments_rejected_before_launch():
     device: arguments (args order: out, query, key_cache, value_cache,
     block_tables, max_blocks_per_seq, context_lens, cu_seqlens_q, num_seqs,
     total_q, max_query_len, Hq, Hkv, head_dim, block_size, num_blocks, scale,
-    dtype, err_flag, stream)."""
+    workspace, workspace_bytes, dtype, err_flag, stream)."""
     L = pa.lib
     f = 1 << 20                          # aligned, never dereferenced: validation fails first
-    ok = dict(mbps=4, S=2, T=8, maxq=8, hq=8, hkv=2, d=128, bs=16, nb=8, scale=0.125, dt=2)
+    ok = dict(mbps=4, S=2, T=8, maxq=8, hq=8, hkv=2, d=128, bs=16, nb=8, scale=0.125, dt=2,
+              ws=f, wsb=pa.PREFILL_WORKSPACE_BYTES)
 
     def call(ptr=f, **kw):
         a = dict(ok, **kw)
         return L.pa_prefill(ptr, f, f, f, f, a["mbps"], f, f, a["S"], a["T"], a["maxq"], a["hq"],
-                            a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["dt"], None, None)
+                            a["hkv"], a["d"], a["bs"], a["nb"], a["scale"], a["ws"], a["wsb"], a["dt"],
+                            None, None)
 
     assert call(S=0) == pa.PA_OK and call(T=0) == pa.PA_OK         # nothing to do
     assert call(ptr=None) == pa.PA_ERR_INVALID
@@ -142,6 +144,9 @@ def test_prefill_bad_arguments_rejected_before_launch():
     assert call(scale=0.0) == pa.PA_ERR_INVALID and call(scale=-1.0) == pa.PA_ERR_INVALID
     assert call(scale=float("inf")) == pa.PA_ERR_INVALID
     assert call(nb=0) == pa.PA_ERR_INVALID and call(mbps=0) == pa.PA_ERR_INVALID
+    assert call(ws=None) == pa.PA_ERR_INVALID                       # the item counter
+    assert call(wsb=pa.PREFILL_WORKSPACE_BYTES - 4) == pa.PA_ERR_INVALID
+    assert call(ws=f + 4) == pa.PA_ERR_INVALID                      # not 16-byte aligned
 
 
 def test_workspace_size_formula():

@@ -209,3 +209,33 @@ def test_prefix_cache_prefills_only_the_suffix():
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     check_close(out_f64(out, "bf16"), ref, "bf16", "prefix-cached prompt, suffix prefill")
+
+
+def test_workspace_left_zeroed_and_reused():
+    """The persistent launch takes work items from a counter in the caller's
+    workspace; every call leaves it zeroed (after a bad table entry too), so
+    back-to-back calls on one workspace give the same output.  More items
+    than SMs (about 300 pairs of tiles), so CTAs take several each."""
+    b = workloads.prefill_custom("bf16", [1200, 700, 900, 333, 1024, 65],
+                                 [1200, 300, 900, 333, 512, 65], 32, 8, 128, 16, seed=11)
+    g = GpuPrefill(b)
+    g.write_chunks()
+    ws = pa.prefill_workspace(g.out.device)
+    outs = []
+    for _ in range(3):
+        g.out.zero_()
+        pa.pa_prefill(g.out, g.q, g.kc, g.vc, g.tab, g.lens, g.cu, g.max_q, b.scale, workspace=ws,
+                      err_flag=g.err)
+        torch.cuda.synchronize()
+        assert int(g.err.item()) == 0
+        assert int(ws.abs().sum().item()) == 0
+        outs.append(g.out.clone())
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+    check_close(out_f64(outs[0], "bf16"), oracle.run_prefill(b).out, "bf16", "persistent items")
+    tab = g.tab.clone()
+    tab[0, 3] = -5                            # a bad entry: the call reports it, ws still zero
+    pa.pa_prefill(g.out, g.q, g.kc, g.vc, tab, g.lens, g.cu, g.max_q, b.scale, workspace=ws,
+                  err_flag=g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == pa.PA_DEV_BAD_BLOCK
+    assert int(ws.abs().sum().item()) == 0

@@ -583,6 +583,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 #pragma unroll
                         for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
                     mraw = mx[0];
+                } else if (vmask == all_pieces) {       // causal edge only
+#pragma unroll
+                    for (int i = 0; i < PF_KT; ++i)
+                        if (i < lim) mraw = fmaxf(mraw, __uint_as_float(v[i]));
                 } else {
 #pragma unroll
                     for (int i = 0; i < PF_KT; ++i)
@@ -618,10 +622,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 // the row sum of the weights before their rounding to T
                 const uint64_t SL2 = f2_pack(sl, sl), NM2 = f2_pack(nmr, nmr), ONE2 = f2_pack(1.f, 1.f);
                 uint64_t acc2 = f2_pack(0.f, 0.f);
-                // two copies of the loop, so that the common one carries no masking
-                // (a per-pair test would split the unrolled loop into blocks the
-                // compiler cannot interleave)
-                auto exps = [&](auto masked) {
+                // three copies of the loop (no masking; the causal edge; the causal
+                // edge and missing blocks), so that the common one carries no
+                // test (a per-pair test would split the unrolled loop into blocks
+                // the compiler cannot interleave)
+                auto exps = [&](auto mode) {
 #pragma unroll
                     for (int h = 0; h < PF_KT / 32; ++h) {
                         uint32_t w[16];
@@ -631,7 +636,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                             float z0, z1;
                             f2_unpack(f2_fma(f2_pack(__uint_as_float(v[k0]), __uint_as_float(v[k0 + 1])), SL2, NM2),
                                       z0, z1);
-                            if (decltype(masked)::value) {
+                            if (decltype(mode)::value == 1) {
+                                z0 = k0 < lim ? z0 : -INFINITY;
+                                z1 = k0 + 1 < lim ? z1 : -INFINITY;
+                            } else if (decltype(mode)::value == 2) {
                                 if (!(k0 < lim && ((vmask >> (k0 >> prl)) & 1u))) z0 = -INFINITY;
                                 if (!(k0 + 1 < lim && ((vmask >> ((k0 + 1) >> prl)) & 1u))) z1 = -INFINITY;
                             }
@@ -642,8 +650,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                         tm_st16_nowait(tSb + (uint32_t)(16 * h), w);
                     }
                 };
-                if (whole) exps(std::false_type{});
-                else exps(std::true_type{});
+                if (whole) exps(std::integral_constant<int, 0>{});
+                else if (vmask == all_pieces) exps(std::integral_constant<int, 1>{});
+                else exps(std::integral_constant<int, 2>{});
                 tm_wait_st();
                 {
                     float a0, a1;

@@ -71,6 +71,7 @@ struct PrefillParams {
     const int32_t* cu;
     int S, total_q, max_q, npair, Hq, Hkv, mbps, NB, bs, bs_log2, nst;
     int n_items;       // npair * S * Hkv work items (pairs of query tiles)
+    int out32;         // out is 32-byte aligned: rows are written 32 bytes a store
     float scale_log2e;
     int32_t* err;
     int* ws;           // [0] next item, [1] CTAs done (zero between calls)
@@ -183,6 +184,14 @@ __device__ __forceinline__ void tm_st16_nowait(uint32_t taddr, const uint32_t (&
         : "memory");
 }
 __device__ __forceinline__ void tm_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 bytes to global memory in one store (the address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* dst, const uint32_t* w) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 ::"l"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]),
+                   "r"(w[7])
+                 : "memory");
+}
 
 // 2^x by the PTX ex2.approx instruction with subnormal results flushed to
 // zero: softmax weights below 2^-126 are zero after rounding to 16 bits
@@ -707,14 +716,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
 #pragma unroll
                         for (int i = 0; i < 64; ++i) o[i] = 0u;
                     }
-                    if (store) {
-                        uint4* o4 = reinterpret_cast<uint4*>(dst + 64 * h);
+                    uint32_t w[32];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            o4[i] = make_uint4(pack2<T>(__uint_as_float(o[8 * i]) * inv, __uint_as_float(o[8 * i + 1]) * inv),
-                                               pack2<T>(__uint_as_float(o[8 * i + 2]) * inv, __uint_as_float(o[8 * i + 3]) * inv),
-                                               pack2<T>(__uint_as_float(o[8 * i + 4]) * inv, __uint_as_float(o[8 * i + 5]) * inv),
-                                               pack2<T>(__uint_as_float(o[8 * i + 6]) * inv, __uint_as_float(o[8 * i + 7]) * inv));
+                    for (int i = 0; i < 32; ++i)
+                        w[i] = pack2<T>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+                    if (store) {
+                        // each lane writes its own row: whole 32-byte sectors a
+                        // store when the rows are 32-byte aligned
+                        if (p.out32) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) st_global_v8(dst + 64 * h + 16 * i, &w[8 * i]);
+                        } else {
+                            uint4* o4 = reinterpret_cast<uint4*>(dst + 64 * h);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                o4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                        }
                     }
                 }
             }
@@ -916,6 +933,7 @@ int pa_prefill(void* out, const void* query, const void* key_cache, const void* 
     p.scale_log2e = scale * 1.4426950408889634f;
     p.err = err_flag;
     p.n_items = (int)n_items;
+    p.out32 = (reinterpret_cast<uintptr_t>(out) & 31) == 0 ? 1 : 0;
     p.ws = static_cast<int*>(workspace);
     L.grid = dim3((unsigned)grid);
     L.stream = (cudaStream_t)stream;

@@ -239,3 +239,20 @@ def test_workspace_left_zeroed_and_reused():
     torch.cuda.synchronize()
     assert int(g.err.item()) == pa.PA_DEV_BAD_BLOCK
     assert int(ws.abs().sum().item()) == 0
+
+
+def test_output_only_16_byte_aligned():
+    """The output rows are written 32 bytes a store when `out` is 32-byte
+    aligned; an output starting 16 bytes into an allocation takes the 16-byte
+    stores and must match the same way."""
+    b = workloads.prefill_custom("f16", [300, 129], [300, 64], 8, 2, 128, 16, seed=5)
+    g = GpuPrefill(b)
+    g.write_chunks()
+    T, hq, d = g.q.shape
+    big = torch.zeros(T * hq * d + 8, dtype=g.out.dtype, device=g.out.device)
+    out = big[8:].view(T, hq, d)                 # 16 bytes past a 256-byte boundary
+    assert out.data_ptr() % 32 == 16
+    pa.pa_prefill(out, g.q, g.kc, g.vc, g.tab, g.lens, g.cu, g.max_q, b.scale, err_flag=g.err)
+    torch.cuda.synchronize()
+    assert int(g.err.item()) == 0
+    check_close(out_f64(out, "f16"), oracle.run_prefill(b).out, "f16", "16-byte aligned output")

@@ -107,8 +107,11 @@ struct PfLayout {
     }
     __host__ __device__ size_t bars() const { return ring(nst); }
     __host__ __device__ size_t misc() const { return ((bars() + (size_t)(2 * nst + NBAR_FIXED) * 8 + 15) / 16) * 16; }
-    __host__ __device__ size_t items() const { return misc() + 64; }   // two 128-byte item slots
-    __host__ __device__ size_t total() const { return items() + 256; }
+    // two item slots: the item (128 bytes) and the loaded-piece masks of its
+    // first 64 stages
+    static constexpr int SLOT = 128 + 64 * 4;
+    __host__ __device__ size_t items() const { return misc() + 64; }
+    __host__ __device__ size_t total() const { return items() + 2 * SLOT; }
 };
 
 // 3-D tiled tensor copy global -> shared (box given by the tensor map).
@@ -281,7 +284,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     int* misc = reinterpret_cast<int*>(smem + ly.misc());
     volatile int* abort_flag = misc;
     // the two item slots of the queue (128 bytes each)
-    auto item_slot = [&](int k) { return reinterpret_cast<PfItem*>(smem + ly.items() + (k & 1) * 128); };
+    auto item_slot = [&](int k) { return reinterpret_cast<PfItem*>(smem + ly.items() + (k & 1) * LY::SLOT); };
+    auto slot_masks = [&](int k) { return reinterpret_cast<uint32_t*>(smem + ly.items() + (k & 1) * LY::SLOT + 128); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc + 8);
 
     if (tid == 0) {
@@ -304,6 +308,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     const uint32_t tmem = *tmem_slot;
     const int PR = p.bs >= 16 ? 16 : p.bs;         // rows of one TMA box (block piece)
     const int prl = p.bs >= 16 ? 4 : p.bs_log2;
+    // loaded-piece mask of stage c of an item: pieces inside its key range
+    // whose table entry is in range (the pieces the producer loads)
+    auto piece_mask = [&](const PfItem& it, int c, int cmax) {
+        const int32_t* trow = p.tables + (size_t)it.s * p.mbps;
+        const int npc = PF_KT / PR;
+        uint32_t mk = 0;
+        for (int qq = 0; qq < npc; ++qq) {
+            const int tok = c * PF_KT + qq * PR;
+            if (c < cmax && tok < it.kend) {
+                const int blk = __ldg(trow + (tok >> p.bs_log2));
+                if (blk >= 0 && blk < p.NB) mk |= 1u << qq;
+            }
+        }
+        return mk;
+    };
 
     if (warp >= 8) {
     // (the whole warpgroup executes this)
@@ -325,10 +344,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
             if (lane == 0) q = atomicAdd(p.ws, 1);
             q = __shfl_sync(PF_FULL, q, 0);
             PfItem it;
+            uint32_t m0 = 0, m1 = 0;                   // masks of stages lane, 32 + lane
             if (q < p.n_items) {
                 it = pf_item<G>(p, q);
                 if (it.bad && it.first && lane == 0) set_err(p.err, PA_DEV_BAD_LEN);
                 if (it.ntile == 0) continue;           // past its sequence's chunk
+                m0 = piece_mask(it, lane, it.nkt_all);
+                m1 = piece_mask(it, 32 + lane, it.nkt_all);
             } else {
                 q = -1;
             }
@@ -338,13 +360,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                 if (lane == 0) w = pf_wait(item_empty + (k & 1), ((k - 2) >> 1) & 1, abort_flag, p.err);
                 if (!__shfl_sync(PF_FULL, w, 0)) break;
             }
+            slot_masks(k)[lane] = m0;
+            slot_masks(k)[32 + lane] = m1;
             if (lane == 0) {
                 PfItem* slot = item_slot(k);
                 if (q >= 0) *slot = it;
                 slot->q = q;
                 slot->g = g;
-                mbar_arrive(item_full + (k & 1));
             }
+            __syncwarp();                              // the lanes' writes before the release
+            if (lane == 0) mbar_arrive(item_full + (k & 1));
             __syncwarp();
             ++k;
             if (q < 0) break;
@@ -519,36 +544,24 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const float sl = p.scale_log2e;
         const int npc = PF_KT / PR;
         const uint32_t all_pieces = (1u << npc) - 1u;
-        // Which pieces of a stage hold loaded blocks: the producer's rule
-        // (piece inside the item's key range, table entry in range), read from
-        // the table here so that only stages that need their V rows zeroed
-        // wait for the copy themselves (the S MMA already did).  Lane i holds
-        // the mask of stage 32k + i for the current group k of 32 stages and
-        // the next one, whose table entries load meanwhile.
-        auto stage_mask = [&](const PfItem& it, int c) {
-            const int32_t* trow = p.tables + (size_t)it.s * p.mbps;
-            uint32_t mk = 0;
-            for (int qq = 0; qq < npc; ++qq) {
-                const int tok = c * PF_KT + qq * PR;
-                if (c < it.nkt[t] && tok < it.kend) {
-                    const int blk = __ldg(trow + (tok >> p.bs_log2));
-                    if (blk >= 0 && blk < p.NB) mk |= 1u << qq;
-                }
-            }
-            return mk;
-        };
+        // Which pieces of a stage hold loaded blocks (piece_mask, the
+        // producer's rule), known here without waiting for the copy, so that
+        // only stages that need their V rows zeroed wait for it themselves
+        // (the S MMA already did).  Lane i holds the mask of stage 32k + i for
+        // the current group k of 32 stages and the next one: the producer
+        // hands the first two groups on with the item, later groups are read
+        // from the table a group ahead.
+        auto stage_mask = [&](const PfItem& it, int c) { return piece_mask(it, c, it.nkt[t]); };
         // take item k from the queue, with the masks of its first two groups
-        // of stages
+        // of stages (the producer's, from the slot)
         auto take = [&](int k, PfItem& it, uint32_t& mc, uint32_t& mn) {
             if (!__all_sync(PF_FULL, pf_wait(item_full + (k & 1), (k >> 1) & 1, abort_flag, p.err)))
                 return false;
             it = *item_slot(k);
+            mc = slot_masks(k)[lane];
+            mn = slot_masks(k)[32 + lane];
             __syncwarp();
             if (lane == 0) mbar_arrive(item_empty + (k & 1));
-            if (it.q >= 0 && t < it.ntile) {
-                mc = stage_mask(it, lane);
-                mn = stage_mask(it, 32 + lane);
-            }
             return true;
         };
         int gs = 0;                                    // this tile's stage count (S buffers, phases)

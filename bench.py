@@ -1114,8 +1114,10 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--only", dest="all_workloads", action="store_false",
                     help="measure only --workload (no per_workload section)")
-    ap.add_argument("--extra-steps", type=int, default=10,
-                    help="timed steps of each other decode batch in per_workload")
+    ap.add_argument("--extra-steps", type=int, default=24,
+                    help="decode steps of each other batch in per_workload (the e2e leg times "
+                         "all but --warmup of them, pipelined: a short run weighs the pipeline's "
+                         "fill and drain too much)")
     ap.add_argument("--sweep", action="store_true",
                     help="block-size / indirection study instead of the benchmark line")
     ap.add_argument("--waste", action="store_true",

@@ -779,13 +779,13 @@ def run_e2e(sess, w, args, world):
     """Same metric through the public API with host buffers, every step: the
     live C++ manager's appends and block tables (host), the step's H2D copies
     from pinned buffers, copy-on-write copies, cache write, decode and the D2H
-    of out.  Steps are pipelined the way a serving loop runs them: while step
-    k's kernels run, the host prepares step k+1 (manager calls into the other
-    pinned set) and step k+1's inputs cross PCIe on a copy stream into the
-    other device set; out of step k returns on a third stream, and the host
-    waits for it one step later.  The device work of the copy and compute
-    stages is CUDA graphs captured beforehand from the same public calls, so
-    Python launch overhead does not pose as step time."""
+    of out.  Steps are pipelined the way a serving loop runs them: step k is
+    one CUDA graph of three branches, step k's cache write and decode, the H2D
+    copies of step k + 1's inputs into the other device set, and the D2H of
+    step k - 1's out, captured beforehand from the same public calls; while it
+    runs, the host prepares step k + 2 (manager calls into the pinned set step
+    k's copies have finished reading).  One graph launch per step: Python
+    launch overhead does not pose as step time."""
     pa = sess.pa
     dev = sess.dev
     _, mgr = sess.prefill(write=False)       # same script -> same pool state
@@ -796,7 +796,6 @@ def run_e2e(sess, w, args, world):
 
     def pinned_set():
         return dict(slots=torch.empty(S, dtype=torch.int64).pin_memory(),
-                    cow=torch.empty((S, 2), dtype=torch.int64).pin_memory(),
                     tab=torch.empty((S, mb), dtype=torch.int32).pin_memory(),
                     lens=torch.empty(S, dtype=torch.int32).pin_memory(),
                     out=torch.empty((S, hq, d), dtype=dt).pin_memory())
@@ -812,6 +811,7 @@ def run_e2e(sess, w, args, world):
                     out=torch.empty((S, hq, d), dtype=dt, device=dev))
     pins = [pinned_set(), pinned_set()]          # step k uses set k % 2
     devs = [device_set(), device_set()]
+    cow_pins = [torch.empty((S, 2), dtype=torch.int64).pin_memory() for _ in range(n)]
     # the batch of each step (which sequences run) is a step input like q/K/V
     seq_ids = [torch.tensor(w.step_seqs(k), dtype=torch.int64) for k in range(n)]
     qs = [w.step_q[k].pin_memory() for k in range(n)]
@@ -820,8 +820,8 @@ def run_e2e(sess, w, args, world):
     main = torch.cuda.current_stream()
     copy_s, out_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def h2d(k, b):
-        D, pin = devs[b], pins[b]
+    def h2d(k):
+        D, pin = devs[k % 2], pins[k % 2]
         D["q"].copy_(qs[k], non_blocking=True)
         D["k"].copy_(kk[k], non_blocking=True)
         D["v"].copy_(vv[k], non_blocking=True)
@@ -829,85 +829,95 @@ def run_e2e(sess, w, args, world):
         D["tab"].copy_(pin["tab"], non_blocking=True)
         D["lens"].copy_(pin["lens"], non_blocking=True)
 
-    def compute(b):
-        D = devs[b]
+    def d2h(k):
+        pins[k % 2]["out"].copy_(devs[k % 2]["out"], non_blocking=True)
+
+    def compute(k):
+        D = devs[k % 2]
         pa.pa_reshape_and_cache(D["k"], D["v"], sess.kc, sess.vc, D["slots"], err_flag=sess.err)
         pa.pa_decode(D["out"], D["q"], sess.kc, sess.vc, D["tab"], D["lens"], sess.max_len,
                      w.scale, partition_size=sess.P, workspace=sess.ws, err_flag=sess.err,
                      engine=sess.engine)
 
-    def host_part(k, b):
-        pin = pins[b]
-        _, cow = mgr.append_step(seq_ids[k], slots_out=pin["slots"], cow_out=pin["cow"])
+    def host_part(k):
+        pin = pins[k % 2]
+        _, cow = mgr.append_step(seq_ids[k], slots_out=pin["slots"], cow_out=cow_pins[k])
         _, lens = mgr.block_tables(seq_ids[k], mb, tables_out=pin["tab"], lens_out=pin["lens"])
-        ncow = cow.shape[0]
-        if ncow:                                 # copy-on-write pairs vary: never in a graph
-            dcow = devs[b]["cow"][:ncow]
-            dcow.copy_(pin["cow"][:ncow], non_blocking=True)
-            pa.pa_copy_blocks(sess.kc, sess.vc, dcow, err_flag=sess.err)
-        return ncow, lens
+        return cow.shape[0], lens
 
-    g_h2d, g_comp = [], []
-    for k in range(n):
+    def cow_copies(k, ncow):
+        # copy-on-write pairs vary: never in a graph; on the stream before step k
+        dcow = devs[k % 2]["cow"][:ncow]
+        dcow.copy_(cow_pins[k][:ncow], non_blocking=True)
+        pa.pa_copy_blocks(sess.kc, sess.vc, dcow, err_flag=sess.err)
+
+    def step_graph(k, first, last):
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=copy_s):
-            h2d(k, k % 2)
-        g_h2d.append(g)
-        g_comp.append(capture(lambda b=k % 2: compute(b)))
-    torch.cuda.synchronize()
-
-    ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
-    h2d_done, comp_done, out_done = ev(), ev(), ev()
-    stats = dict(bytes=0, h2d=0, d2h=0)
+        with torch.cuda.graph(g):
+            s0 = torch.cuda.current_stream()
+            copy_s.wait_stream(s0)
+            out_s.wait_stream(s0)
+            with torch.cuda.stream(copy_s):
+                if k + 1 <= last:
+                    h2d(k + 1)
+            with torch.cuda.stream(out_s):
+                if k - 1 >= first:
+                    d2h(k - 1)
+            compute(k)
+            s0.wait_stream(copy_s)
+            s0.wait_stream(out_s)
+        return g
 
     def run(ks, count):
-        pend = host_part(ks[0], ks[0] % 2)
+        first, last = ks[0], ks[-1]
+        graphs = [step_graph(k, first, last) for k in ks]
+        torch.cuda.synchronize()
+        done = [torch.cuda.Event() for _ in ks]
+        first_in = torch.cuda.Event()
+        t0 = time.perf_counter()
+        pend = {first: host_part(first)}
+        h2d(first)                               # the first step's inputs
+        first_in.record(main)
+        if first + 1 <= last:
+            pend[first + 1] = host_part(first + 1)
         for i, k in enumerate(ks):
-            b = k % 2
-            ncow, lens = pend
-            copy_s.wait_event(comp_done[b])      # compute k-2 has read device set b
-            with torch.cuda.stream(copy_s):
-                g_h2d[k].replay()
-                h2d_done[b].record(copy_s)
-            main.wait_event(h2d_done[b])
-            main.wait_event(out_done[b])         # D2H k-2 has read out of set b
-            g_comp[k].replay()
-            comp_done[b].record(main)
-            out_s.wait_event(comp_done[b])
-            with torch.cuda.stream(out_s):
-                pins[b]["out"].copy_(devs[b]["out"], non_blocking=True)
-                out_done[b].record(out_s)
+            ncow, lens = pend.pop(k)
+            if ncow:
+                cow_copies(k, ncow)
+            graphs[i].replay()                   # step k, step k + 1's H2D, step k - 1's D2H
+            done[i].record(main)
             if count:                            # counted after the timed region
-                seen.append((k, b, ncow, lens.clone()))
-            if i + 1 < len(ks):
-                nb = ks[i + 1] % 2
-                h2d_done[nb].synchronize()       # step k-1's copies have read pinned set nb
-                pend = host_part(ks[i + 1], nb)
-            if i >= 1:
-                out_done[(k - 1) % 2].synchronize()   # step k-1's out is in host memory
-        out_done[ks[-1] % 2].synchronize()
+                seen.append((k, ncow, lens.clone()))
+            if k + 2 <= last:
+                # step k's H2D (graph k - 1, or the copies before the first
+                # graph) has read pinned set k % 2, which step k + 2 refills
+                (done[i - 1] if i >= 1 else first_in).synchronize()
+                pend[k + 2] = host_part(k + 2)
+        d2h(last)
+        torch.cuda.synchronize()                 # every step's out is in host memory
+        t1 = time.perf_counter()
+        return t1 - t0
 
     seen = []
+    stats = dict(bytes=0, h2d=0, d2h=0)
     run(list(range(args.warmup)), False)
     torch.cuda.synchronize()
     barrier(world)
-    t0 = time.perf_counter()
-    run(list(range(args.warmup, n)), True)
-    t1 = time.perf_counter()
+    dt_s = run(list(range(args.warmup, n)), True)
     assert int(sess.err.item()) == 0, f"e2e: device error flag {int(sess.err.item())}"
-    del g_h2d, g_comp
-    for k, b, ncow, lens in seen:
+    for k, ncow, lens in seen:
         stats["bytes"] += sess.bytes_of(lens.tolist())
         stats["h2d"] = (sum(t.numel() * t.element_size() for t in
-                            (qs[k], kk[k], vv[k], pins[b]["slots"], pins[b]["tab"],
-                             pins[b]["lens"])) + ncow * 16)
-        stats["d2h"] = pins[b]["out"].numel() * pins[b]["out"].element_size()
-    total_bytes, span_ms, gbs = aggregate(stats["bytes"], (t1 - t0) * 1e3, world)
+                            (qs[k], kk[k], vv[k], pins[k % 2]["slots"], pins[k % 2]["tab"],
+                             pins[k % 2]["lens"])) + ncow * 16)
+        stats["d2h"] = pins[k % 2]["out"].numel() * pins[k % 2]["out"].element_size()
+    total_bytes, span_ms, gbs = aggregate(stats["bytes"], dt_s * 1e3, world)
     K = n - args.warmup
     return {"value": round(gbs, 1), "unit": "GB/s",
             "h2d_bytes_per_step": stats["h2d"], "d2h_bytes_per_step": stats["d2h"],
             "ms_per_step": round(span_ms / K, 4),
-            "device_part": "cuda graphs (copy and compute stages), pipelined one step ahead"}
+            "device_part": "one cuda graph per step (its compute, the next step's H2D, the "
+                           "previous step's D2H), host prepared two steps ahead"}
 
 
 # ----------------------------------------------------------------------------- the oracle on the host

@@ -53,6 +53,22 @@ def test_prefill_matches_oracle(dtype, hq, hkv, d, bs):
     check_close(got, ref, dtype, f"prefill {dtype} {hq}/{hkv} d{d} bs{bs}")
 
 
+MANY_LENS = [900, 700, 1200, 333, 1024, 65, 1500, 257]
+MANY_QLENS = [900, 300, 600, 333, 512, 65, 700, 257]
+
+
+@pytest.mark.parametrize("dtype,hq,hkv,d,bs", [("f16", 8, 8, 64, 8), ("bf16", 16, 8, 128, 32),
+                                               ("bf16", 64, 8, 64, 16)])
+def test_several_items_per_cta(dtype, hq, hkv, d, bs):
+    """More pairs of query tiles than SMs (256, 512 and 1856 items), so the
+    persistent CTAs take several items each, across item boundaries of every
+    kind (one-tile items, short and long ones), at block sizes 8-32 and both
+    head dims."""
+    b = workloads.prefill_custom(dtype, MANY_LENS, MANY_QLENS, hq, hkv, d, bs, seed=hq + 7 * bs + d)
+    got, ref, _ = _run(b)
+    check_close(got, ref, dtype, f"prefill items {dtype} {hq}/{hkv} d{d} bs{bs}")
+
+
 def test_unwritten_slots_never_leak():
     """Every cache element no token wrote is NaN; keys past a chunk's range
     and the tail of its last block must still get weight 0 and a finite V."""

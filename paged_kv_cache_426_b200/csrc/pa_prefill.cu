@@ -26,9 +26,9 @@
 // warpgroup (8-11) hands registers to the softmax warps.  The two softmax
 // groups run side by side (two warps per SM sub-partition); S (and the P
 // written over it) is double-buffered in tensor memory per tile, so the tensor
-// core computes the next stage's S while the softmax works.  With no P in
-// shared memory the K/V ring holds five 64-key stages, more than the copy
-// latency needs.  The row maximum m is moved lazily: only when a stage
+// core computes the next stage's S while the softmax works.  The K/V ring
+// holds four 64-key stages, enough to cover the copy latency (five were no
+// faster).  The row maximum m is moved lazily: only when a stage
 // exceeds it by 2^8 is O rescaled in tensor memory.  Keys past the row's
 // position get weight 0; keys past the item's key range or in a block whose
 // table entry is bad also get their V rows zeroed in shared memory (the
@@ -59,7 +59,7 @@ constexpr int PF_TILES = 2;        // query tiles per CTA
 constexpr int PF_THREADS = 384;
 constexpr int PF_REGS_HIGH = 208, PF_REGS_LOW = 80;
 static_assert(256 * PF_REGS_HIGH + 128 * PF_REGS_LOW <= PF_THREADS * 168, "register split");
-constexpr int PF_MAX_STAGES = 6;
+constexpr int PF_MAX_STAGES = 4;
 constexpr float kPfRescaleLog2 = 8.f;
 constexpr uint32_t PF_FULL = 0xffffffffu;
 

@@ -7,7 +7,9 @@
 A step is one decode step of the workload's batch: copy-on-write block
 copies (when the host manager reports any), the cache write of the step's new
 tokens, and decode attention over every sequence (the decode kernel plus the
-split-K merge).  The host metadata of every step (slot mapping, copy pairs,
+split-K merge).  The cache write is part of the pa_decode call (its
+key_new / value_new / slot_mapping option): the tensor-core decode kernel
+stores each new token just before it copies the block that holds it.  The host metadata of every step (slot mapping, copy pairs,
 block tables, lengths) is produced by the library's C++ manager before the
 timed region and sits in HBM with the queries and new K/V rows.  Each step is
 captured once as a CUDA graph from the public calls and replayed; CUDA events
@@ -462,28 +464,31 @@ class Session:
                 v=w.step_v[k].to(self.dev)))
         return plan
 
-    def write(self, st):
-        """Copy-on-write copies (when the manager reported any) and the cache
-        write of one step.  Returns the launches."""
-        pa = self.pa
-        n = 0
-        if st["cow"] is not None:
-            pa.pa_copy_blocks(self.kc, self.vc, st["cow"], err_flag=self.err)
-            n += 1
-        pa.pa_reshape_and_cache(st["k"], st["v"], self.kc, self.vc, st["slots"], err_flag=self.err)
-        return n + 1
+    def cow(self, st):
+        """Copy-on-write copies of one step, when the manager reported any.
+        Returns the launches."""
+        if st["cow"] is None:
+            return 0
+        self.pa.pa_copy_blocks(self.kc, self.vc, st["cow"], err_flag=self.err)
+        return 1
 
-    def decode(self, st, out):
-        """One pa_decode call: the decode kernel, plus the split-K merge kernel
-        when a sequence can span several partitions.  Returns the launches."""
+    def decode(self, st, out, write=False):
+        """One pa_decode call, with the step's cache write when ``write``: the
+        decode kernel (which writes the new tokens itself on the tensor-core
+        engine; the CUDA-core engine gets a write launch first), plus the
+        split-K merge kernel unless the decode kernel merges the splits
+        itself.  Returns the launches."""
         self.pa.pa_decode(out, st["q"], self.kc, self.vc, st["tab"], st["lens"], self.max_len,
                           self.w.scale, partition_size=self.P, workspace=self.ws,
-                          err_flag=self.err, engine=self.engine)
+                          err_flag=self.err, engine=self.engine,
+                          write=(st["k"], st["v"], st["slots"]) if write else None)
         n_pmax = -(-self.max_len // self.P) if self.P > 0 else 1
-        return 2 if n_pmax > 1 else 1
+        tensor = self.w.dtype != "f32" and self.engine not in ("core", 1)
+        merged_inside = tensor and n_pmax <= 4
+        return 1 + (n_pmax > 1 and not merged_inside) + (write and not tensor)
 
     def step(self, st, out):
-        return self.write(st) + self.decode(st, out)
+        return self.cow(st) + self.decode(st, out, write=True)
 
     def bytes_of(self, lens):
         w = self.w
@@ -583,7 +588,8 @@ L2_BYTES = 126 << 20
 def measure(name, args, dev, n_timed, world, engine="auto", flush_buf=None, warm_too=False,
             sampler=None):
     """Device-timed steps of one workload.  Every step (copy-on-write copies,
-    cache write, decode + merge) and, separately, its decode call alone are
+    decode with the step's cache write, merge) and, separately, its decode
+    call alone (no write) are
     captured as CUDA graphs and replayed in step order with CUDA events around
     each replay.  Returns the numbers and the session (for the end-to-end
     leg)."""
@@ -778,9 +784,9 @@ def run_ours(args, rank, world, local):
 def run_e2e(sess, w, args, world):
     """Same metric through the public API with host buffers, every step: the
     live C++ manager's appends and block tables (host), the step's H2D copies
-    from pinned buffers, copy-on-write copies, cache write, decode and the D2H
-    of out.  Steps are pipelined the way a serving loop runs them: step k is
-    one CUDA graph of three branches, step k's cache write and decode, the H2D
+    from pinned buffers, copy-on-write copies, decode with the cache write, and
+    the D2H of out.  Steps are pipelined the way a serving loop runs them: step
+    k is one CUDA graph of three branches, step k's decode (and write), the H2D
     copies of step k + 1's inputs into the other device set, and the D2H of
     step k - 1's out, captured beforehand from the same public calls; while it
     runs, the host prepares step k + 2 (manager calls into the pinned set step
@@ -834,10 +840,9 @@ def run_e2e(sess, w, args, world):
 
     def compute(k):
         D = devs[k % 2]
-        pa.pa_reshape_and_cache(D["k"], D["v"], sess.kc, sess.vc, D["slots"], err_flag=sess.err)
         pa.pa_decode(D["out"], D["q"], sess.kc, sess.vc, D["tab"], D["lens"], sess.max_len,
                      w.scale, partition_size=sess.P, workspace=sess.ws, err_flag=sess.err,
-                     engine=sess.engine)
+                     engine=sess.engine, write=(D["k"], D["v"], D["slots"]))
 
     def host_part(k):
         pin = pins[k % 2]

@@ -105,7 +105,7 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * Long contexts are split into partitions of `partition_size` tokens
  * (a positive multiple of 16; 0 = one partition per sequence) whose partial
  * results are merged with their log-sum-exp weights.  With the tensor-core
- * engine and ceil(max_context_len / partition_size) <= 16 the work unit that
+ * engine and ceil(max_context_len / partition_size) <= 4 the work unit that
  * completes a split sequence merges it inside the decode kernel (one launch
  * per call); otherwise, when ceil(max_context_len / partition_size) > 1, a
  * second kernel on the same stream merges (two launches).
@@ -173,8 +173,11 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
 
 /* pa_decode_ex - pa_decode with per-call options; options = NULL is exactly
  * pa_decode.  The options apply to this call only (no process-wide state).
- *   struct_size  sizeof(pa_decode_options) as the caller was compiled (a
- *                smaller value returns PA_ERR_INVALID)
+ *   struct_size  sizeof(pa_decode_options) as the caller was compiled; at
+ *                least the size of the first three fields (a smaller value
+ *                returns PA_ERR_INVALID).  Fields past struct_size read as
+ *                zero / NULL, so callers built against an older header keep
+ *                working.
  *   engine       PA_ENGINE_AUTO (pa_decode's choice): tcgen05 tensor-core
  *                MMAs with accumulators in tensor memory for f16/bf16 (the
  *                CUDA-core engine when its shared-memory ring does not fit,
@@ -189,12 +192,39 @@ int pa_decode_static(void* out, const void* query, const void* key_cache,
  *                the 2 s wait limit, set PA_DEV_TIMEOUT in err_flag and
  *                return; the context and the workspace stay usable.  No GPU
  *                fault is involved.  The pages have no counterpart.
+ *   key_new, value_new, slot_mapping  the step's cache write, done by this
+ *                call ([VEL] 작동 예시 / [119] 해법: the new token's K/V goes
+ *                into the slot its table assigns, then attention reads it).
+ *                All NULL (the default): no write.  All set: the result is
+ *                that of pa_reshape_and_cache(key_new, value_new, ...,
+ *                slot_mapping, num_tokens = num_seqs) on the same stream
+ *                followed by this decode, with one difference in launches:
+ *                the tensor-core engine writes each sequence's token from
+ *                inside the decode kernel, just before the copy of the block
+ *                that holds it (one launch fewer per step); the CUDA-core
+ *                engine launches the cache write first.
+ *                  key_new, value_new  device [num_seqs][num_kv_heads][head_dim]
+ *                    dtype, contiguous, 16-B aligned: row s is sequence s's
+ *                    new token (the one at position context_lens[s] - 1)
+ *                  slot_mapping  device int64 [num_seqs]: slot_mapping[s] <
+ *                    0 skips sequence s's write; otherwise it must be the
+ *                    slot of position context_lens[s] - 1 through
+ *                    block_tables[s], else PA_DEV_BAD_SLOT is set and that
+ *                    token is not written (any engine).
+ *                The block holding a written slot must not be read by another
+ *                sequence of this call (a block manager's copy-on-write
+ *                before the write guarantees it); otherwise what that other
+ *                sequence reads of the written row is unspecified.
+ *                Only some of the three set: PA_ERR_INVALID.
  * Out-of-range option values return PA_ERR_INVALID before any launch. */
 enum { PA_ENGINE_AUTO = 0, PA_ENGINE_CUDA_CORE = 1, PA_ENGINE_TENSOR = 2 };
 typedef struct pa_decode_options {
     int struct_size;
     int engine;
     int test_withhold_stage;
+    const void* key_new;
+    const void* value_new;
+    const int64_t* slot_mapping;
 } pa_decode_options;
 int pa_decode_ex(void* out, const void* query, const void* key_cache,
                  const void* value_cache, const int32_t* block_tables,

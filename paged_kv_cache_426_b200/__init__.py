@@ -159,7 +159,8 @@ def alloc_workspace(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_l
 
 class pa_decode_options(C.Structure):
     """Per-call options of pa_decode_ex (include/pa.h)."""
-    _fields_ = [("struct_size", C.c_int), ("engine", C.c_int), ("test_withhold_stage", C.c_int)]
+    _fields_ = [("struct_size", C.c_int), ("engine", C.c_int), ("test_withhold_stage", C.c_int),
+                ("key_new", C.c_void_p), ("value_new", C.c_void_p), ("slot_mapping", C.c_void_p)]
 
 
 ENGINES = {"auto": PA_ENGINE_AUTO, "core": PA_ENGINE_CUDA_CORE, "tensor": PA_ENGINE_TENSOR}
@@ -167,12 +168,16 @@ ENGINES = {"auto": PA_ENGINE_AUTO, "core": PA_ENGINE_CUDA_CORE, "tensor": PA_ENG
 
 def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len,
               scale, *, partition_size=0, workspace=None, err_flag=None, stream=None,
-              engine=None, test_withhold_stage=-1):
+              engine=None, test_withhold_stage=-1, write=None):
     """out/query [S, Hq, D]; caches [NB, Hkv, bs, D]; block_tables int32 [S, max_blocks];
     context_lens int32 [S].  ``engine`` ("auto", "core", "tensor" or a PA_ENGINE_*
-    value) and ``test_withhold_stage`` are per-call options (pa_decode_ex);
-    with neither given this is the plain pa_decode call."""
+    value), ``test_withhold_stage`` and ``write`` = (key_new, value_new,
+    slot_mapping) - the step's cache write, [S, Hkv, D] twice and int64 [S],
+    done by this call - are per-call options (pa_decode_ex); with none given
+    this is the plain pa_decode call."""
     _cuda(out, query, key_cache, value_cache, block_tables, context_lens, workspace, err_flag)
+    if write is not None:
+        _cuda(*write)
     S, hq, d = query.shape
     NB, hkv, bs, _ = key_cache.shape
     if workspace is None:
@@ -182,12 +187,14 @@ def pa_decode(out, query, key_cache, value_cache, block_tables, context_lens, ma
             NB, float(scale), int(partition_size), _ptr(workspace),
             workspace.numel() * workspace.element_size(), pa_dtype(query), _ptr(err_flag),
             _stream(stream))
-    if engine is None and test_withhold_stage == -1:
+    if engine is None and test_withhold_stage == -1 and write is None:
         check(lib.pa_decode(*args), "pa_decode")
         return
     eng = ENGINES[engine] if isinstance(engine, str) else (PA_ENGINE_AUTO if engine is None
                                                             else int(engine))
-    opts = pa_decode_options(C.sizeof(pa_decode_options), eng, int(test_withhold_stage))
+    kn, vn, sm = write if write is not None else (None, None, None)
+    opts = pa_decode_options(C.sizeof(pa_decode_options), eng, int(test_withhold_stage),
+                             _ptr(kn), _ptr(vn), _ptr(sm))
     check(lib.pa_decode_ex(*args, C.byref(opts)), "pa_decode_ex")
 
 

@@ -48,6 +48,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 
@@ -93,6 +94,14 @@ struct DecodeParams {
     int* split_cnt;    // [S*Hkv] partitions of a split (sequence, KV head) finished so far
     int fused_merge;   // the unit finishing a split last merges it (no merge kernel)
     int32_t* err;
+    // the step's cache write done by the decode call (wslot null: none): row
+    // s of wk / wv (16-byte pieces, [S][Hkv][D]) goes to slot wslot[s], which
+    // must be the slot of position lens[s] - 1; kc / vc are the caches
+    const uint4* wk;
+    const uint4* wv;
+    const int64_t* wslot;
+    uint4* kc;
+    uint4* vc;
 };
 
 // Shared-memory layout (dynamic, 1024-byte aligned base).  Every pipeline has
@@ -146,6 +155,54 @@ __device__ __forceinline__ int clamp_len(int L, const DecodeParams& p) {
 }
 
 __device__ __forceinline__ int n_parts(int L, int P) { return max(1, ceil_div(L, P)); }
+
+// Orders this thread's generic-proxy global writes before later async-proxy
+// (TMA) accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// The step's new token of sequence s: whether wslot[s] = `slot` is to be
+// written, i.e. non-negative and equal to the slot the table gives position
+// pos = L - 1 (block bl, row pos % bs).  A mismatch sets PA_DEV_BAD_SLOT when
+// `report`; a negative slot is a skipped write, no error.
+__device__ __forceinline__ bool new_token_slot_ok(const DecodeParams& p, int64_t slot, int pos,
+                                                  int bl, bool report) {
+    if (slot < 0) return false;
+    const bool ok = pos >= 0 && bl >= 0 && bl < p.NB &&
+                    slot == (int64_t)bl * p.bs + (pos & (p.bs - 1));
+    if (!ok && report) set_err(p.err, PA_DEV_BAD_SLOT);
+    return ok;
+}
+
+// Copies KV head j's K and V rows of sequence s's new token into block bl,
+// row pos % bs: 2 * nv 16-byte pieces, this thread's from i0 in steps of di.
+__device__ __forceinline__ void put_new_token(const DecodeParams& p, int s, int j, int pos, int bl,
+                                              int nv, int i0, int di) {
+    const size_t src = ((size_t)s * p.Hkv + j) * nv;
+    const size_t dst = (((size_t)bl * p.Hkv + j) * p.bs + (pos & (p.bs - 1))) * nv;
+    for (int e = i0; e < 2 * nv; e += di) {
+        const bool isv = e >= nv;
+        const int x = isv ? e - nv : e;
+        (isv ? p.vc : p.kc)[dst + x] = __ldg((isv ? p.wv : p.wk) + src + x);
+    }
+}
+
+// The step's cache write for engines that do not do it inside the decode
+// kernel: one CTA per sequence, every KV head, with the same slot check.  A
+// programmatic dependent of the kernel before it; the decode after it waits
+// for its completion.
+__global__ void __launch_bounds__(128) new_token_write_kernel(DecodeParams p, int nv) {
+    grid_dependency_wait();
+    const int s = blockIdx.x;
+    const int64_t slot = __ldg(p.wslot + s);
+    if (slot < 0) return;
+    const int L = clamp_len(__ldg(p.lens + s), p);
+    const int pos = L - 1;
+    const int bl = pos >= 0 ? __ldg(p.tables + (size_t)s * p.mbps + (pos >> p.bs_log2)) : -1;
+    if (!new_token_slot_ok(p, slot, pos, bl, threadIdx.x == 0)) return;
+    for (int j = 0; j < p.Hkv; ++j) put_new_token(p, s, j, pos, bl, nv, threadIdx.x, blockDim.x);
+}
 
 // Bounded wait that also gives up as soon as another warp has given up.
 // mbar_try_wait sleeps until the phase completes (suspend hint), so the abort
@@ -1081,6 +1138,9 @@ __device__ void schedule_units(const DecodeParams& p, int* lens_s, int* preF, in
     for (int k = beg; k < end; ++k) {
         const int L = clamp_len(__ldg(p.lens + k), p);
         lens_s[k] = L;
+        // a sequence with no tokens has no position for a new one
+        if (p.wslot != nullptr && L == 0 && blockIdx.x == 0 && __ldg(p.wslot + k) >= 0)
+            set_err(p.err, PA_DEV_BAD_SLOT);
         full += n_parts(L, p.P) - 1;
         const int b = bucket(L);
 #pragma unroll
@@ -1160,12 +1220,30 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
     const int PR = bs >= 16 ? 16 : bs;                // rows per piece
     const int NPC = TTOK / PR;                         // pieces per stage
     const int nops = NPC * 2 * LY::NBOX;               // <= 64
+    constexpr int NV = LY::ROWB / 16;                  // 16-byte pieces of a K or V row
+    static_assert(2 * NV <= 32, "one piece of the new token's K and V rows per lane");
     struct Plan {
         int u, s, j, i, t0, t1, nst, n_p, nblk;
         const int32_t* trow;
         int ids_a, ids_b;
+        bool wr;           // the step's new token falls in this unit (its last partition)
+        bool wld;          // ... and its slot, block and row pieces are loaded
+        int wbl;           // block of position L - 1 through the table
+        long long wsl;     // slot_mapping entry of the sequence
+        uint4 wpc;         // this lane's piece: K row (lanes < NV), V row (NV <= lanes < 2 NV)
     };
-    auto prepare = [&](int u) {
+    // The new token's slot, block and row pieces, loaded into registers a unit
+    // ahead (only after the dependency wait: the inputs may come from the
+    // kernel before this one).
+    auto load_write = [&](Plan& q) {
+        const int pos = q.t1 - 1;
+        q.wsl = __ldg(p.wslot + q.s);
+        q.wbl = __ldg(q.trow + ((pos >> bsl) - (q.t0 >> bsl)));
+        if (lane < 2 * NV)
+            q.wpc = __ldg((lane < NV ? p.wk : p.wv) + ((size_t)q.s * p.Hkv + q.j) * NV + lane % NV);
+        q.wld = true;
+    };
+    auto prepare = [&](int u, bool dep_done) {
         Plan q{};
         q.u = u;
         if (u >= U) return q;
@@ -1195,6 +1273,8 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
         q.trow = p.tables + (size_t)q.s * p.mbps + b0;
         q.ids_a = (lane < q.nblk) ? __ldg(q.trow + lane) : -1;
         q.ids_b = (lane + 32 < q.nblk) ? __ldg(q.trow + 32 + lane) : -1;
+        q.wr = p.wslot != nullptr && q.i == q.n_p - 1 && q.nst > 0;
+        if (q.wr && dep_done) load_write(q);
         return q;
     };
     // Latency hiding at unit boundaries: lane 0 holds the tickets of the two
@@ -1205,7 +1285,7 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
     // reads included - before the dependency wait; later units come from the
     // ticket counter, which hands out gridDim.x onwards.
     int gstage = 0, st = 0, round = 0, ucount = 0, t1 = 0, t2 = 0;
-    Plan cur = prepare((int)blockIdx.x);
+    Plan cur = prepare((int)blockIdx.x, false);
     // The kernel before this one has completed and its writes are visible:
     // the cache may be read, and the scheduler ticket is free (a decode call
     // just before on the same workspace has reset it).
@@ -1246,26 +1326,43 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
         Plan nxt{};
         bool have_next = false;
         auto next_plan = [&]() {            // after the unit's first stage is issued
-            nxt = prepare(__shfl_sync(FULL, t1, 0));
+            nxt = prepare(__shfl_sync(FULL, t1, 0), true);
             have_next = true;
             if (lane == 0) {
                 t1 = t2;
                 t2 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
             }
         };
+        if (cur.wr) {
+            // The step's new token (position L - 1, in this unit's last
+            // stage) goes into the cache now, with the values loaded a unit
+            // ahead; the fence before the last stage's copies orders the
+            // stores before them.  Only this unit reads that row: partitions
+            // start at multiples of 16 tokens and pieces are at most 16 rows.
+            if (!cur.wld) load_write(cur);        // a CTA's first unit
+            const int pos = cur.t1 - 1;
+            if (new_token_slot_ok(p, cur.wsl, pos, cur.wbl, lane == 0) && lane < 2 * NV)
+                (lane < NV ? p.kc : p.vc)[(((size_t)cur.wbl * p.Hkv + cur.j) * bs + (pos & (bs - 1))) * NV +
+                                          lane % NV] = cur.wpc;
+        }
         int win = 0;
         const int b0 = cur.t0 >> bsl;
         for (int c = 0; c < cur.nst; ++c) {
             const int tok0 = cur.t0 + c * TTOK;
-            if (round > 0) {
-                bool w = true;
-                if (lane == 0) w = wait_or_abort(empty + st, (round - 1) & 1, abort_flag, p.err);
-                if (!__shfl_sync(FULL, w, 0)) { ok = false; break; }
-            }
             while ((tok0 >> bsl) - b0 - win >= 32) {      // keep the stage's blocks in the window
                 win += 32;
                 cur.ids_a = cur.ids_b;
                 cur.ids_b = (lane + win + 32 < cur.nblk) ? __ldg(cur.trow + win + 32 + lane) : -1;
+            }
+            if (cur.wr && c == cur.nst - 1) {
+                fence_proxy_async_global();               // the new token's stores before
+                __syncwarp();                             // this stage's copies
+                fence_proxy_async_global();
+            }
+            if (round > 0) {
+                bool w = true;
+                if (lane == 0) w = wait_or_abort(empty + st, (round - 1) & 1, abort_flag, p.err);
+                if (!__shfl_sync(FULL, w, 0)) { ok = false; break; }
             }
             int blk[2], tok[2];
             bool live[2];
@@ -2103,7 +2200,7 @@ int decode_launch(void* out, const void* query, const void* key_cache, const voi
                   int max_context_len, int num_seqs, int num_q_heads, int num_kv_heads,
                   int head_dim, int block_size, int num_blocks, float scale, int partition_size,
                   void* workspace, pa_dtype dtype, int32_t* err_flag, void* stream, int engine,
-                  int hold_stage) {
+                  int hold_stage, const void* wkey, const void* wval, const int64_t* wslot) {
     const int G = num_q_heads / num_kv_heads;
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
     DevInfo di;
@@ -2142,6 +2239,12 @@ int decode_launch(void* out, const void* query, const void* key_cache, const voi
     p.fused_merge = 0;       // set by the engine that takes it
     p.err = err_flag;
     p.hold_stage = hold_stage;
+    p.wslot = wslot;
+    p.wk = wslot ? static_cast<const uint4*>(wkey) : nullptr;
+    p.wv = wslot ? static_cast<const uint4*>(wval) : nullptr;
+    // the caches are written only with the step's cache write requested
+    p.kc = static_cast<uint4*>(const_cast<void*>(key_cache));
+    p.vc = static_cast<uint4*>(const_cast<void*>(value_cache));
 
     const int64_t units_ub = (int64_t)num_seqs * num_kv_heads * n_pmax;
     L.units_ub = units_ub;
@@ -2161,15 +2264,25 @@ int decode_launch(void* out, const void* query, const void* key_cache, const voi
         }
         return (int)PA_ERR_INVALID;
     };
+    // the CUDA-core engine gets the step's cache write as a launch before it
+    auto run_core = [&]() {
+        if (wslot) {
+            const int nv = head_dim * (dtype == PA_F32 ? 4 : 2) / 16;
+            const int w = launch_dependent(new_token_write_kernel, dim3((unsigned)num_seqs), 128, 0,
+                                           L.stream, L.p, nv);
+            if (w != PA_OK) return w;
+        }
+        return run(false);
+    };
     if (tensor) {
         st = maps.get(&L.qmap, query, dtype, head_dim, (int64_t)num_seqs * num_q_heads, G);
         if (st != PA_OK) return st;
         st = run(true);
         // by default, shapes whose stage ring does not fit (very many
-        // sequences) go to the CUDA-core engine
-        if (st == PA_ERR_UNSUPPORTED && engine == PA_ENGINE_AUTO) st = run(false);
+        // sequences) go to the CUDA-core engine (nothing was launched)
+        if (st == PA_ERR_UNSUPPORTED && engine == PA_ENGINE_AUTO) st = run_core();
     } else {
-        st = run(false);
+        st = run_core();
     }
     // sequences split into several partitions are merged by a second launch,
     // unless the decode kernel merged them itself
@@ -2207,11 +2320,26 @@ int pa_decode_ex(void* out, const void* query, const void* key_cache, const void
                  void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* err_flag,
                  void* stream, const pa_decode_options* options) {
     int engine = PA_ENGINE_AUTO, hold = -1;
+    const void* wkey = nullptr;
+    const void* wval = nullptr;
+    const int64_t* wslot = nullptr;
     if (options) {
-        if (options->struct_size < (int)sizeof(pa_decode_options)) return PA_ERR_INVALID;
+        // fields past struct_size (a caller built against an older header) read as unset
+        const int size = options->struct_size;
+        auto has = [size](size_t off, size_t len) { return (size_t)size >= off + len; };
+        if (!has(offsetof(pa_decode_options, test_withhold_stage), sizeof(int))) return PA_ERR_INVALID;
         engine = options->engine;
         hold = options->test_withhold_stage;
         if (engine < PA_ENGINE_AUTO || engine > PA_ENGINE_TENSOR || hold < -1) return PA_ERR_INVALID;
+        if (has(offsetof(pa_decode_options, key_new), sizeof(void*))) wkey = options->key_new;
+        if (has(offsetof(pa_decode_options, value_new), sizeof(void*))) wval = options->value_new;
+        if (has(offsetof(pa_decode_options, slot_mapping), sizeof(void*)))
+            wslot = options->slot_mapping;
+        const int nset = (wkey != nullptr) + (wval != nullptr) + (wslot != nullptr);
+        if (nset != 0 && nset != 3) return PA_ERR_INVALID;
+        if (nset == 3 && (!aligned16(wkey) || !aligned16(wval) ||
+                          (reinterpret_cast<uintptr_t>(wslot) & 7)))
+            return PA_ERR_INVALID;
     }
     if (num_seqs == 0) return PA_OK;
     int st = validate_args(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
@@ -2224,7 +2352,7 @@ int pa_decode_ex(void* out, const void* query, const void* key_cache, const void
     return decode_launch(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                          context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
                          head_dim, block_size, num_blocks, scale, partition_size, workspace, dtype,
-                         err_flag, stream, engine, hold);
+                         err_flag, stream, engine, hold, wkey, wval, wslot);
 }
 
 int pa_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
@@ -2335,5 +2463,5 @@ extern "C" int pa_decode_static(void* out, const void* query, const void* key_ca
     return decode_launch(out, query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                          context_lens, max_context_len, num_seqs, num_q_heads, num_kv_heads,
                          head_dim, block_size, num_blocks, scale, partition_size, ws, dtype,
-                         err_flag, stream, PA_ENGINE_AUTO, -1);
+                         err_flag, stream, PA_ENGINE_AUTO, -1, nullptr, nullptr, nullptr);
 }

@@ -56,9 +56,10 @@ class CudaPathRun:
     """The CUDA path driven through a workload's script."""
 
     def __init__(self, w, rec: oracle.OracleRun, *, partition_size=None, device="cuda",
-                 max_blocks=None, engine=None):
+                 max_blocks=None, engine=None, fused=False):
         self.w = w
         self.engine = engine          # None: plain pa_decode; else a per-call engine option
+        self.fused = fused            # the step's cache write done by the pa_decode call
         self.dev = device
         self.P = w.partition_size if partition_size is None else partition_size
         self.mb = max_blocks if max_blocks is not None else oracle.max_blocks_needed(w)
@@ -109,13 +110,14 @@ class CudaPathRun:
         dev = self.dev
         if cow.shape[0]:
             pa.pa_copy_blocks(self.kc, self.vc, cow.to(dev), err_flag=self.err)
-        pa.pa_reshape_and_cache(w.step_k[k].to(dev), w.step_v[k].to(dev), self.kc, self.vc,
-                                slots.to(dev), err_flag=self.err)
+        new = (w.step_k[k].to(dev), w.step_v[k].to(dev), slots.to(dev))
+        if not self.fused:
+            pa.pa_reshape_and_cache(*new[:2], self.kc, self.vc, new[2], err_flag=self.err)
         q = w.step_q[k].to(dev)
         out = torch.empty_like(q)
         pa.pa_decode(out, q, self.kc, self.vc, tab.to(dev), lens.to(dev), self.max_len, w.scale,
                      partition_size=self.P, workspace=self.ws, err_flag=self.err,
-                     engine=self.engine)
+                     engine=self.engine, write=new if self.fused else None)
         torch.cuda.synchronize()
         assert int(self.err.item()) == 0, f"err_flag {int(self.err.item())}"
         return out

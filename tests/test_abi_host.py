@@ -83,11 +83,20 @@ def test_decode_options_are_per_call():
     assert call(None) == pa.PA_ERR_UNSUPPORTED
     assert call(pa.pa_decode_options(size, pa.PA_ENGINE_TENSOR, -1)) == pa.PA_ERR_UNSUPPORTED
     assert call(pa.pa_decode_options(size, pa.PA_ENGINE_CUDA_CORE, 3)) == pa.PA_ERR_UNSUPPORTED
+    # a caller built against the first three fields only: the rest read as unset
+    assert call(pa.pa_decode_options(12, 0, -1, 1, 2, 3)) == pa.PA_ERR_UNSUPPORTED
+    # the step's cache write: all three pointers, 16-B aligned rows, 8-B aligned slots
+    g = 1 << 21
+    assert call(pa.pa_decode_options(size, 0, -1, f, g, f)) == pa.PA_ERR_UNSUPPORTED
     # bad options are rejected first
-    assert call(pa.pa_decode_options(size - 4, 0, -1)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(8, 0, -1)) == pa.PA_ERR_INVALID
     assert call(pa.pa_decode_options(size, 3, -1)) == pa.PA_ERR_INVALID
     assert call(pa.pa_decode_options(size, -1, -1)) == pa.PA_ERR_INVALID
     assert call(pa.pa_decode_options(size, 0, -2)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 0, -1, f, None, f)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 0, -1, None, None, f)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 0, -1, f + 8, g, f)) == pa.PA_ERR_INVALID
+    assert call(pa.pa_decode_options(size, 0, -1, f, g, f + 4)) == pa.PA_ERR_INVALID
 
 
 def test_static_decode_checks_arguments_before_the_device():

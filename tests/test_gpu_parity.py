@@ -37,11 +37,11 @@ def engine(request):
     return request.param
 
 
-def run_full_compare(w, partition_size=None, steps=None, engine="auto"):
+def run_full_compare(w, partition_size=None, steps=None, engine="auto", fused=False):
     if engine == "tensor" and w.dtype == "f32":
         pytest.skip("the tensor-core engine takes 16-bit types")
     rec = oracle.run(w, keep_prefill_cache=True, steps=steps)
-    g = CudaPathRun(w, rec, partition_size=partition_size, engine=engine)
+    g = CudaPathRun(w, rec, partition_size=partition_size, engine=engine, fused=fused)
     g.replay_prefill()
     errs = []
     for k in range(len(rec.steps)):
@@ -385,7 +385,8 @@ FULL = [
 @pytest.mark.parametrize("name,kw", FULL, ids=[f[0] for f in FULL])
 def test_full_size(name, kw):
     """Full-size workload in the benchmark's launch configuration (its
-    partition size), every decode step.  Step 0, every 8th step and the last
+    partition size, the step's cache write done by the decode call), every
+    decode step.  Step 0, every 8th step and the last
     step are compared element by element (every sequence, query head and
     column) with the oracle's output computed from the cache as it stands at
     that step; the other steps on sampled (sequence, head) rows the oracle
@@ -394,7 +395,7 @@ def test_full_size(name, kw):
     n = w.num_steps
     full = {0, n - 1} | set(range(0, n, 8))
     rec = oracle.run(w, keep_prefill_cache=True, decode_steps=full)
-    g = CudaPathRun(w, rec)
+    g = CudaPathRun(w, rec, fused=True)
     g.replay_prefill()
     S, Hq = rec.steps[0].context_lens.shape[0], w.num_q_heads
     for k in range(len(rec.steps)):

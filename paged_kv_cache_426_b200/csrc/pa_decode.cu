@@ -190,10 +190,12 @@ __device__ __forceinline__ void put_new_token(const DecodeParams& p, int s, int 
 
 // The step's cache write for engines that do not do it inside the decode
 // kernel: one CTA per sequence, every KV head, with the same slot check.  A
-// programmatic dependent of the kernel before it; the decode after it waits
-// for its completion.
+// programmatic dependent of the kernel before it; it lets the decode after it
+// launch at once (it writes neither lengths nor tables), which waits for its
+// completion before reading the cache.
 __global__ void __launch_bounds__(128) new_token_write_kernel(DecodeParams p, int nv) {
     grid_dependency_wait();
+    launch_dependents();
     const int s = blockIdx.x;
     const int64_t slot = __ldg(p.wslot + s);
     if (slot < 0) return;

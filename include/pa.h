@@ -128,8 +128,11 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * that kernel has completed if that kernel lets dependents start early
  * (griddepcontrol.launch_dependents); everything else (queries, cache,
  * workspace, every write) waits for its completion.  Of this library's
- * kernels only pa_reshape_and_cache starts dependents early, and it writes
- * neither.
+ * kernels pa_reshape_and_cache and the tensor-core decode kernel let their
+ * dependents start early (the decode from its start, so the next step's
+ * decode sets up during this one's tail); none writes lengths or tables.
+ * A kernel launched after pa_decode with programmatic stream serialization
+ * must wait (griddepcontrol.wait) before it reads what the call writes.
  */
 int pa_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads,
                              int head_dim, int max_context_len,

@@ -1140,9 +1140,6 @@ __device__ void schedule_units(const DecodeParams& p, int* lens_s, int* preF, in
     for (int k = beg; k < end; ++k) {
         const int L = clamp_len(__ldg(p.lens + k), p);
         lens_s[k] = L;
-        // a sequence with no tokens has no position for a new one
-        if (p.wslot != nullptr && L == 0 && blockIdx.x == 0 && __ldg(p.wslot + k) >= 0)
-            set_err(p.err, PA_DEV_BAD_SLOT);
         full += n_parts(L, p.P) - 1;
         const int b = bucket(L);
 #pragma unroll
@@ -1295,6 +1292,12 @@ __device__ void producer_tc(const CUtensorMap* kmap, const CUtensorMap* vmap,
     if (lane == 0) {
         t1 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
         t2 = (int)gridDim.x + atomicAdd(&p.hdr->next_unit, 1);
+    }
+    if (p.wslot != nullptr) {
+        // a sequence with no tokens has no position for a new one (its slot
+        // is read only now: the inputs may come from the kernel before)
+        for (int k = (int)blockIdx.x * 32 + lane; k < p.S; k += (int)gridDim.x * 32)
+            if (lens_s[k] == 0 && __ldg(p.wslot + k) >= 0) set_err(p.err, PA_DEV_BAD_SLOT);
     }
     bool ok = true;
     while (ok) {
@@ -1488,12 +1491,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
-    // Launched as a programmatic dependent of the kernel before it (the cache
-    // write): the lengths may be read, the unit order computed and the first
-    // unit's block-table entries read while that kernel still runs (it writes
-    // only the cache); the scheduler ticket, the queries, the cache and every
-    // write wait for griddepcontrol.wait (in the producer before its first
-    // ticket and copy, in every other warp before its loop).
+    // The kernel after this one in the stream (the merge kernel, or the next
+    // step's decode) may be scheduled from now on: its CTAs take the SM slots
+    // this grid's CTAs free in its tail and do their own set-up there; they
+    // read nothing this kernel writes before their griddepcontrol.wait.
+    launch_dependents();
+    // Launched as a programmatic dependent of the kernel before it: the
+    // lengths may be read, the unit order computed and the first unit's
+    // block-table entries read while that kernel still runs (no kernel of
+    // this library writes lengths or tables); the scheduler ticket, the
+    // queries, the new tokens, the cache and every write wait for
+    // griddepcontrol.wait (in the producer before its first ticket and copy,
+    // in every other warp before its loop).
     schedule_units<TC_THREADS>(p, lens_s, preF, order, reinterpret_cast<int*>(smem + ly.sched()), wsum, tid);
     tc::fence_before();
     __syncthreads();

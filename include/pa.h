@@ -129,8 +129,9 @@ int pa_reshape_and_cache(const void* key, const void* value, void* key_cache,
  * (griddepcontrol.launch_dependents); everything else (queries, cache,
  * workspace, every write) waits for its completion.  Of this library's
  * kernels pa_reshape_and_cache and the tensor-core decode kernel let their
- * dependents start early (the decode from its start, so the next step's
- * decode sets up during this one's tail); none writes lengths or tables.
+ * dependents start early (the decode from its start when no merge kernel
+ * follows it, so the next step's decode sets up during this one's tail);
+ * none writes lengths or tables.
  * A kernel launched after pa_decode with programmatic stream serialization
  * must wait (griddepcontrol.wait) before it reads what the call writes.
  */

@@ -1491,11 +1491,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         prefetch_tensormap(&vmap);
         prefetch_tensormap(&qmap);
     }
-    // The kernel after this one in the stream (the merge kernel, or the next
-    // step's decode) may be scheduled from now on: its CTAs take the SM slots
-    // this grid's CTAs free in its tail and do their own set-up there; they
-    // read nothing this kernel writes before their griddepcontrol.wait.
-    launch_dependents();
+    // Without a merge launch after this kernel, the kernel after it in the
+    // stream (e.g. the next step's decode) may be scheduled from now on: its
+    // CTAs take the SM slots this grid's CTAs free in its tail and do their
+    // own set-up there; they read nothing this kernel writes before their
+    // griddepcontrol.wait.  (A merge kernel scheduled this early slowed the
+    // split batches: it is released at the end instead.)
+    const bool merge_follows = p.n_pmax > 1 && !p.fused_merge;
+    if (!merge_follows) launch_dependents();
     // Launched as a programmatic dependent of the kernel before it: the
     // lengths may be read, the unit order computed and the first unit's
     // block-table entries read while that kernel still runs (no kernel of
@@ -1870,7 +1873,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
 
     tc::fence_before();
     __syncthreads();
-    launch_dependents();                 // the merge kernel may be scheduled
+    if (merge_follows) launch_dependents();   // the merge kernel may be scheduled
     if (warp == 0) {
         tc::fence_after();
         tc::dealloc(tmem, LY::TM_COLS);

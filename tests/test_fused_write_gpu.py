@@ -155,3 +155,38 @@ def test_fused_write_slot_checks(engine, P):
     assert err.item() == 0
     assert torch.equal(kc.view(torch.int16), kref.view(torch.int16))
     assert torch.equal(vc.view(torch.int16), vref.view(torch.int16))
+
+
+@pytest.mark.parametrize("engine", ["core", "tensor"])
+def test_fused_write_zero_length_sequence(engine):
+    """A sequence with no tokens has no position for a new one: a
+    non-negative slot for it sets PA_DEV_BAD_SLOT (and nothing is written);
+    -1 is a skipped write, no error."""
+    d, hkv, G, bs, NB = 64, 1, 4, 16, 4
+    gen = torch.Generator().manual_seed(9)
+    kc = torch.randn(NB, hkv, bs, d, generator=gen).half().cuda()
+    vc = torch.randn(NB, hkv, bs, d, generator=gen).half().cuda()
+    q = torch.randn(2, hkv * G, d, generator=gen).half().cuda()
+    kn = torch.randn(2, hkv, d, generator=gen).half().cuda()
+    vn = torch.randn(2, hkv, d, generator=gen).half().cuda()
+    tab = torch.tensor([[0, 1], [-1, -1]], dtype=torch.int32, device="cuda")
+    lens = torch.tensor([17, 0], dtype=torch.int32, device="cuda")
+    ws = pa.alloc_workspace(2, hkv * G, hkv, d, 32, 16)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kref, vref = kc.clone(), vc.clone()
+    kref[1, :, 0] = kn[0]
+    vref[1, :, 0] = vn[0]
+    for slot1, want in ((-1, 0), (40, pa.PA_DEV_BAD_SLOT)):
+        kc.copy_(kref); vc.copy_(vref)
+        kc[1, :, 0] = 0
+        vc[1, :, 0] = 0
+        err.zero_()
+        slots = torch.tensor([16, slot1], dtype=torch.int64, device="cuda")
+        pa.pa_decode(out, q, kc, vc, tab, lens, 32, 0.125, partition_size=16, workspace=ws,
+                     err_flag=err, engine=engine, write=(kn, vn, slots))
+        torch.cuda.synchronize()
+        assert err.item() == want
+        assert torch.equal(kc.view(torch.int16), kref.view(torch.int16))
+        assert torch.equal(vc.view(torch.int16), vref.view(torch.int16))
+        assert not out[1].any()
